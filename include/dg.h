@@ -1,0 +1,204 @@
+/*
+ * dg.h -- C ABI of the B200 (sm_100a) fine-grained-scaled low-precision GEMM
+ * library:  D = C + A * B^T.
+ *
+ * Problem statement (sources are cited by page title and section):
+ *   - "DeepGEMM：统一高性能张量核心 GEMM 计算库编译与使用指南" (zhouruolin.cn),
+ *     section 五 "使用方法": the naming convention D = C + A @ B with the NT
+ *     layout (A [M,K] not transposed, B [N,K] transposed, both K-major); SM100
+ *     takes packed UE8M0 scale factors; grouping only along M with N and K
+ *     shared (contiguous layout for prefill / training forward, masked layout
+ *     for decoding); utilities set_num_sms / get_num_sms and
+ *     get_mk_alignment_for_contiguous_layout.
+ *   - "DeepSeek 开源第三弹 ... DeepGEMM" (app.myzaker.com), section "DeepGEMM":
+ *     FP8 with the fine-grained scaling of DeepSeek-V3 -- one scale per 1x128
+ *     row-group of A, one per 128x128 block of B; FP32 accumulation.
+ *   - "DeepSeek 发布 DeepGEMM 重大更新" (linlog.top), section "FP4 精度支持":
+ *     FP8 x FP4 GEMM, FP4 weights with UE8M0 scales packed 4 per int32.
+ *   - "DeepGEMM：FP8 GEMM 与 Mega-MoE" (charles2530.github.io), sections
+ *     "难点解释" (the scale layout is part of the interface) and "四、在 MoE
+ *     Serving 里的位置" (masked layout is CUDA-Graph friendly).
+ *
+ * Data types.  "e4m3": OCP FP8 E4M3FN codes, one byte each.  "e2m1": OCP FP4
+ * E2M1 codes packed two per byte along K, low nibble = even k.  "ue8m0": one
+ * byte e meaning 2^(e-127).  "bf16": bfloat16 bit patterns.  Accumulation is
+ * FP32; D is C + A*B^T rounded once to bf16 (round to nearest even).
+ *
+ * Packed scale layout ("sf words").  Scale codes of a matrix with R rows and
+ * G scale columns along K are packed into int32 words, 4 codes per word:
+ *     words[Q][ceil(R/128)][128],  Q = ceil(G/4);
+ *     the word of (row r, word-group q) is words[q][r/128][(r%32)*4 + (r%128)/32]
+ *     and its byte j (little endian) is the code of scale column 4q+j;
+ *     unused bytes hold 127.
+ * dg_pack_sf() produces it; dg_packed_sf_words() gives its length.  For e4m3
+ * operands the scale columns are the K/128 blocks (B's 128x128 block scales
+ * are expanded to one copy per row by dg_pack_sf with row_div = 128); for the
+ * e2m1 operand they are the K/32 groups.  Grouped operands store one packed
+ * block per group, back to back.
+ *
+ * Pointers.  Every matrix / scale / index pointer is a DEVICE pointer owned
+ * by the caller, 16-byte aligned, and may not alias an output (except C == D
+ * for in-place accumulation in the dense calls).  `stream` is a cudaStream_t
+ * (NULL = the legacy default stream).  Every call is asynchronous and
+ * stream-ordered; none synchronises the host, except dg_get_last_error.
+ *
+ * Errors.  Argument checks happen on the host before anything is launched
+ * and return DG_ERR_INVALID_ARG (nothing is written).  A launch failure
+ * returns DG_ERR_CUDA.  Conditions only the device can see (a wait that ran
+ * past its time limit, group metadata out of range) are recorded in a
+ * device-side error word and reported later by dg_get_last_error().
+ *
+ * Scratch memory.  The split-K path of the dense calls (chosen by the host
+ * heuristic for small M) keeps an FP32 workspace per (device, stream),
+ * allocated stream-ordered on first use and grown on demand; dg_shutdown()
+ * releases it.  No other call allocates device memory.
+ */
+#ifndef DG_H_
+#define DG_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DG_OK = 0,
+  DG_ERR_INVALID_ARG = -1,   /* rejected on the host, nothing launched        */
+  DG_ERR_UNSUPPORTED = -2,   /* valid but not implemented (e.g. no sm_100a)   */
+  DG_ERR_CUDA = -3,          /* a CUDA runtime call or launch failed          */
+  DG_ERR_TIMEOUT = -4,       /* a device wait ran past its limit (reported by
+                                dg_get_last_error)                            */
+  DG_ERR_BAD_METADATA = -5   /* masked_m outside [0, max_m] or m_indices >=
+                                num_groups, seen on the device                */
+} dg_status;
+
+/* ---------------------------------------------------------------- GEMMs */
+
+/* Dense NT FP8 GEMM: D[M,N] = C + A * B^T.
+ *   a    e4m3 [m][k] row-major          sfa  sf words of A: R = m, G = k/128
+ *   b    e4m3 [n][k] row-major          sfb  sf words of B: R = n, G = k/128
+ *                                            (128x128 block codes expanded per row)
+ *   c    bf16 [m][n] or NULL (C = 0); may equal d
+ *   d    bf16 [m][n]
+ * Requires m >= 0, n > 0 and n % 8 == 0, k > 0 and k % 128 == 0.  m == 0 is a
+ * no-op.  Source: zhouruolin.cn guide, section 五, "非分组 FP8 GEMM". */
+dg_status dg_fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                         const void* c, void* d, int m, int n, int k, void* stream);
+
+/* M-grouped contiguous FP8 GEMM (MoE prefill / training forward): the rows of
+ * all groups are concatenated along M, each group padded to a multiple of
+ * dg_get_mk_alignment_for_contiguous_layout() (= 128) rows.
+ *   a          e4m3 [m_total][k]           sfa  sf words, R = m_total, G = k/128
+ *   b          e4m3 [num_groups][n][k]     sfb  num_groups blocks of sf words, R = n
+ *   c          bf16 [m_total][n] or NULL
+ *   d          bf16 [m_total][n]
+ *   m_indices  int32 [m_total] on the device: group of each row, or -1 for a
+ *              padding row.  All rows of one 128-row block belong to one group
+ *              or are padding; a block whose first row is padding is skipped.
+ * D rows of padding rows are unspecified.  Requires m_total % 128 == 0.
+ * Source: zhouruolin.cn guide, section 五, m_grouped_fp8_gemm_nt_contiguous. */
+dg_status dg_m_grouped_fp8_gemm_nt_contiguous(const void* a, const int32_t* sfa, const void* b,
+                                              const int32_t* sfb, const void* c, void* d,
+                                              const int32_t* m_indices, int m_total, int n, int k,
+                                              int num_groups, void* stream);
+
+/* M-grouped masked FP8 GEMM (MoE decode): group g uses rows [0, masked_m[g])
+ * of its [max_m][k] slab of A.
+ *   a         e4m3 [num_groups][max_m][k]  sfa  num_groups blocks of sf words, R = max_m
+ *   b         e4m3 [num_groups][n][k]      sfb  num_groups blocks of sf words, R = n
+ *   d         bf16 [num_groups][max_m][n]; rows m >= masked_m[g] are never written
+ *   masked_m  int32 [num_groups] on the device (read inside the kernel, so the
+ *             call can be captured in a CUDA graph and replayed with new counts)
+ *   expected_m host-side hint of the typical masked_m (heuristic only; may be 0)
+ * Requires 1 <= num_groups <= 1024, max_m > 0.  masked_m values outside
+ * [0, max_m] are clamped and reported as DG_ERR_BAD_METADATA.
+ * Source: zhouruolin.cn guide, section 五, m_grouped_fp8_gemm_nt_masked. */
+dg_status dg_m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa, const void* b,
+                                          const int32_t* sfb, void* d, const int32_t* masked_m,
+                                          int num_groups, int max_m, int n, int k, int expected_m,
+                                          void* stream);
+
+/* FP8 x FP4 dense NT GEMM: as dg_fp8_gemm_nt but
+ *   b    e2m1 [n][k/2] (two codes per byte, low nibble = even k)
+ *   sfb  sf words of B: R = n, G = k/32 (one UE8M0 code per 1x32 group)
+ * Source: linlog.top update, section "FP4 精度支持". */
+dg_status dg_fp8_fp4_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                             const void* c, void* d, int m, int n, int k, void* stream);
+
+/* FP8 x FP4 M-grouped contiguous GEMM: as the FP8 contiguous call with B in
+ * e2m1 [num_groups][n][k/2] and per-group sf words R = n, G = k/32. */
+dg_status dg_m_grouped_fp8_fp4_gemm_nt_contiguous(const void* a, const int32_t* sfa, const void* b,
+                                                  const int32_t* sfb, const void* c, void* d,
+                                                  const int32_t* m_indices, int m_total, int n, int k,
+                                                  int num_groups, void* stream);
+
+/* ------------------------------------------------------ input preparation */
+
+/* Quantise FP32 x [rows][cols] to e4m3 with one UE8M0 scale per
+ * block_rows x 128 block (block_rows = 1: activations, 1x128; block_rows =
+ * 128: weights, 128x128).  scale = 2^i, i = min{ i : 448 * 2^i >= amax }
+ * (amax = 0 gives i = 0), q = e4m3(x / scale) rounded to nearest even.
+ *   q   e4m3 [rows][cols]
+ *   sf  ue8m0 [ceil(rows/block_rows)][cols/128]
+ * Requires cols % 128 == 0. */
+dg_status dg_quantize_fp8(const float* x, int rows, int cols, int block_rows, uint8_t* q, uint8_t* sf,
+                          void* stream);
+
+/* Quantise FP32 x [rows][cols] to e2m1 with one UE8M0 scale per 1x32 group
+ * (qmax = 6).  q: e2m1 [rows][cols/2]; sf: ue8m0 [rows][cols/32].
+ * Requires cols % 32 == 0. */
+dg_status dg_quantize_fp4(const float* x, int rows, int cols, uint8_t* q, uint8_t* sf, void* stream);
+
+/* Pack UE8M0 codes sf [ceil(rows/row_div)][num_sf_cols] into sf words (layout
+ * above) for a matrix of `rows` rows; row r reads code row r/row_div
+ * (row_div = 1 per-row scales, 128 for 128x128 block scales).
+ * packed has dg_packed_sf_words(rows, num_sf_cols) int32 entries. */
+dg_status dg_pack_sf(const uint8_t* sf, int rows, int num_sf_cols, int row_div, int32_t* packed,
+                     void* stream);
+
+/* Number of int32 words of the packed layout: ceil(cols/4) * ceil(rows/128) * 128. */
+int64_t dg_packed_sf_words(int rows, int num_sf_cols);
+
+/* --------------------------------------------------------------- utilities */
+
+/* Number of SMs the GEMM kernels use (default: all SMs of the current
+ * device).  dg_set_num_sms(0) restores the default. */
+int dg_get_num_sms(void);
+dg_status dg_set_num_sms(int num_sms);
+
+/* Row alignment of groups in the contiguous layout: 128. */
+int dg_get_mk_alignment_for_contiguous_layout(void);
+
+/* Synchronises `stream`, then returns and clears the first device-side error
+ * recorded on the current device (DG_OK if none). */
+dg_status dg_get_last_error(void* stream);
+
+/* Test hook: launches a kernel whose single wait can never be satisfied and
+ * must give up after limit_us microseconds; dg_get_last_error() then reports
+ * DG_ERR_TIMEOUT.  Faults nothing and leaves the context usable. */
+dg_status dg_debug_starved_wait(unsigned int limit_us, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* dg_status_string(int status);
+
+/* Kernels this library has launched in this process (all devices). */
+uint64_t dg_launch_count(void);
+
+/* Configuration the dense heuristic picks for (m, n, k): block_n, split-K
+ * slices, work units and grid size (any pointer may be NULL). */
+dg_status dg_query_dense_config(int m, int n, int k, int* block_n, int* splits, int* units, int* grid);
+
+/* Output tiles of an m x n problem cut into block_m x block_n tiles (the
+ * count the heuristic balances against the SM count; "DeepSeek 开源第三弹 ...
+ * DeepGEMM" (app.myzaker.com), section "非对齐块大小"). */
+int64_t dg_num_tiles(int m, int n, int block_m, int block_n);
+
+/* Releases the split-K workspaces of all devices (synchronises each). */
+void dg_shutdown(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DG_H_ */

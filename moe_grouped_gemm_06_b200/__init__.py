@@ -1,0 +1,220 @@
+"""B200 (sm_100a) fine-grained-scaled FP8 / FP8xFP4 GEMM:  D = C + A @ B^T.
+
+Thin Python binding over the C ABI in ``include/dg.h`` (``libdg.so``, built
+in-tree by ``moe_grouped_gemm_06_b200/build.py``).  Each function here has
+the name of the C entry point it calls and does argument marshalling only:
+it reads shapes and device pointers off torch tensors and passes the current
+CUDA stream.  Every step of the computation runs in the library's kernels;
+there is no fallback of any kind, and importing this package raises if the
+library has not been built.
+
+torch is used for device memory and streams only.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "DGError", "lib", "dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
+    "dg_m_grouped_fp8_gemm_nt_masked", "dg_fp8_fp4_gemm_nt", "dg_m_grouped_fp8_fp4_gemm_nt_contiguous",
+    "dg_quantize_fp8", "dg_quantize_fp4", "dg_pack_sf", "dg_packed_sf_words", "dg_get_num_sms",
+    "dg_set_num_sms", "dg_get_mk_alignment_for_contiguous_layout", "dg_get_last_error",
+    "dg_debug_starved_wait", "dg_launch_count", "dg_query_dense_config", "dg_num_tiles", "dg_shutdown",
+    "SYMBOLS",
+]
+
+# DG_LIBRARY may name another build of the same library (e.g. one compiled
+# with -DDG_SELF_CHECK); by default the in-tree libdg.so is loaded.
+LIB_PATH = os.environ.get("DG_LIBRARY") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdg.so")
+
+_VP, _I32P, _INT, _I64 = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+
+# C signatures of every exported entry point (name -> (restype, argtypes)).
+SYMBOLS = {
+    "dg_fp8_gemm_nt": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _INT, _INT, _INT, _VP]),
+    "dg_m_grouped_fp8_gemm_nt_contiguous": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _I32P, _INT, _INT, _INT,
+                                                   _INT, _VP]),
+    "dg_m_grouped_fp8_gemm_nt_masked": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _I32P, _INT, _INT, _INT, _INT, _INT,
+                                               _VP]),
+    "dg_fp8_fp4_gemm_nt": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _INT, _INT, _INT, _VP]),
+    "dg_m_grouped_fp8_fp4_gemm_nt_contiguous": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _I32P, _INT, _INT,
+                                                       _INT, _INT, _VP]),
+    "dg_quantize_fp8": (_INT, [_VP, _INT, _INT, _INT, _VP, _VP, _VP]),
+    "dg_quantize_fp4": (_INT, [_VP, _INT, _INT, _VP, _VP, _VP]),
+    "dg_pack_sf": (_INT, [_VP, _INT, _INT, _INT, _VP, _VP]),
+    "dg_packed_sf_words": (_I64, [_INT, _INT]),
+    "dg_get_num_sms": (_INT, []),
+    "dg_set_num_sms": (_INT, [_INT]),
+    "dg_get_mk_alignment_for_contiguous_layout": (_INT, []),
+    "dg_get_last_error": (_INT, [_VP]),
+    "dg_debug_starved_wait": (_INT, [ctypes.c_uint, _VP]),
+    "dg_status_string": (ctypes.c_char_p, [_INT]),
+    "dg_launch_count": (ctypes.c_uint64, []),
+    "dg_query_dense_config": (_INT, [_INT, _INT, _INT, _VP, _VP, _VP, _VP]),
+    "dg_num_tiles": (_I64, [_INT, _INT, _INT, _INT]),
+    "dg_shutdown": (None, []),
+}
+
+_lib = None
+
+
+class DGError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libdg.so (raises if it was never built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m moe_grouped_gemm_06_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SYMBOLS.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().dg_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise DGError(status, where)
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _bytes2(t):
+    """2-D byte view [rows, cols] of a uint8 / float8 / packed tensor."""
+    return t.shape[-2], t.shape[-1]
+
+
+# ------------------------------------------------------------------ GEMMs
+
+def dg_fp8_gemm_nt(a, sfa, b, sfb, c, d, stream=None) -> None:
+    """D = C + A @ B^T.  a: e4m3 [m, k]; b: e4m3 [n, k]; sfa/sfb: packed sf
+    words (int32); c: bf16 [m, n] or None; d: bf16 [m, n]."""
+    m, k = a.shape
+    n = b.shape[0]
+    _check(lib().dg_fp8_gemm_nt(_p(a), _p(sfa), _p(b), _p(sfb), _p(c), _p(d), m, n, k, _stream(stream)),
+           "dg_fp8_gemm_nt")
+
+
+def dg_fp8_fp4_gemm_nt(a, sfa, b, sfb, c, d, stream=None) -> None:
+    """As dg_fp8_gemm_nt with b: e2m1 packed [n, k/2] and per-1x32 sfb."""
+    m, k = a.shape
+    n = b.shape[0]
+    _check(lib().dg_fp8_fp4_gemm_nt(_p(a), _p(sfa), _p(b), _p(sfb), _p(c), _p(d), m, n, k, _stream(stream)),
+           "dg_fp8_fp4_gemm_nt")
+
+
+def dg_m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, c, d, m_indices, stream=None) -> None:
+    """a: e4m3 [m_total, k]; b: e4m3 [groups, n, k]; m_indices: int32 [m_total]."""
+    m_total, k = a.shape
+    g, n = b.shape[0], b.shape[1]
+    _check(lib().dg_m_grouped_fp8_gemm_nt_contiguous(_p(a), _p(sfa), _p(b), _p(sfb), _p(c), _p(d), _p(m_indices),
+                                                     m_total, n, k, g, _stream(stream)),
+           "dg_m_grouped_fp8_gemm_nt_contiguous")
+
+
+def dg_m_grouped_fp8_fp4_gemm_nt_contiguous(a, sfa, b, sfb, c, d, m_indices, stream=None) -> None:
+    """a: e4m3 [m_total, k]; b: e2m1 [groups, n, k/2]; m_indices: int32 [m_total]."""
+    m_total, k = a.shape
+    g, n = b.shape[0], b.shape[1]
+    _check(lib().dg_m_grouped_fp8_fp4_gemm_nt_contiguous(_p(a), _p(sfa), _p(b), _p(sfb), _p(c), _p(d),
+                                                         _p(m_indices), m_total, n, k, g, _stream(stream)),
+           "dg_m_grouped_fp8_fp4_gemm_nt_contiguous")
+
+
+def dg_m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, masked_m, expected_m: int = 0, stream=None) -> None:
+    """a: e4m3 [groups, max_m, k]; b: e4m3 [groups, n, k]; d: bf16 [groups, max_m, n];
+    masked_m: int32 [groups] on the device."""
+    g, max_m, k = a.shape
+    n = b.shape[1]
+    _check(lib().dg_m_grouped_fp8_gemm_nt_masked(_p(a), _p(sfa), _p(b), _p(sfb), _p(d), _p(masked_m), g, max_m,
+                                                 n, k, int(expected_m), _stream(stream)),
+           "dg_m_grouped_fp8_gemm_nt_masked")
+
+
+# ------------------------------------------------------- input preparation
+
+def dg_quantize_fp8(x, q, sf, block_rows: int, stream=None) -> None:
+    """x: float32 [rows, cols] -> q: e4m3 [rows, cols], sf: ue8m0 [ceil(rows/block_rows), cols/128]."""
+    rows, cols = x.shape
+    _check(lib().dg_quantize_fp8(_p(x), rows, cols, int(block_rows), _p(q), _p(sf), _stream(stream)),
+           "dg_quantize_fp8")
+
+
+def dg_quantize_fp4(x, q, sf, stream=None) -> None:
+    """x: float32 [rows, cols] -> q: e2m1 [rows, cols/2], sf: ue8m0 [rows, cols/32]."""
+    rows, cols = x.shape
+    _check(lib().dg_quantize_fp4(_p(x), rows, cols, _p(q), _p(sf), _stream(stream)), "dg_quantize_fp4")
+
+
+def dg_pack_sf(sf, rows: int, packed, row_div: int = 1, stream=None) -> None:
+    """sf: ue8m0 [ceil(rows/row_div), cols] -> packed int32 [dg_packed_sf_words(rows, cols)]."""
+    cols = sf.shape[-1]
+    _check(lib().dg_pack_sf(_p(sf), int(rows), int(cols), int(row_div), _p(packed), _stream(stream)),
+           "dg_pack_sf")
+
+
+def dg_packed_sf_words(rows: int, cols: int) -> int:
+    return int(lib().dg_packed_sf_words(int(rows), int(cols)))
+
+
+# ---------------------------------------------------------------- utilities
+
+def dg_get_num_sms() -> int:
+    return int(lib().dg_get_num_sms())
+
+
+def dg_set_num_sms(n: int) -> None:
+    _check(lib().dg_set_num_sms(int(n)), "dg_set_num_sms")
+
+
+def dg_get_mk_alignment_for_contiguous_layout() -> int:
+    return int(lib().dg_get_mk_alignment_for_contiguous_layout())
+
+
+def dg_get_last_error(stream=None) -> int:
+    """Synchronises the stream; returns and clears the device-side error (0 = none)."""
+    return int(lib().dg_get_last_error(_stream(stream)))
+
+
+def dg_debug_starved_wait(limit_us: int, stream=None) -> None:
+    _check(lib().dg_debug_starved_wait(int(limit_us), _stream(stream)), "dg_debug_starved_wait")
+
+
+def dg_launch_count() -> int:
+    return int(lib().dg_launch_count())
+
+
+def dg_query_dense_config(m: int, n: int, k: int) -> dict:
+    vals = [ctypes.c_int(0) for _ in range(4)]
+    _check(lib().dg_query_dense_config(m, n, k, *[ctypes.byref(v) for v in vals]), "dg_query_dense_config")
+    return dict(zip(("block_n", "splits", "units", "grid"), (v.value for v in vals)))
+
+
+def dg_num_tiles(m: int, n: int, block_m: int, block_n: int) -> int:
+    return int(lib().dg_num_tiles(m, n, block_m, block_n))
+
+
+def dg_shutdown() -> None:
+    lib().dg_shutdown()

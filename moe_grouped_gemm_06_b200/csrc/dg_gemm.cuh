@@ -1,0 +1,524 @@
+// dg_gemm.cuh -- the persistent, warp-specialised, block-scaled GEMM for sm_100a.
+//
+//   D = C + A * B^T   (A: M x K e4m3, B: N x K e4m3 or e2m1, both K-major;
+//                      C, D: bf16 row-major; FP32 accumulation in TMEM)
+//
+// with DeepSeek-V3 fine-grained scaling: one UE8M0 scale per 1x128 row-group
+// of A and per 128x128 block of B (FP4 B: per 1x32 row-group).  Sources:
+// "DeepSeek 开源第三弹 ... DeepGEMM" (app.myzaker.com), sections "DeepGEMM"
+// (fine-grained scaling), "优化技术" (persistent warp specialisation, TMA
+// loads/stores, unified block scheduler with L2 rasterisation, unaligned
+// block sizes); "DeepGEMM：统一高性能张量核心 GEMM 计算库编译与使用指南"
+// (zhouruolin.cn), section 五 (D = C + A @ B, NT layout, packed UE8M0 scales,
+// M-grouped contiguous and masked layouts); "DeepSeek 发布 DeepGEMM 重大更新"
+// (linlog.top), section "FP4 精度支持" (FP8 x FP4).
+//
+// Roles (192 threads, one CTA per SM, persistent over work units):
+//   warp 0      TMA producer: A/B tiles (128-byte swizzle) and packed scale
+//               words into a STAGES-deep shared-memory ring.
+//   warp 1      allocates TMEM; one lane issues tcgen05.cp (scales -> TMEM)
+//               and tcgen05.mma.kind::mxf8f6f4.block_scale into a
+//               double-buffered FP32 accumulator.
+//   warps 2..5  epilogue: tcgen05.ld -> (+C) -> bf16 -> swizzled smem -> TMA
+//               store; rows past a masked group's count are never written.
+//               With split-K they write FP32 partials instead.
+//
+// The scales are applied inside the MMA: the UE8M0 code of a 1x128 group is
+// used for each of the four K=32 steps of its 128-wide block (the instruction
+// descriptor's scale-factor id selects the byte of the packed word), which
+// replaces the Hopper design's CUDA-core promotion of every K-block.
+#pragma once
+#include <cuda_bf16.h>
+#include "dg_ptx.cuh"
+
+namespace dg {
+
+constexpr int kBM = 128;           // rows of A per tile (= TMEM lanes)
+constexpr int kBK = 128;           // K per pipeline stage (= one scale block)
+constexpr int kThreads = 192;
+constexpr int kEpiCols = 32;       // columns per epilogue store box
+constexpr int kTmemCols = 512;
+constexpr int kMaxMaskedGroups = 1024;
+
+enum : int { kDense = 0, kContig = 1, kMasked = 2 };
+
+struct GemmArgs {
+  const int32_t* sfa;        // packed scale words of A
+  const int32_t* sfb;        // packed scale words of B
+  const uint16_t* c;         // bf16 bits [rows][n] or nullptr
+  uint16_t* d;               // bf16 bits (predicated-store path)
+  float* ws;                 // split-K partials [splits][rows][n]
+  const int32_t* m_indices;  // contiguous: group of each row (-1 = padding)
+  const int32_t* masked_m;   // masked: valid rows per group
+  int rows;                  // dense: M; contiguous: M_total; masked: max_m
+  int n, k;
+  int num_groups;
+  int num_m_blocks;          // per group for masked
+  int num_n_blocks;
+  int kb_total;              // k / 128
+  int splits, kb_per_split;
+  int sfa_chunks, sfb_chunks;          // ceil(rows/128), ceil(n/128)
+  long long sfa_group_words, sfb_group_words;
+  int sfa_q, sfb_q;                    // packed groups along K
+  int raster;                          // m-blocks per raster band
+  unsigned long long timeout_ns;
+  long long sfa_words, sfb_words;      // total packed words (self-check bounds)
+};
+
+template <int BN, bool FP4>
+struct Cfg {
+  // The scale-factor operand of the MMA is addressed in TMEM columns of 32
+  // rows (a 128-row chunk spans 4 columns), and that address must be even:
+  // a tile starting 32 or 96 rows into a chunk (odd column) faults with a
+  // misaligned-address error.  Block widths are therefore multiples of 64, so
+  // a tile starts 0 or 64 rows into its first chunk.
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
+  static constexpr int kSfbChunks = 3;                       // 128-row scale chunks a tile can touch
+  static constexpr int kAccBufs = (BN <= 224) ? 2 : 1;
+  // accumulator buffers start at TMEM columns 0 and 256
+  static constexpr int kABytes = kBM * kBK;                  // 16 KB
+  static constexpr int kBBytes = BN * kBK;                   // smem bytes (FP4 lands padded to 1 B/elt)
+  static constexpr int kBTxBytes = FP4 ? BN * kBK / 2 : BN * kBK;  // bytes the TMA copy reports (packed)
+  static constexpr int kSfaBytes = 512;
+  static constexpr int kSfbBytes = kSfbChunks * 512;
+  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+  static constexpr int kEpiBytes = 4 * 2 * 32 * 64;          // 4 warps x 2 buffers x (32 rows x 64 B)
+  static constexpr int kMaskBytes = ((kMaxMaskedGroups + 1) * 4 + 15) / 16 * 16;
+  static constexpr int kBarBytes = 256;
+  static constexpr int kBudget = 232448 - 1024;              // 227 KB minus alignment slack
+  static constexpr int kStagesRaw = (kBudget - kEpiBytes - kMaskBytes - kBarBytes) / kStageBytes;
+  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  static_assert(kStages >= 2, "stages");
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kEpiBytes + kMaskBytes + kBarBytes;
+  static constexpr uint32_t kColAcc = 0;
+  static constexpr uint32_t kAccStride = 256;
+  static constexpr uint32_t kColSfa = (kAccBufs == 2) ? 256 + BN : BN;   // even, 4-column aligned
+  static constexpr uint32_t kColSfb = kColSfa + 4;
+  static_assert(kColSfb + 4 * kSfbChunks <= kTmemCols, "TMEM columns");
+  // Instruction descriptor of kind::mxf8f6f4 with block scaling: A = E4M3,
+  // B = E4M3 (0) or E2M1 (5), both K-major, UE8M0 scales, M = 128, N = BN.
+  static constexpr uint32_t kIdesc = (0u << 7) | ((FP4 ? 5u : 0u) << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                     (1u << 23) | ((uint32_t)(kBM >> 4) << 24);
+};
+
+struct Unit {
+  int g, mb, nb, split;
+  bool valid;
+};
+
+// Work-unit order: split-K slice slowest, then L2-rasterised (m, n) tiles in
+// bands of `raster` m-blocks (m fastest inside a band), so that the CTAs
+// running at the same time share the A rows and B columns of one band.
+// Masked: group by group, n-blocks, m-blocks fastest (m-blocks of a group
+// share its B tiles).
+template <int LAYOUT>
+__device__ __forceinline__ Unit decode_unit(int t, const GemmArgs& a, const int* s_prefix) {
+  Unit u;
+  u.valid = true;
+  if (LAYOUT == kMasked) {
+    int g = 0;
+    while (s_prefix[g + 1] <= t) ++g;
+    int local = t - s_prefix[g];
+    int valid_rows = min(max(__ldg(a.masked_m + g), 0), a.rows);
+    int mcount = (valid_rows + kBM - 1) / kBM;
+    u.g = g;
+    u.nb = local / mcount;
+    u.mb = local % mcount;
+    u.split = 0;
+    return u;
+  }
+  int tiles = a.num_m_blocks * a.num_n_blocks;
+  u.split = t / tiles;
+  int tl = t - u.split * tiles;
+  int band_tiles = a.raster * a.num_n_blocks;
+  int band = tl / band_tiles;
+  int rem = tl - band * band_tiles;
+  int band_rows = min(a.raster, a.num_m_blocks - band * a.raster);
+  u.mb = band * a.raster + rem % band_rows;
+  u.nb = rem / band_rows;
+  u.g = 0;
+  if (LAYOUT == kContig) {
+    int g = __ldg(a.m_indices + (long long)u.mb * kBM);
+    u.g = g;
+    u.valid = (g >= 0 && g < a.num_groups);
+  }
+  return u;
+}
+
+template <int BN, bool FP4, int LAYOUT>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                const __grid_constant__ CUtensorMap tm_d, const GemmArgs args) {
+  using C = Cfg<BN, FP4>;
+  constexpr int S = C::kStages;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* s_a = smem;
+  uint8_t* s_b = s_a + S * C::kABytes;
+  uint8_t* s_sfa = s_b + S * C::kBBytes;
+  uint8_t* s_sfb = s_sfa + S * C::kSfaBytes;
+  uint8_t* s_epi = s_sfb + S * C::kSfbBytes;
+  int* s_prefix = reinterpret_cast<int*>(s_epi + C::kEpiBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(s_prefix) + C::kMaskBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* tfull = bars + 2 * S;
+  uint64_t* tempty = bars + 2 * S + 2;
+  uint64_t* drain = bars + 2 * S + 4;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+
+  const int warp = threadIdx.x / 32;
+  const uint32_t lane = lane_id();
+  const GemmArgs& a = args;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_b);
+    prefetch_tmap(&tm_d);
+  }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, kTmemCols);
+    tmem_relinquish();
+  }
+  int num_units;
+  if (LAYOUT == kMasked) {
+    // tiles per group, read from device memory (so the call stays
+    // graph-capturable), then an exclusive prefix over the groups
+    for (int g = threadIdx.x; g < a.num_groups; g += kThreads) {
+      int mm = __ldg(a.masked_m + g);
+      if (mm < 0 || mm > a.rows) record_error(-5 /* DG_ERR_BAD_METADATA */);
+      mm = min(max(mm, 0), a.rows);
+      s_prefix[g + 1] = ((mm + kBM - 1) / kBM) * a.num_n_blocks;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      s_prefix[0] = 0;
+      for (int g = 0; g < a.num_groups; ++g) s_prefix[g + 1] += s_prefix[g];
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  if (LAYOUT == kMasked)
+    num_units = s_prefix[a.num_groups];
+  else
+    num_units = a.num_m_blocks * a.num_n_blocks * a.splits;
+
+  const uint64_t limit = a.timeout_ns;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t filled_phase[8];
+      uint32_t filled_mask = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_units && ok; t += gridDim.x) {
+        Unit u = decode_unit<LAYOUT>(t, a, s_prefix);
+        if (LAYOUT == kContig && !u.valid) {
+          if (u.g >= a.num_groups) record_error(-5);
+          continue;
+        }
+        const int kb0 = u.split * a.kb_per_split;
+        const int kb1 = min(a.kb_total, kb0 + a.kb_per_split);
+        const int n0 = u.nb * BN;
+        const int c0 = n0 / 128;
+        const int c1 = (min(n0 + BN, a.n) - 1) / 128;
+        const int nchunks = c1 - c0 + 1;
+        const int a_row = u.mb * kBM;
+        const int a_grp = (LAYOUT == kMasked) ? u.g : 0;
+        const int b_grp = (LAYOUT == kDense) ? 0 : u.g;
+        const int32_t* sfa_g = a.sfa + (LAYOUT == kMasked ? (long long)u.g * a.sfa_group_words : 0);
+        const int32_t* sfb_g = a.sfb + (long long)b_grp * a.sfb_group_words;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!dg_wait(&empty[stage], phase ^ 1, s_abort, limit)) {
+            ok = false;
+            break;
+          }
+          const bool new_sfa = ((kb & 3) == 0) || kb == kb0;
+          const bool new_sfb = FP4 || new_sfa;
+          uint32_t bytes = C::kABytes + C::kBTxBytes;
+          if (new_sfa) bytes += C::kSfaBytes;
+          if (new_sfb) bytes += 512u * nchunks;
+          DG_CHECK(((smem_u32(s_a + stage * C::kABytes) | smem_u32(s_b + stage * C::kBBytes)) & 1023) == 0 &&
+                       u.mb < a.num_m_blocks && u.nb < a.num_n_blocks && kb < a.kb_total,
+                   6);
+          mbar_arrive_expect_tx(&full[stage], bytes);
+          tma_load_3d(s_a + stage * C::kABytes, &tm_a, &full[stage], kb * kBK, a_row, a_grp);
+          tma_load_3d(s_b + stage * C::kBBytes, &tm_b, &full[stage], kb * kBK, n0, b_grp);
+          if (new_sfa) {
+            const int32_t* src = sfa_g + ((long long)(kb >> 2) * a.sfa_chunks + u.mb) * 128;
+            if (DG_CHECK(src >= a.sfa && src + 128 <= a.sfa + a.sfa_words &&
+                             ((reinterpret_cast<uintptr_t>(src) | smem_u32(s_sfa + stage * C::kSfaBytes)) & 15) == 0,
+                         4))
+              bulk_load(s_sfa + stage * C::kSfaBytes, src, C::kSfaBytes, &full[stage]);
+          }
+          if (new_sfb) {
+            const int q = FP4 ? kb : (kb >> 2);
+            const int32_t* src = sfb_g + ((long long)q * a.sfb_chunks + c0) * 128;
+            if (DG_CHECK(src >= a.sfb && src + 128 * nchunks <= a.sfb + a.sfb_words && nchunks >= 1 &&
+                             nchunks <= C::kSfbChunks &&
+                             ((reinterpret_cast<uintptr_t>(src) | smem_u32(s_sfb + stage * C::kSfbBytes)) & 15) == 0,
+                         5))
+              bulk_load(s_sfb + stage * C::kSfbBytes, src, 512u * nchunks, &full[stage]);
+          }
+          filled_phase[stage] = phase;
+          filled_mask |= 1u << stage;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // never leave copies in flight into shared memory: wait (bounded) for
+        // the last fill of every stage
+        for (int s = 0; s < S; ++s)
+          if (filled_mask & (1u << s)) {
+            uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(&full[s], filled_phase[s]) && global_timer_ns() - t0 < limit) {
+            }
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      const uint32_t sfa_t = tmem_base + C::kColSfa;
+      for (int t = blockIdx.x; t < num_units && ok; t += gridDim.x) {
+        Unit u = decode_unit<LAYOUT>(t, a, s_prefix);
+        if (LAYOUT == kContig && !u.valid) continue;
+        const int kb0 = u.split * a.kb_per_split;
+        const int kb1 = min(a.kb_total, kb0 + a.kb_per_split);
+        const int n0 = u.nb * BN;
+        const int nchunks = (min(n0 + BN, a.n) - 1) / 128 - n0 / 128 + 1;
+        const uint32_t sfb_t = tmem_base + C::kColSfb + (uint32_t)((n0 % 128) / 32);
+        const int buf = (C::kAccBufs == 2) ? (local & 1) : 0;
+        const uint32_t use = (C::kAccBufs == 2) ? (uint32_t)(local >> 1) : (uint32_t)local;
+        if (!dg_wait(&tempty[buf], (use & 1) ^ 1, s_abort, limit)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_t = tmem_base + C::kColAcc + buf * C::kAccStride;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!dg_wait(&full[stage], phase, s_abort, limit)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const bool new_sfa = ((kb & 3) == 0) || kb == kb0;
+          const bool new_sfb = FP4 || new_sfa;
+          if (new_sfa) tc_cp_32x128b_x4(sfa_t, sdesc_sf_32x16(s_sfa + stage * C::kSfaBytes));
+          if (new_sfb)
+            for (int ch = 0; ch < nchunks; ++ch)
+              tc_cp_32x128b_x4(tmem_base + C::kColSfb + 4 * ch,
+                               sdesc_sf_32x16(s_sfb + stage * C::kSfbBytes + ch * 512));
+          const uint64_t adesc = sdesc_k_sw128(s_a + stage * C::kABytes);
+          const uint64_t bdesc = sdesc_k_sw128(s_b + stage * C::kBBytes);
+          const uint32_t ida = (uint32_t)(kb & 3);
+#pragma unroll
+          for (int ks = 0; ks < kBK / 32; ++ks) {
+            const uint32_t idb = FP4 ? (uint32_t)ks : ida;
+            const uint32_t idesc = C::kIdesc | (ida << 29) | (idb << 4);
+            tc_mma_mxf8f6f4(d_t, adesc + (uint64_t)(ks * 2), bdesc + (uint64_t)(ks * 2), idesc,
+                            sfa_t | (ida << 30), sfb_t | (idb << 30), (kb > kb0 || ks > 0) ? 1u : 0u);
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&tfull[buf]);
+        ++local;
+      }
+      // all tcgen05 work of this thread complete before TMEM is released
+      tc_commit(drain);
+      uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < limit) {
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM sub-partition of this warp: lanes 32q..32q+31
+    uint8_t* stg0 = s_epi + (warp - 2) * (2 * 32 * 64);
+    int local = 0;
+    uint32_t store_seq = 0;
+    for (int t = blockIdx.x; t < num_units; t += gridDim.x) {
+      Unit u = decode_unit<LAYOUT>(t, a, s_prefix);
+      if (LAYOUT == kContig && !u.valid) continue;
+      const int buf = (C::kAccBufs == 2) ? (local & 1) : 0;
+      const uint32_t use = (C::kAccBufs == 2) ? (uint32_t)(local >> 1) : (uint32_t)local;
+      int ok = 1;
+      if (lane == 0) ok = dg_wait(&tfull[buf], use & 1, s_abort, limit) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const int r0 = u.mb * kBM + q * 32;  // first row of this warp (within the group for masked)
+      int limit_rows = a.rows;
+      if (LAYOUT == kMasked) limit_rows = min(max(__ldg(a.masked_m + u.g), 0), a.rows);
+      const int vr = min(32, limit_rows - r0);
+      const int row = r0 + (int)lane;
+      const long long grow = (LAYOUT == kMasked) ? (long long)u.g * a.rows + row : row;
+      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + C::kColAcc + buf * C::kAccStride;
+#pragma unroll 1
+      for (int j = 0; j < BN / kEpiCols; ++j) {
+        const int col0 = u.nb * BN + j * kEpiCols;
+        if (vr <= 0 || col0 >= a.n) break;
+        // C for this thread's row segment, fetched before the TMEM read
+        float cv[kEpiCols];
+#pragma unroll
+        for (int i = 0; i < kEpiCols; ++i) cv[i] = 0.f;
+        if (a.c != nullptr && a.splits == 1 && (int)lane < vr &&
+            DG_CHECK(((reinterpret_cast<uintptr_t>(a.c + grow * a.n + col0) & 15) == 0) && row < a.rows &&
+                         grow >= 0, 1)) {
+          const uint4* src = reinterpret_cast<const uint4*>(a.c + grow * a.n + col0);
+#pragma unroll
+          for (int v = 0; v < kEpiCols / 8; ++v) {
+            if (col0 + 8 * v < a.n) {
+              uint4 w = __ldg(src + v);
+              const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                cv[8 * v + 2 * h] = __uint_as_float(ww[h] << 16);
+                cv[8 * v + 2 * h + 1] = __uint_as_float(ww[h] & 0xFFFF0000u);
+              }
+            }
+          }
+        }
+        uint32_t acc[kEpiCols];
+        DG_CHECK(((t_row & 0xFFFF) + j * kEpiCols + kEpiCols <= (uint32_t)kTmemCols) &&
+                     ((t_row >> 16) & 0xFFFF) == (uint32_t)(q * 32) + (tmem_base >> 16) && (warp & 3) == q,
+                 8);
+        tc_ld_32x32b_x32(t_row + j * kEpiCols, acc);
+        tc_wait_ld_regs(acc);
+        if (a.splits > 1) {
+          // FP32 partials of this K slice: ws[split][row][col]
+          if ((int)lane < vr &&
+              DG_CHECK(a.ws != nullptr && u.split < a.splits && row < a.rows &&
+                           (reinterpret_cast<uintptr_t>(a.ws + ((long long)u.split * a.rows + row) * a.n + col0) & 15) == 0,
+                       3)) {
+            float4* dst = reinterpret_cast<float4*>(a.ws + ((long long)u.split * a.rows + row) * a.n + col0);
+#pragma unroll
+            for (int v = 0; v < kEpiCols / 4; ++v)
+              if (col0 + 4 * v < a.n)
+                dst[v] = make_float4(__uint_as_float(acc[4 * v]), __uint_as_float(acc[4 * v + 1]),
+                                     __uint_as_float(acc[4 * v + 2]), __uint_as_float(acc[4 * v + 3]));
+          }
+          continue;
+        }
+        uint32_t packed[kEpiCols / 2];
+#pragma unroll
+        for (int i = 0; i < kEpiCols / 2; ++i) {
+          __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(acc[2 * i]) + cv[2 * i],
+                                                   __uint_as_float(acc[2 * i + 1]) + cv[2 * i + 1]);
+          packed[i] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        if (vr == 32) {
+          // full 32-row box: swizzled staging (64-byte rows) + TMA store
+          uint8_t* stg = stg0 + (store_seq & 1) * (32 * 64);
+          DG_CHECK((smem_u32(stg) & 1023) == 0 && stg >= s_epi && stg + 2048 <= s_epi + C::kEpiBytes &&
+                       (col0 % 8) == 0 && r0 + 32 <= (LAYOUT == kMasked ? limit_rows : a.rows),
+                   7);
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            const int pos = ch ^ ((lane >> 1) & 3);
+            *reinterpret_cast<uint4*>(stg + lane * 64 + pos * 16) =
+                make_uint4(packed[4 * ch], packed[4 * ch + 1], packed[4 * ch + 2], packed[4 * ch + 3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&tm_d, stg, col0, r0, (LAYOUT == kMasked) ? u.g : 0);
+            bulk_commit_group();
+          }
+          ++store_seq;
+        } else if ((int)lane < vr &&
+                   DG_CHECK((reinterpret_cast<uintptr_t>(a.d + grow * a.n + col0) & 15) == 0 && row < limit_rows,
+                            2)) {
+          // partial box (M tail or masked group tail): predicated row stores
+          uint4* dst = reinterpret_cast<uint4*>(a.d + grow * a.n + col0);
+#pragma unroll
+          for (int v = 0; v < kEpiCols / 8; ++v)
+            if (col0 + 8 * v < a.n)
+              dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+      ++local;
+    }
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// Split-K reduction: D = bf16(sum_s ws[s] + C), 8 columns per thread.
+__global__ void splitk_reduce_kernel(const float* __restrict__ ws, const uint16_t* __restrict__ c,
+                                     uint16_t* __restrict__ d, int rows, int n, int splits) {
+  const long long units = (long long)rows * (n / 8);
+  for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < units;
+       u += (long long)gridDim.x * blockDim.x) {
+    const long long r = u / (n / 8);
+    const int col = (int)(u - r * (n / 8)) * 8;
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int s = 0; s < splits; ++s) {
+      const float4* p = reinterpret_cast<const float4*>(ws + ((long long)s * rows + r) * n + col);
+      float4 x = __ldg(p), y = __ldg(p + 1);
+      acc[0] += x.x; acc[1] += x.y; acc[2] += x.z; acc[3] += x.w;
+      acc[4] += y.x; acc[5] += y.y; acc[6] += y.z; acc[7] += y.w;
+    }
+    if (c != nullptr) {
+      uint4 w = __ldg(reinterpret_cast<const uint4*>(c + r * n + col));
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        acc[2 * h] += __uint_as_float(ww[h] << 16);
+        acc[2 * h + 1] += __uint_as_float(ww[h] & 0xFFFF0000u);
+      }
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * h], acc[2 * h + 1]);
+      o[h] = *reinterpret_cast<uint32_t*>(&b);
+    }
+    *reinterpret_cast<uint4*>(d + r * n + col) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+}  // namespace dg

@@ -1,0 +1,480 @@
+// dg_lib.cu -- host side of the C ABI declared in include/dg.h: argument
+// validation, the tile/split heuristic, TMA descriptor encoding, split-K
+// workspaces and kernel launches.  All device code lives in the included
+// headers so that this file is the library's single translation unit.
+#include <atomic>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "../../include/dg.h"
+#include "dg_gemm.cuh"
+#include "dg_prep.cuh"
+
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+int g_num_sms_override = 0;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+unsigned long long timeout_ns() {
+  static unsigned long long v = [] {
+    const char* e = std::getenv("DG_TIMEOUT_MS");
+    long long ms = e ? std::atoll(e) : 4000;
+    if (ms <= 0) ms = 4000;
+    return (unsigned long long)ms * 1000000ull;
+  }();
+  return v;
+}
+
+bool log_enabled() {
+  static bool v = [] {
+    const char* e = std::getenv("DG_LOG");
+    return e && e[0] == '1';
+  }();
+  return v;
+}
+
+int device_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return sms;
+}
+
+int num_sms() {
+  if (g_num_sms_override > 0) return g_num_sms_override;
+  return device_sms();
+}
+
+// ------------------------------------------------------------ tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (EncodeTiledFn) nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// 3-D map: dims {d0 (innermost, elements), d1, d2}, strides in bytes of dims 1, 2.
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+              uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1, s2};
+  cuuint32_t box[3] = {b0, b1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------ heuristic
+
+constexpr int kBlockNs[] = {128, 192, 256};  // multiples of 64 (see Cfg in dg_gemm.cuh)
+
+struct Plan {
+  int bn = 128;
+  int splits = 1;
+  int kb_per_split = 1;
+  long long units = 0;
+  int grid = 0;
+};
+
+long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
+
+// Estimated critical path (per SM) in units of "B rows x K-blocks" streamed
+// through the tensor core: waves x (BN x K-blocks per unit + a per-unit
+// overhead of 4 K-blocks), with a 3% surcharge per extra split-K slice for
+// the partial-sum round trip.  Minimised over the instantiated block sizes;
+// ties keep fewer slices, then the larger block.
+Plan plan_gemm(long long m_blocks, int n, int k, int sms, bool allow_split) {
+  Plan best;
+  double best_cost = 1e300;
+  const int kb = k / 128;
+  for (int bn : kBlockNs) {
+    const long long tiles = m_blocks * ceil_div(n, bn);
+    const int max_s = allow_split ? std::max(1, std::min(16, kb / 2)) : 1;
+    for (int s = 1; s <= max_s; ++s) {
+      const int kbps = (int)ceil_div(kb, s);
+      const int s_eff = (int)ceil_div(kb, kbps);
+      if (s_eff != s) continue;
+      const long long units = tiles * s;
+      const double waves = (double)ceil_div(units, sms);
+      const double cost = waves * (double)bn * (kbps + 4) * (1.0 + 0.03 * (s - 1));
+      if (cost < best_cost * (1 - 1e-9)) {
+        best_cost = cost;
+        best.bn = bn;
+        best.splits = s;
+        best.kb_per_split = kbps;
+        best.units = units;
+      }
+    }
+  }
+  best.grid = (int)std::min<long long>(best.units, sms);
+  if (best.grid < 1) best.grid = 1;
+  return best;
+}
+
+// ------------------------------------------------------------ workspaces
+
+struct Workspace {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+std::mutex g_ws_mutex;
+std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+
+float* workspace(size_t bytes, cudaStream_t s) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(g_ws_mutex);
+  Workspace& w = g_ws[{dev, s}];
+  if (w.bytes < bytes) {
+    if (w.ptr) cudaFreeAsync(w.ptr, s);
+    w.ptr = nullptr;
+    w.bytes = 0;
+    if (cudaMallocAsync(&w.ptr, bytes, s) != cudaSuccess) return nullptr;
+    w.bytes = bytes;
+  }
+  return static_cast<float*>(w.ptr);
+}
+
+// ------------------------------------------------------------ launches
+
+template <int BN, bool FP4, int LAYOUT>
+dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td, const dg::GemmArgs& args,
+                      int grid, cudaStream_t s) {
+  using C = dg::Cfg<BN, FP4>;
+  auto kern = dg::gemm_kernel<BN, FP4, LAYOUT>;
+  static std::atomic<uint64_t> attr_set_mask{0};  // one bit per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(attr_set_mask.load() & bit)) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+      return DG_ERR_CUDA;
+    attr_set_mask.fetch_or(bit);
+  }
+  kern<<<grid, dg::kThreads, C::kSmemBytes, s>>>(ta, tb, td, args);
+  if (cudaGetLastError() != cudaSuccess) return DG_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return DG_OK;
+}
+
+template <bool FP4, int LAYOUT>
+dg_status dispatch(int bn, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
+                   const dg::GemmArgs& args, int grid, cudaStream_t s) {
+  switch (bn) {
+    case 128: return launch_gemm<128, FP4, LAYOUT>(ta, tb, td, args, grid, s);
+    case 192: return launch_gemm<192, FP4, LAYOUT>(ta, tb, td, args, grid, s);
+    case 256: return launch_gemm<256, FP4, LAYOUT>(ta, tb, td, args, grid, s);
+    default: return DG_ERR_UNSUPPORTED;
+  }
+}
+
+struct Problem {
+  const void* a;
+  const int32_t* sfa;
+  const void* b;
+  const int32_t* sfb;
+  const void* c;
+  void* d;
+  const int32_t* m_indices;
+  const int32_t* masked_m;
+  int rows;        // dense m, contiguous m_total, masked max_m
+  int n, k;
+  int groups;      // 1 for dense
+  int expected_m;  // masked hint
+};
+
+template <bool FP4, int LAYOUT>
+dg_status run_gemm(const Problem& p, cudaStream_t s) {
+  const int sms = num_sms();
+  if (sms <= 0) return DG_ERR_CUDA;
+  const long long m_blocks = ceil_div(p.rows, dg::kBM);
+  Plan plan;
+  if (LAYOUT == dg::kMasked) {
+    const int em = p.expected_m > 0 ? std::min(p.expected_m, p.rows) : p.rows;
+    plan = plan_gemm((long long)p.groups * ceil_div(em, dg::kBM), p.n, p.k, sms, false);
+    plan.grid = (int)std::min<long long>((long long)p.groups * m_blocks * ceil_div(p.n, plan.bn), sms);
+  } else {
+    const bool allow_split = (LAYOUT == dg::kDense) && p.rows <= 1024;
+    plan = plan_gemm(m_blocks, p.n, p.k, sms, allow_split);
+  }
+
+  dg::GemmArgs args{};
+  args.sfa = p.sfa;
+  args.sfb = p.sfb;
+  args.c = static_cast<const uint16_t*>(p.c);
+  args.d = static_cast<uint16_t*>(p.d);
+  args.ws = nullptr;
+  args.m_indices = p.m_indices;
+  args.masked_m = p.masked_m;
+  args.rows = p.rows;
+  args.n = p.n;
+  args.k = p.k;
+  args.num_groups = p.groups;
+  args.num_m_blocks = (int)m_blocks;
+  args.num_n_blocks = (int)ceil_div(p.n, plan.bn);
+  args.kb_total = p.k / 128;
+  args.splits = plan.splits;
+  args.kb_per_split = plan.kb_per_split;
+  args.sfa_chunks = (int)ceil_div(p.rows, 128);
+  args.sfb_chunks = (int)ceil_div(p.n, 128);
+  args.sfa_q = (int)ceil_div(p.k / 128, 4);
+  args.sfb_q = FP4 ? p.k / 128 : args.sfa_q;
+  args.sfa_group_words = (long long)args.sfa_q * args.sfa_chunks * 128;
+  args.sfb_group_words = (long long)args.sfb_q * args.sfb_chunks * 128;
+  args.raster = 8;
+  args.timeout_ns = timeout_ns();
+  args.sfa_words = args.sfa_group_words * ((LAYOUT == dg::kMasked) ? p.groups : 1);
+  args.sfb_words = args.sfb_group_words * ((LAYOUT == dg::kDense) ? 1 : p.groups);
+
+  if (plan.splits > 1) {
+    args.ws = workspace((size_t)plan.splits * p.rows * p.n * sizeof(float), s);
+    if (!args.ws) return DG_ERR_CUDA;
+  }
+
+  const int ga = (LAYOUT == dg::kMasked) ? p.groups : 1;
+  const int gb = (LAYOUT == dg::kDense) ? 1 : p.groups;
+  CUtensorMap ta, tb, td;
+  bool ok = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.a, p.k, p.rows, ga, (uint64_t)p.k,
+                     (uint64_t)p.rows * p.k, 128, dg::kBM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (FP4)
+    ok = ok && make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, p.b, p.k, p.n, gb, (uint64_t)p.k / 2,
+                        (uint64_t)p.n * p.k / 2, 128, plan.bn, CU_TENSOR_MAP_SWIZZLE_128B);
+  else
+    ok = ok && make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.b, p.k, p.n, gb, (uint64_t)p.k, (uint64_t)p.n * p.k,
+                        128, plan.bn, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok = ok && make_map(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.d, p.n, p.rows, ga, (uint64_t)p.n * 2,
+                      (uint64_t)p.rows * p.n * 2, dg::kEpiCols, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (!ok) return DG_ERR_CUDA;
+
+  if (log_enabled())
+    std::fprintf(stderr, "[dg] layout=%d fp4=%d rows=%d n=%d k=%d groups=%d -> block_n=%d splits=%d units=%lld grid=%d\n",
+                 LAYOUT, (int)FP4, p.rows, p.n, p.k, p.groups, plan.bn, plan.splits, plan.units, plan.grid);
+
+  dg_status st = dispatch<FP4, LAYOUT>(plan.bn, ta, tb, td, args, plan.grid, s);
+  if (st != DG_OK || plan.splits == 1) return st;
+
+  const long long units = (long long)p.rows * (p.n / 8);
+  const int threads = 256;
+  const int blocks = (int)std::min<long long>(ceil_div(units, threads), (long long)sms * 8);
+  dg::splitk_reduce_kernel<<<blocks, threads, 0, s>>>(args.ws, args.c, args.d, p.rows, p.n, plan.splits);
+  if (cudaGetLastError() != cudaSuccess) return DG_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return DG_OK;
+}
+
+dg_status check_common(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, const void* c,
+                       const void* d, int n, int k) {
+  if (!a || !sfa || !b || !sfb || !d) return DG_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(sfa) || !aligned16(b) || !aligned16(sfb) || !aligned16(d)) return DG_ERR_INVALID_ARG;
+  if (c && !aligned16(c)) return DG_ERR_INVALID_ARG;
+  if (n <= 0 || n % 8 != 0 || k <= 0 || k % 128 != 0) return DG_ERR_INVALID_ARG;
+  return DG_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+dg_status dg_fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, const void* c, void* d,
+                         int m, int n, int k, void* stream) {
+  if (m < 0) return DG_ERR_INVALID_ARG;
+  dg_status st = check_common(a, sfa, b, sfb, c, d, n, k);
+  if (st != DG_OK) return st;
+  if (m == 0) return DG_OK;
+  Problem p{a, sfa, b, sfb, c, d, nullptr, nullptr, m, n, k, 1, 0};
+  return run_gemm<false, dg::kDense>(p, static_cast<cudaStream_t>(stream));
+}
+
+dg_status dg_fp8_fp4_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, const void* c,
+                             void* d, int m, int n, int k, void* stream) {
+  if (m < 0) return DG_ERR_INVALID_ARG;
+  dg_status st = check_common(a, sfa, b, sfb, c, d, n, k);
+  if (st != DG_OK) return st;
+  if (m == 0) return DG_OK;
+  Problem p{a, sfa, b, sfb, c, d, nullptr, nullptr, m, n, k, 1, 0};
+  return run_gemm<true, dg::kDense>(p, static_cast<cudaStream_t>(stream));
+}
+
+static dg_status contiguous_impl(bool fp4, const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                                 const void* c, void* d, const int32_t* m_indices, int m_total, int n, int k,
+                                 int num_groups, void* stream) {
+  if (m_total < 0 || m_total % 128 != 0 || num_groups <= 0 || !m_indices) return DG_ERR_INVALID_ARG;
+  dg_status st = check_common(a, sfa, b, sfb, c, d, n, k);
+  if (st != DG_OK) return st;
+  if (c == d && c != nullptr) return DG_ERR_INVALID_ARG;
+  if (m_total == 0) return DG_OK;
+  Problem p{a, sfa, b, sfb, c, d, m_indices, nullptr, m_total, n, k, num_groups, 0};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return fp4 ? run_gemm<true, dg::kContig>(p, s) : run_gemm<false, dg::kContig>(p, s);
+}
+
+dg_status dg_m_grouped_fp8_gemm_nt_contiguous(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                                              const void* c, void* d, const int32_t* m_indices, int m_total, int n,
+                                              int k, int num_groups, void* stream) {
+  return contiguous_impl(false, a, sfa, b, sfb, c, d, m_indices, m_total, n, k, num_groups, stream);
+}
+
+dg_status dg_m_grouped_fp8_fp4_gemm_nt_contiguous(const void* a, const int32_t* sfa, const void* b,
+                                                  const int32_t* sfb, const void* c, void* d,
+                                                  const int32_t* m_indices, int m_total, int n, int k,
+                                                  int num_groups, void* stream) {
+  return contiguous_impl(true, a, sfa, b, sfb, c, d, m_indices, m_total, n, k, num_groups, stream);
+}
+
+dg_status dg_m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                                          void* d, const int32_t* masked_m, int num_groups, int max_m, int n, int k,
+                                          int expected_m, void* stream) {
+  if (num_groups <= 0 || num_groups > dg::kMaxMaskedGroups || max_m <= 0 || !masked_m || expected_m < 0)
+    return DG_ERR_INVALID_ARG;
+  dg_status st = check_common(a, sfa, b, sfb, nullptr, d, n, k);
+  if (st != DG_OK) return st;
+  Problem p{a, sfa, b, sfb, nullptr, d, nullptr, masked_m, max_m, n, k, num_groups, expected_m};
+  return run_gemm<false, dg::kMasked>(p, static_cast<cudaStream_t>(stream));
+}
+
+dg_status dg_quantize_fp8(const float* x, int rows, int cols, int block_rows, uint8_t* q, uint8_t* sf,
+                          void* stream) {
+  if (!x || !q || !sf || rows < 0 || cols <= 0 || cols % 128 != 0) return DG_ERR_INVALID_ARG;
+  if (block_rows != 1 && block_rows != 128) return DG_ERR_INVALID_ARG;
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(q) & 3u)) return DG_ERR_INVALID_ARG;
+  if (rows == 0) return DG_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int sms = std::max(1, device_sms());
+  if (block_rows == 1) {
+    const long long warps = (long long)rows * (cols / 128);
+    const int blocks = (int)std::min<long long>(ceil_div(warps * 32, 256), (long long)sms * 16);
+    dg::quant_fp8_1x128_kernel<<<blocks, 256, 0, s>>>(x, rows, cols, q, sf);
+  } else {
+    const long long nblk = ceil_div(rows, 128) * (cols / 128);
+    const int blocks = (int)std::min<long long>(nblk, (long long)sms * 8);
+    dg::quant_fp8_128x128_kernel<<<blocks, 256, 0, s>>>(x, rows, cols, q, sf);
+  }
+  if (cudaGetLastError() != cudaSuccess) return DG_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return DG_OK;
+}
+
+dg_status dg_quantize_fp4(const float* x, int rows, int cols, uint8_t* q, uint8_t* sf, void* stream) {
+  if (!x || !q || !sf || rows < 0 || cols <= 0 || cols % 32 != 0) return DG_ERR_INVALID_ARG;
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(q) & 3u)) return DG_ERR_INVALID_ARG;
+  if (rows == 0) return DG_OK;
+  const int sms = std::max(1, device_sms());
+  const long long thr = (long long)rows * (cols / 32) * 4;
+  const int blocks = (int)std::min<long long>(ceil_div(thr, 256), (long long)sms * 16);
+  dg::quant_fp4_1x32_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, rows, cols, q, sf);
+  if (cudaGetLastError() != cudaSuccess) return DG_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return DG_OK;
+}
+
+int64_t dg_packed_sf_words(int rows, int num_sf_cols) {
+  if (rows <= 0 || num_sf_cols <= 0) return 0;
+  return (int64_t)ceil_div(num_sf_cols, 4) * ceil_div(rows, 128) * 128;
+}
+
+dg_status dg_pack_sf(const uint8_t* sf, int rows, int num_sf_cols, int row_div, int32_t* packed, void* stream) {
+  if (!sf || !packed || rows <= 0 || num_sf_cols <= 0 || row_div <= 0) return DG_ERR_INVALID_ARG;
+  const long long total = dg_packed_sf_words(rows, num_sf_cols);
+  const int sms = std::max(1, device_sms());
+  const int blocks = (int)std::min<long long>(ceil_div(total, 256), (long long)sms * 16);
+  dg::pack_sf_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(sf, rows, num_sf_cols, row_div, packed);
+  if (cudaGetLastError() != cudaSuccess) return DG_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return DG_OK;
+}
+
+int dg_get_num_sms(void) { return num_sms(); }
+
+dg_status dg_set_num_sms(int n) {
+  if (n < 0) return DG_ERR_INVALID_ARG;
+  g_num_sms_override = n;
+  return DG_OK;
+}
+
+int dg_get_mk_alignment_for_contiguous_layout(void) { return dg::kBM; }
+
+dg_status dg_get_last_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DG_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, dg::g_error_word, sizeof(int)) != cudaSuccess) return DG_ERR_CUDA;
+  if (v != 0) {
+    int zero = 0;
+    if (cudaMemcpyToSymbol(dg::g_error_word, &zero, sizeof(int)) != cudaSuccess) return DG_ERR_CUDA;
+  }
+  return static_cast<dg_status>(v);
+}
+
+dg_status dg_debug_starved_wait(unsigned int limit_us, void* stream) {
+  dg::starved_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>((unsigned long long)limit_us * 1000ull);
+  if (cudaGetLastError() != cudaSuccess) return DG_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return DG_OK;
+}
+
+const char* dg_status_string(int status) {
+  switch (status) {
+    case DG_OK: return "DG_OK";
+    case DG_ERR_INVALID_ARG: return "DG_ERR_INVALID_ARG";
+    case DG_ERR_UNSUPPORTED: return "DG_ERR_UNSUPPORTED";
+    case DG_ERR_CUDA: return "DG_ERR_CUDA";
+    case DG_ERR_TIMEOUT: return "DG_ERR_TIMEOUT";
+    case DG_ERR_BAD_METADATA: return "DG_ERR_BAD_METADATA";
+    default: return "DG_ERR_UNKNOWN";
+  }
+}
+
+uint64_t dg_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+dg_status dg_query_dense_config(int m, int n, int k, int* block_n, int* splits, int* units, int* grid) {
+  if (m <= 0 || n <= 0 || k <= 0 || k % 128 != 0) return DG_ERR_INVALID_ARG;
+  const int sms = num_sms();
+  if (sms <= 0) return DG_ERR_CUDA;
+  Plan p = plan_gemm(ceil_div(m, dg::kBM), n, k, sms, m <= 1024);
+  if (block_n) *block_n = p.bn;
+  if (splits) *splits = p.splits;
+  if (units) *units = (int)p.units;
+  if (grid) *grid = p.grid;
+  return DG_OK;
+}
+
+int64_t dg_num_tiles(int m, int n, int block_m, int block_n) {
+  if (m <= 0 || n <= 0 || block_m <= 0 || block_n <= 0) return 0;
+  return ceil_div(m, block_m) * ceil_div(n, block_n);
+}
+
+void dg_shutdown(void) {
+  std::lock_guard<std::mutex> lock(g_ws_mutex);
+  int prev = 0;
+  cudaGetDevice(&prev);
+  for (auto& kv : g_ws) {
+    if (kv.second.ptr) {
+      cudaSetDevice(kv.first.first);
+      cudaStreamSynchronize(kv.first.second);
+      cudaFree(kv.second.ptr);
+    }
+  }
+  g_ws.clear();
+  cudaSetDevice(prev);
+}
+
+}  // extern "C"

@@ -1,0 +1,321 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.  Floating-point outputs are checked under the method's
+tolerances (tests/gpu_util.py); integer, byte and index work bit-exactly."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_util import (Dense, bf16_dev_to_f64, check_close, dev, host, quantize_groups_b)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dg():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    from moe_grouped_gemm_06_b200 import build
+    build.build()
+    import moe_grouped_gemm_06_b200 as dg
+    assert dg.dg_get_last_error() == 0
+    yield dg
+    assert dg.dg_get_last_error() == 0
+
+
+# ------------------------------------------------------------------ prep
+
+@pytest.mark.parametrize("rows,cols", [(1, 128), (300, 512)])
+def test_quantize_fp8_rowwise_bit_exact(dg, rows, cols):
+    x = synth.normal_f32(1000 + rows, (rows, cols)) * np.float32(5.0)
+    x[0, :128] = 0.0
+    if rows > 2:
+        x[1, 128:256] = np.float32(3e-39)      # subnormal block
+        x[2, :] *= np.float32(1e20)
+    q, e = oracle.quantize_fp8(x, 1)
+    tq = torch.empty((rows, cols), dtype=torch.uint8, device="cuda")
+    te = torch.empty((rows, cols // 128), dtype=torch.uint8, device="cuda")
+    dg.dg_quantize_fp8(dev(x), tq, te, 1)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(te), e)
+    assert np.array_equal(host(tq), q)
+
+
+def test_quantize_fp8_blockwise_bit_exact(dg):
+    rows, cols = 300, 384
+    x = synth.normal_f32(1100, (rows, cols))
+    q, e = oracle.quantize_fp8(x, 128)
+    tq = torch.empty((rows, cols), dtype=torch.uint8, device="cuda")
+    te = torch.empty(e.shape, dtype=torch.uint8, device="cuda")
+    dg.dg_quantize_fp8(dev(x), tq, te, 128)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(te), e)
+    assert np.array_equal(host(tq), q)
+
+
+def test_quantize_fp4_bit_exact(dg):
+    rows, cols = 70, 256
+    x = synth.normal_f32(1200, (rows, cols))
+    x[3, :32] = 0.0
+    q, e = oracle.quantize_fp4(x, 32)
+    tq = torch.empty((rows, cols // 2), dtype=torch.uint8, device="cuda")
+    te = torch.empty((rows, cols // 32), dtype=torch.uint8, device="cuda")
+    dg.dg_quantize_fp4(dev(x), tq, te)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(te), e)
+    assert np.array_equal(host(tq), q)
+
+
+@pytest.mark.parametrize("rows,ng,row_div", [(300, 7, 1), (128, 4, 1), (2112, 56, 128), (1, 1, 1)])
+def test_pack_sf_bit_exact(dg, rows, ng, row_div):
+    e = synth.junk_bytes(1300 + rows, ((rows + row_div - 1) // row_div, ng))
+    want = oracle.pack_sf(e, rows, row_div=row_div)
+    out = torch.full((dg.dg_packed_sf_words(rows, ng),), -1, dtype=torch.int32, device="cuda")
+    dg.dg_pack_sf(dev(e), rows, out, row_div=row_div)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(out), want.ravel())
+
+
+# ------------------------------------------------------------------ dense
+
+@pytest.mark.parametrize("M,N,K,with_c", [
+    (128, 512, 1024, False),    # the small worked configuration (C = 0)
+    (200, 328, 384, True),      # ragged M and N tails, K of three blocks
+    (1100, 520, 512, True),     # several m-blocks, no split-K, ragged tails
+    (64, 2112, 7168, True),     # split-K path
+    (3, 64, 256, True),         # tiny M
+])
+def test_dense_matches_oracle(dg, M, N, K, with_c):
+    p = Dense(2000 + M + N, M, N, K, with_c=with_c).upload()
+    d = p.run(dg)
+    stats = check_close(d, p.ref(), f"dense {M}x{N}x{K}")
+    assert stats["n"] == M * N
+
+
+def test_dense_long_k_accumulation(dg):
+    # K = 16384: 128 scaled K-blocks accumulated in FP32 inside TMEM
+    p = Dense(2100, 128, 256, 16384, with_c=False).upload()
+    check_close(p.run(dg), p.ref(), "dense K=16384")
+
+
+def test_dense_in_place_c_equals_d(dg):
+    p = Dense(2200, 256, 256, 512, with_c=True).upload()
+    p.t_d.copy_(p.t_c)
+    dg.dg_fp8_gemm_nt(p.t_a, p.t_sfa, p.t_b, p.t_sfb, p.t_d, p.t_d)
+    torch.cuda.synchronize()
+    check_close(bf16_dev_to_f64(p.t_d), p.ref(), "dense in-place")
+
+
+@pytest.mark.parametrize("M", [128, 2048])
+def test_dense_scale_doubling_is_bit_exact(dg, M):
+    # C = 0 and a single non-zero K-block: raising that block's A scale by
+    # one must double every output exactly (scaling by 2 commutes with the
+    # bf16 rounding away from overflow and underflow).
+    N, K = 256, 512
+    p = Dense(2300 + M, M, N, K, with_c=False)
+    p.qa[:, :128] = 0
+    p.qa[:, 256:] = 0
+    p.sfa = oracle.pack_sf(p.ea, M)
+    p.upload()
+    d1 = p.run(dg)
+    ea2 = p.ea.copy()
+    ea2[:, 1] += 1
+    p.t_sfa = dev(oracle.pack_sf(ea2, M))
+    d2 = p.run(dg)
+    assert np.array_equal(d2, 2.0 * d1)
+    assert np.count_nonzero(d1) > 0.9 * d1.size
+
+
+def test_dense_full_size_sampled(dg):
+    # every dense shape of the DeepSeek-V3 projection sweep, sampled outputs
+    for (N, K) in synth.DENSE_NK:
+        xb = synth.normal_f32(3000 + N + K, (N, K))
+        for M in synth.DENSE_M:
+            print(f"dense full size {M}x{N}x{K}: {dg.dg_query_dense_config(M, N, K)}", flush=True)
+            p = Dense(3100 + M + N + K, M, N, K, with_c=True, xb=xb).upload()
+            d = p.run(dg)
+            pm, pn = synth.sample_points(3200 + M, np.arange(M), N, 2048)
+            check_close(d[pm, pn], p.ref_points(pm, pn), f"dense {M}x{N}x{K}")
+            del p
+            torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------------------ contiguous
+
+def _contiguous_case(seed, G, lo, hi, N, K, fp4=False, with_c=True):
+    rows, mi = synth.contiguous_layout(seed, G, lo, hi)
+    M = mi.size
+    xa = synth.normal_f32(seed + 1, (M, K))
+    qa, ea = oracle.quantize_fp8(xa, 1)
+    pad = mi < 0
+    qa[pad] = synth.junk_bytes(seed + 2, (int(pad.sum()), K))   # junk incl. NaN codes
+    qa[pad, ::7] = 0x7F
+    ea[pad] = synth.junk_bytes(seed + 3, (int(pad.sum()), K // 128))
+    qb, eb, sfb = quantize_groups_b(seed + 10, G, N, K, fp4=fp4)
+    c = synth.normal_bf16_bits(seed + 4, (M, N)) if with_c else None
+    return dict(rows=rows, mi=mi, M=M, qa=qa, ea=ea, sfa=oracle.pack_sf(ea, M), qb=qb, eb=eb, sfb=sfb, c=c)
+
+
+def _run_contiguous(dg, cs, N, fp4=False):
+    d = torch.empty((cs["M"], N), dtype=torch.int16, device="cuda")
+    fn = dg.dg_m_grouped_fp8_fp4_gemm_nt_contiguous if fp4 else dg.dg_m_grouped_fp8_gemm_nt_contiguous
+    c = dev(cs["c"].view(np.int16)) if cs["c"] is not None else None
+    fn(dev(cs["qa"]), dev(cs["sfa"]), dev(cs["qb"]), dev(cs["sfb"]), c, d, dev(cs["mi"]))
+    torch.cuda.synchronize()
+    return bf16_dev_to_f64(d)
+
+
+@pytest.mark.parametrize("fp4", [False, True])
+def test_contiguous_matches_oracle(dg, fp4):
+    N, K = 384, 512
+    cs = _contiguous_case(4000 + fp4, 4, 50, 300, N, K, fp4=fp4)
+    d = _run_contiguous(dg, cs, N, fp4=fp4)
+    ref = oracle.gemm_contiguous(cs["qa"], cs["ea"], cs["qb"], cs["eb"], cs["mi"], c=cs["c"], b_fp4=fp4)
+    valid = cs["mi"] >= 0
+    check_close(d[valid], ref[valid], "contiguous")
+    # and each group equals the dense call on its own rows
+    for g in range(4):
+        sel = np.nonzero(cs["mi"] == g)[0]
+        assert sel.size == cs["rows"][g]
+
+
+@pytest.mark.parametrize("N,K", synth.GROUPED_NK)
+def test_contiguous_full_size_sampled(dg, N, K):
+    cs = _contiguous_case(4100 + N, 8, 6000, 10000, N, K)
+    d = _run_contiguous(dg, cs, N)
+    valid_rows = np.nonzero(cs["mi"] >= 0)[0]
+    pm, pn = synth.sample_points(4200 + N, valid_rows, N, 4096)
+    ref = np.empty(pm.size)
+    for g in range(8):
+        sel = cs["mi"][pm] == g
+        ref[sel] = oracle.gemm_points(cs["qa"], cs["ea"], cs["qb"][g], cs["eb"][g], pm[sel], pn[sel], c=cs["c"])
+    check_close(d[pm, pn], ref, f"contiguous {N}x{K}")
+
+
+# ------------------------------------------------------------------ masked
+
+SENTINEL = 0x7FC1  # a bf16 NaN pattern no GEMM result can produce
+
+
+_B_CACHE = {}
+
+
+def _grouped_b(seed, G, N, K):
+    key = (seed, G, N, K)
+    if key not in _B_CACHE:
+        _B_CACHE.clear()
+        _B_CACHE[key] = quantize_groups_b(seed, G, N, K)
+    return _B_CACHE[key]
+
+
+def _masked_case(seed, G, max_m, N, K, masked_m, b_seed=None):
+    xa = synth.normal_f32(seed, (G * max_m, K))
+    qa, ea = oracle.quantize_fp8(xa, 1)
+    qa = qa.reshape(G, max_m, K)
+    ea = ea.reshape(G, max_m, K // 128)
+    for g in range(G):                           # junk beyond the valid rows
+        v = min(int(masked_m[g]), max_m)
+        qa[g, v:] = synth.junk_bytes(seed + 100 + g, (max_m - v, K))
+    sfa = np.concatenate([oracle.pack_sf(ea[g], max_m).ravel() for g in range(G)])
+    qb, eb, sfb = _grouped_b(seed + 1000 if b_seed is None else b_seed, G, N, K)
+    return qa, ea, sfa, qb, eb, sfb
+
+
+def _run_masked(dg, G, max_m, N, qa, sfa, qb, sfb, masked_m, expected_m=0):
+    d = torch.full((G, max_m, N), SENTINEL, dtype=torch.int16, device="cuda")
+    dg.dg_m_grouped_fp8_gemm_nt_masked(dev(qa), dev(sfa), dev(qb), dev(sfb), d, dev(masked_m.astype(np.int32)),
+                                       expected_m=expected_m)
+    torch.cuda.synchronize()
+    return d
+
+
+def test_masked_matches_oracle_and_leaves_rows(dg):
+    G, max_m, N, K = 6, 256, 384, 512
+    mm = np.array([0, 1, 127, 128, 200, 256], np.int32)
+    qa, ea, sfa, qb, eb, sfb = _masked_case(5000, G, max_m, N, K, mm)
+    d = _run_masked(dg, G, max_m, N, qa, sfa, qb, sfb, mm)
+    bits = host(d).view(np.uint16)
+    ref = oracle.gemm_masked(qa, ea, qb, eb, mm)
+    dd = bf16_dev_to_f64(d)
+    for g in range(G):
+        v = int(mm[g])
+        assert np.all(bits[g, v:] == SENTINEL), f"group {g}: rows >= masked_m were written"
+        if v:
+            check_close(dd[g, :v], ref[g, :v], f"masked group {g}")
+
+
+def test_masked_count_above_max_is_clamped_and_reported(dg):
+    G, max_m, N, K = 2, 128, 128, 256
+    mm = np.array([300, 5], np.int32)
+    qa, ea, sfa, qb, eb, sfb = _masked_case(5100, G, max_m, N, K, np.minimum(mm, max_m))
+    d = _run_masked(dg, G, max_m, N, qa, sfa, qb, sfb, mm)
+    assert dg.dg_get_last_error() == -5
+    ref = oracle.gemm_masked(qa, ea, qb, eb, mm)
+    dd = bf16_dev_to_f64(d)
+    check_close(dd[0], ref[0], "masked clamped group")
+    assert np.all(host(d).view(np.uint16)[1, 5:] == SENTINEL)
+
+
+@pytest.mark.parametrize("N,K", synth.GROUPED_NK)
+@pytest.mark.parametrize("expected_m", [16, 64, 128])
+def test_masked_full_size_sampled(dg, expected_m, N, K):
+    G, max_m = 32, 256
+    mm = synth.masked_counts(5200 + expected_m, G, expected_m, max_m)
+    qa, ea, sfa, qb, eb, sfb = _masked_case(5300 + expected_m + N, G, max_m, N, K, mm, b_seed=5500 + N)
+    d = _run_masked(dg, G, max_m, N, qa, sfa, qb, sfb, mm, expected_m=expected_m)
+    rows_valid = torch.arange(max_m, device="cuda")[None, :] < dev(mm)[:, None]
+    untouched = (d == SENTINEL).all(dim=2)
+    assert bool(untouched[~rows_valid].all()), "rows >= masked_m were written"
+    dd = bf16_dev_to_f64(d)
+    valid = [(g, m) for g in range(G) for m in range(int(mm[g]))]
+    rng = synth.rng(5400 + expected_m)
+    pick = rng.choice(len(valid), size=min(2048, len(valid)), replace=False)
+    pn = rng.integers(0, N, size=pick.size)
+    ref = np.empty(pick.size)
+    got = np.empty(pick.size)
+    for i, (j, n) in enumerate(zip(pick, pn)):
+        g, m = valid[j]
+        got[i] = dd[g, m, n]
+    for g in range(G):
+        sel = np.array([valid[j][0] == g for j in pick])
+        if sel.any():
+            ms = np.array([valid[j][1] for j in pick[sel]])
+            ref[sel] = oracle.gemm_points(qa[g], ea[g], qb[g], eb[g], ms, pn[sel])
+    check_close(got, ref, f"masked {N}x{K} em={expected_m}")
+
+
+# ------------------------------------------------------------------ FP8 x FP4
+
+@pytest.mark.parametrize("M,N,K", [(256, 384, 512), (200, 136, 256), (64, 2112, 2048)])
+def test_fp8_fp4_dense_matches_oracle(dg, M, N, K):
+    p = Dense(6000 + M + N, M, N, K, with_c=True, fp4=True).upload()
+    check_close(p.run(dg), p.ref(), f"fp8xfp4 {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("N,K", synth.GROUPED_NK)
+def test_fp8_fp4_full_size_sampled(dg, N, K):
+    p = Dense(6100 + N, 4096, N, K, with_c=True, fp4=True).upload()
+    d = p.run(dg)
+    pm, pn = synth.sample_points(6200 + N, np.arange(4096), N, 2048)
+    check_close(d[pm, pn], p.ref_points(pm, pn), f"fp8xfp4 4096x{N}x{K}")
+
+
+# ------------------------------------------------------------------ failure paths
+
+def test_starved_wait_times_out_and_context_survives(dg):
+    dg.dg_debug_starved_wait(20000)   # 20 ms
+    assert dg.dg_get_last_error() == -4
+    assert dg.dg_get_last_error() == 0
+    p = Dense(7000, 128, 128, 256).upload()
+    check_close(p.run(dg), p.ref(), "after timeout")
+
+
+def test_contiguous_group_index_out_of_range_is_reported(dg):
+    N, K = 128, 256
+    cs = _contiguous_case(7100, 2, 100, 120, N, K)
+    mi = cs["mi"].copy()
+    mi[128:256][mi[128:256] >= 0] = 7      # second block claims group 7 of 2
+    cs["mi"] = mi
+    _run_contiguous(dg, cs, N)
+    assert dg.dg_get_last_error() == -5
