@@ -1,0 +1,442 @@
+#!/usr/bin/env python
+"""Benchmark of the fine-grained-scaled FP8 GEMM  D = C + A @ B^T  on B200.
+
+One step = one pass over the dense NT FP8 sweep of DeepSeek-V3 projection
+shapes: M in {64, 128, 4096} x (N, K) in {(2112,7168), (24576,1536),
+(32768,512), (7168,16384), (4096,7168), (7168,2048)}, A/B ~ N(0,1) quantised
+with 1x128 / 128x128 UE8M0 scales, C ~ N(0,1) bf16 (synthetic, seeded).
+Each GEMM call is timed with CUDA events on its stream after an L2 flush (a
+256 MB write), so no call reads its inputs from a warm L2.
+
+  value   = total FLOPs of the sweep (all ranks) / device time (max over ranks)
+  e2e     = the same sweep through the C ABI from pinned HOST buffers, the
+            host->device copies of A, SFA, B, SFB, C and the device->host copy
+            of D inside the timed region
+  roofline: the dominant kernel (largest share of step time) against the
+            measured peak (MEASURED_PEAKS.json), FP8 peak = measured bf16 x 2
+  cpu_baseline: the CPU oracle on a bounded sample of the same sweep
+
+Multi-GPU: the sweep does not shard (replicas only); with --gpus N each rank
+runs the full sweep on its own GPU and value aggregates all ranks ("weak").
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                  [--shape M,N,K] [--no-e2e] [--no-cpu]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "FP8 TFLOPS per shape & % of B200 dense FP8 peak (GB/s vs HBM for decode)"
+UNIT = "TFLOPS"
+DENSE_NK = [(2112, 7168), (24576, 1536), (32768, 512), (7168, 16384), (4096, 7168), (7168, 2048)]
+DENSE_M = [64, 128, 4096]
+FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_PER_BF16 = 2.0  # nominal dense FP8 : BF16 tensor throughput (4.5 : 2.25 PFLOP/s)
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--shape", default=None, help="run one M,N,K shape instead of the sweep")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+def shapes_from(args):
+    if args.shape:
+        m, n, k = (int(v) for v in args.shape.split(","))
+        return [(m, n, k)]
+    return [(m, n, k) for (n, k) in DENSE_NK for m in DENSE_M]
+
+
+def flops(m, n, k):
+    return 2.0 * m * n * k
+
+
+def alg_bytes(m, n, k, with_c=True):
+    """A + SFA + B + SFB (128x128 block codes) + D (+ C), in bytes."""
+    sfa = m * (k // 128)
+    sfb = ((n + 127) // 128) * (k // 128)
+    return m * k + sfa + n * k + sfb + 2 * m * n + (2 * m * n if with_c else 0)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha1()
+    for name in ("dg_gemm.cuh", "dg_ptx.cuh", "dg_lib.cu"):
+        with open(os.path.join(ROOT, "moe_grouped_gemm_06_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    src = kernel_source_hash()
+    for line in open(path):
+        parts = line.split()
+        if len(parts) >= 3 and not line.startswith("#") and parts[0] == src and parts[1] == workload:
+            return float(parts[2])
+    return None
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        rows = []
+        with open(self.file.name) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.file.name)
+        if not rows:
+            return None
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        power = [num(r[3]) for r in rows if num(r[3]) is not None]
+        pmax = max(power) if power else 0.0
+        loaded = [num(r[1]) for r in rows if num(r[3]) is not None and num(r[3]) >= 0.5 * pmax]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(loaded or sm) if sm else None,
+                "sm_max_mhz": num(rows[0][2]), "power_w_max": pmax, "samples": len(rows),
+                "reasons": reasons}
+
+
+# ---------------------------------------------------------------- inputs
+
+def make_inputs(dg, torch, m, n, k, gen):
+    """Device-resident inputs, quantised and packed by the library's own kernels."""
+    dev = "cuda"
+    xa = torch.randn((m, k), generator=gen, device=dev, dtype=torch.float32)
+    xb = torch.randn((n, k), generator=gen, device=dev, dtype=torch.float32)
+    a = torch.empty((m, k), dtype=torch.uint8, device=dev)
+    b = torch.empty((n, k), dtype=torch.uint8, device=dev)
+    ea = torch.empty((m, k // 128), dtype=torch.uint8, device=dev)
+    eb = torch.empty(((n + 127) // 128, k // 128), dtype=torch.uint8, device=dev)
+    dg.dg_quantize_fp8(xa, a, ea, 1)
+    dg.dg_quantize_fp8(xb, b, eb, 128)
+    sfa = torch.empty(dg.dg_packed_sf_words(m, k // 128), dtype=torch.int32, device=dev)
+    sfb = torch.empty(dg.dg_packed_sf_words(n, k // 128), dtype=torch.int32, device=dev)
+    dg.dg_pack_sf(ea, m, sfa, row_div=1)
+    dg.dg_pack_sf(eb, n, sfb, row_div=128)
+    c = torch.randn((m, n), generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    d = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+    del xa, xb, ea, eb
+    return {"a": a, "sfa": sfa, "b": b, "sfb": sfb, "c": c, "d": d}
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_prepare(shapes, seed=0):
+    """Host inputs for the CPU oracle: for each shape, R = min(threads, M)
+    rows of A (so every OpenMP thread of the oracle's row loop has a row)
+    and the whole B, quantised by the oracle; B is shared per (N, K)."""
+    import oracle
+    import synth
+    oracle.build()
+    threads = oracle.num_threads()
+    bcache, prepared = {}, []
+    for (m, n, k) in shapes:
+        if (n, k) not in bcache:
+            bcache[(n, k)] = oracle.quantize_fp8(synth.normal_f32(seed + n + k, (n, k)), 128)
+        qb, eb = bcache[(n, k)]
+        r = min(threads, m)
+        qa, ea = oracle.quantize_fp8(synth.normal_f32(seed + m + n + k, (r, k)), 1)
+        c = synth.normal_bf16_bits(seed + 7 + m, (r, n))
+        prepared.append((r, n, k, qa, ea, qb, eb, c))
+    return prepared, threads
+
+
+def oracle_step(prepared):
+    """One pass of the CPU oracle over the sample; returns its FLOPs."""
+    import oracle
+    f = 0.0
+    for (r, n, k, qa, ea, qb, eb, c) in prepared:
+        oracle.gemm(qa, ea, qb, eb, c=c)
+        f += 2.0 * r * n * k
+    return f
+
+
+def oracle_sample_text(prepared, threads, passes):
+    rows = sorted({p[0] for p in prepared})
+    return (f"{passes} pass(es) over the {len(prepared)} sweep shapes; per shape R = min(threads, M) "
+            f"= {rows} full output rows (all N columns, full K); CPU FP64 oracle, {threads} OpenMP threads")
+
+
+def oracle_sample_tflops(shapes, seconds):
+    """The CPU oracle, as it stands, on a bounded sample of the sweep (about
+    `seconds` of wall time).  Returns (TFLOPS, threads, description)."""
+    prepared, threads = oracle_prepare(shapes)
+    total, passes = 0.0, 0
+    t0 = time.perf_counter()
+    while True:
+        total += oracle_step(prepared)
+        passes += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return total / dt / 1e12, threads, oracle_sample_text(prepared, threads, passes)
+
+
+def reference_arm(args, rank):
+    """--impl reference: the CPU oracle timed per step on a bounded sample of
+    the same sweep (rank 0 only; other ranks exit without work)."""
+    if rank != 0:
+        return
+    shapes = shapes_from(args)
+    prepared, threads = oracle_prepare(shapes)
+    for _ in range(args.warmup):
+        oracle_step(prepared)
+    t0 = time.perf_counter()
+    total = 0.0
+    for _ in range(args.steps):
+        total += oracle_step(prepared)
+    dt = time.perf_counter() - t0
+    value = total / dt / 1e12
+    sample = "per step: " + oracle_sample_text(prepared, threads, 1)
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": "dense NT FP8 sweep (sampled rows), DeepSeek-V3 shapes", "shapes": len(shapes)},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- main
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        reference_arm(args, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import moe_grouped_gemm_06_b200 as dg
+
+    torch.cuda.set_device(local_rank)
+    use_dist = world > 1
+    if use_dist:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
+
+    shapes = shapes_from(args)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(1234 + rank)
+    inputs = [make_inputs(dg, torch, m, n, k, gen) for (m, n, k) in shapes]
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+
+    def call(x):
+        dg.dg_fp8_gemm_nt(x["a"], x["sfa"], x["b"], x["sfb"], x["c"], x["d"], stream=stream)
+
+    def sweep(events):
+        for i, x in enumerate(inputs):
+            flush.zero_()
+            if events is not None:
+                events[i][0].record(stream)
+            call(x)
+            if events is not None:
+                events[i][1].record(stream)
+
+    for _ in range(max(args.warmup, 1)):
+        sweep(None)
+    assert dg.dg_get_last_error() == 0, "device error during warm-up"
+
+    events = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in shapes] for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank)
+    if use_dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    launches0 = dg.dg_launch_count()
+    wall0 = time.perf_counter()
+    for s in range(args.steps):
+        sweep(events[s])
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    launches = dg.dg_launch_count() - launches0
+    if use_dist:
+        dist.barrier()
+    clocks = sampler.stop()
+    assert dg.dg_get_last_error() == 0, "device error during timing"
+
+    per_shape_ms = [sum(events[s][i][0].elapsed_time(events[s][i][1]) for s in range(args.steps)) / args.steps
+                    for i in range(len(shapes))]
+    step_ms = sum(per_shape_ms)
+    t = torch.tensor([step_ms], dtype=torch.float64, device="cuda")
+    if use_dist:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    step_ms_max = float(t.item())
+
+    sweep_flops = sum(flops(*s) for s in shapes)
+    value = world * sweep_flops / (step_ms_max * 1e-3) / 1e12
+
+    peaks, peak_kind = load_peaks()
+    fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
+    hbm = peaks["hbm_gbs"]
+    ridge = fp8_peak * 1e12 / (hbm * 1e9)
+    per_shape = []
+    for (m, n, k), ms in zip(shapes, per_shape_ms):
+        f, by = flops(m, n, k), alg_bytes(m, n, k)
+        tf = f / (ms * 1e-3) / 1e12
+        gbs = by / (ms * 1e-3) / 1e9
+        bound = "tensor" if f / by >= ridge else "hbm"
+        frac = tf / fp8_peak if bound == "tensor" else gbs / hbm
+        per_shape.append({"m": m, "n": n, "k": k, "us": round(ms * 1e3, 2), "tflops": round(tf, 1),
+                          "gbs": round(gbs, 1), "bound": bound, "frac": round(frac, 4)})
+
+    dom = max(range(len(shapes)), key=lambda i: per_shape_ms[i])
+    (dm, dn, dk) = shapes[dom]
+    dom_bound = per_shape[dom]["bound"]
+    dom_workload = f"dense_{dm}x{dn}x{dk}"
+    if dom_bound == "tensor":
+        achieved = flops(dm, dn, dk) / (per_shape_ms[dom] * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(fp8_peak, 1),
+                    "unit": "TFLOP/s", "frac": round(achieved / fp8_peak, 4)}
+    else:
+        achieved = alg_bytes(dm, dn, dk) / (per_shape_ms[dom] * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                    "frac": round(achieved / hbm, 4)}
+    roofline["traffic"] = recorded_traffic(dom_workload)
+    roofline["kernel"] = f"gemm_kernel on {dom_workload} ({per_shape_ms[dom] / step_ms * 100:.0f}% of step time)"
+    roofline["peak_source"] = (f"{peak_kind}: FP8 = bf16 burst {peaks['bf16_tflops']} x {FP8_PER_BF16} "
+                               f"(nominal FP8:BF16 ratio); HBM {hbm} GB/s")
+
+    # ---- end to end through the C ABI from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        host = []
+        h2d = d2h = 0
+        for x in inputs:
+            hx = {key: x[key].cpu().pin_memory() for key in ("a", "sfa", "b", "sfb", "c")}
+            hx["d"] = torch.empty(x["d"].shape, dtype=x["d"].dtype).pin_memory()
+            host.append(hx)
+            h2d += sum(hx[key].numel() * hx[key].element_size() for key in ("a", "sfa", "b", "sfb", "c"))
+            d2h += hx["d"].numel() * hx["d"].element_size()
+
+        def e2e_step():
+            for x, hx in zip(inputs, host):
+                for key in ("a", "sfa", "b", "sfb", "c"):
+                    x[key].copy_(hx[key], non_blocking=True)
+                call(x)
+                hx["d"].copy_(x["d"], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2e_steps = max(1, min(args.steps, 5))
+        if use_dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1) / e2e_steps
+        te = torch.tensor([ems], dtype=torch.float64, device="cuda")
+        if use_dist:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": round(world * sweep_flops / (float(te.item()) * 1e-3) / 1e12, 2), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": round(float(te.item()), 3)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        v, cores, sample = oracle_sample_tflops(shapes, args.cpu_seconds)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(step_ms_max, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+            "config": {"workload": ("dense NT FP8 sweep, DeepSeek-V3 shapes M in {64,128,4096} x (N,K) in "
+                                    "{(2112,7168),(24576,1536),(32768,512),(7168,16384),(4096,7168),(7168,2048)}"
+                                    if not args.shape else f"dense NT FP8 {args.shape}"),
+                       "shapes": len(shapes), "accumulate": "f32 (TMEM)", "out": "bf16", "c": "N(0,1) bf16",
+                       "scales": "UE8M0 1x128 (A), 128x128 (B)",
+                       "l2": "flushed before every timed GEMM call (256 MB write, not timed)",
+                       "parallelism": f"replicas x{world}", "wall_s_timed_region": round(wall, 3)},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
+            "clocks": clocks, "per_shape": per_shape,
+        }
+        print(json.dumps(line), flush=True)
+    if use_dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
