@@ -56,6 +56,7 @@
 #ifndef DG_H_
 #define DG_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -69,8 +70,10 @@ typedef enum {
   DG_ERR_CUDA = -3,          /* a CUDA runtime call or launch failed          */
   DG_ERR_TIMEOUT = -4,       /* a device wait ran past its limit (reported by
                                 dg_get_last_error)                            */
-  DG_ERR_BAD_METADATA = -5   /* masked_m outside [0, max_m] or m_indices >=
+  DG_ERR_BAD_METADATA = -5,  /* masked_m outside [0, max_m] or m_indices >=
                                 num_groups, seen on the device                */
+  DG_ERR_SCRATCH_LIMIT = -6  /* dg_fp8_gemm_nt_noalloc: the problem needs more
+                                split-K scratch than the fixed array holds    */
 } dg_status;
 
 /* ---------------------------------------------------------------- GEMMs */
@@ -118,6 +121,34 @@ dg_status dg_m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa, con
                                           const int32_t* sfb, void* d, const int32_t* masked_m,
                                           int num_groups, int max_m, int n, int k, int expected_m,
                                           void* stream);
+
+/* Dense NT FP8 GEMM that allocates no memory.  The pages have no counterpart
+ * of this call; it exists for callers that cannot allocate device memory at
+ * call time -- for example code running under another framework's memory
+ * manager, a serving loop whose memory is fixed up front, or a library whose
+ * own rule forbids cudaMalloc/cudaFree on the hot path (they can synchronise
+ * the device and they fail when memory is exhausted).
+ *
+ * Arguments, results and errors are those of dg_fp8_gemm_nt.  When the host
+ * heuristic splits K (small m), the FP32 partial sums go to one fixed device
+ * array of dg_noalloc_scratch_bytes() = 32 MiB that is part of this library's
+ * device image: every GPU that loads the library holds it until the process
+ * exits.  A problem whose split needs more than that (splits * m * n * 4
+ * bytes) returns DG_ERR_SCRATCH_LIMIT before anything is launched.  Nothing
+ * in the array has to start at zero: every partial that is read is first
+ * written by the same call.
+ *
+ * All calls on a device share the array and it keeps the last call's
+ * contents, so two calls whose kernels overlap on the GPU (different streams,
+ * or different host threads without ordering) race and give wrong results;
+ * order them on one stream.  The first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture. */
+dg_status dg_fp8_gemm_nt_noalloc(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                                 const void* c, void* d, int m, int n, int k, void* stream);
+
+/* Size in bytes of the fixed scratch array used by dg_fp8_gemm_nt_noalloc. */
+size_t dg_noalloc_scratch_bytes(void);
 
 /* FP8 x FP4 dense NT GEMM: as dg_fp8_gemm_nt but
  *   b    e2m1 [n][k/2] (two codes per byte, low nibble = even k)

@@ -19,7 +19,7 @@ import torch
 
 __all__ = [
     "DGError", "lib", "dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
-    "dg_m_grouped_fp8_gemm_nt_masked", "dg_fp8_fp4_gemm_nt", "dg_m_grouped_fp8_fp4_gemm_nt_contiguous",
+    "dg_m_grouped_fp8_gemm_nt_masked", "dg_fp8_gemm_nt_noalloc", "dg_noalloc_scratch_bytes", "dg_fp8_fp4_gemm_nt", "dg_m_grouped_fp8_fp4_gemm_nt_contiguous",
     "dg_quantize_fp8", "dg_quantize_fp4", "dg_pack_sf", "dg_packed_sf_words", "dg_get_num_sms",
     "dg_set_num_sms", "dg_get_mk_alignment_for_contiguous_layout", "dg_get_last_error",
     "dg_debug_starved_wait", "dg_launch_count", "dg_query_dense_config", "dg_num_tiles", "dg_shutdown",
@@ -39,6 +39,8 @@ SYMBOLS = {
                                                    _INT, _VP]),
     "dg_m_grouped_fp8_gemm_nt_masked": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _I32P, _INT, _INT, _INT, _INT, _INT,
                                                _VP]),
+    "dg_fp8_gemm_nt_noalloc": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _INT, _INT, _INT, _VP]),
+    "dg_noalloc_scratch_bytes": (ctypes.c_size_t, []),
     "dg_fp8_fp4_gemm_nt": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _INT, _INT, _INT, _VP]),
     "dg_m_grouped_fp8_fp4_gemm_nt_contiguous": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _I32P, _INT, _INT,
                                                        _INT, _INT, _VP]),
@@ -115,6 +117,21 @@ def dg_fp8_gemm_nt(a, sfa, b, sfb, c, d, stream=None) -> None:
     n = b.shape[0]
     _check(lib().dg_fp8_gemm_nt(_p(a), _p(sfa), _p(b), _p(sfb), _p(c), _p(d), m, n, k, _stream(stream)),
            "dg_fp8_gemm_nt")
+
+
+def dg_fp8_gemm_nt_noalloc(a, sfa, b, sfb, c, d, stream=None) -> None:
+    """As dg_fp8_gemm_nt, for callers that cannot allocate device memory at
+    call time: split-K partials use the library's fixed 32 MiB device array
+    (dg_noalloc_scratch_bytes()).  Calls that overlap on the GPU share that
+    array and race; the first call on a device must precede stream capture."""
+    m, k = a.shape
+    n = b.shape[0]
+    _check(lib().dg_fp8_gemm_nt_noalloc(_p(a), _p(sfa), _p(b), _p(sfb), _p(c), _p(d), m, n, k, _stream(stream)),
+           "dg_fp8_gemm_nt_noalloc")
+
+
+def dg_noalloc_scratch_bytes() -> int:
+    return int(lib().dg_noalloc_scratch_bytes())
 
 
 def dg_fp8_fp4_gemm_nt(a, sfa, b, sfb, c, d, stream=None) -> None:

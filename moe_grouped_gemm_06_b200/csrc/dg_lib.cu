@@ -203,8 +203,11 @@ struct Problem {
   int expected_m;  // masked hint
 };
 
+// fixed_ws / fixed_ws_bytes: when given, split-K partials go to this caller-
+// provided device buffer instead of the per-stream workspace, and a plan that
+// needs more than fixed_ws_bytes is rejected with DG_ERR_SCRATCH_LIMIT.
 template <bool FP4, int LAYOUT>
-dg_status run_gemm(const Problem& p, cudaStream_t s) {
+dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, size_t fixed_ws_bytes = 0) {
   const int sms = num_sms();
   if (sms <= 0) return DG_ERR_CUDA;
   const long long m_blocks = ceil_div(p.rows, dg::kBM);
@@ -247,8 +250,14 @@ dg_status run_gemm(const Problem& p, cudaStream_t s) {
   args.sfb_words = args.sfb_group_words * ((LAYOUT == dg::kDense) ? 1 : p.groups);
 
   if (plan.splits > 1) {
-    args.ws = workspace((size_t)plan.splits * p.rows * p.n * sizeof(float), s);
-    if (!args.ws) return DG_ERR_CUDA;
+    const size_t need = (size_t)plan.splits * p.rows * p.n * sizeof(float);
+    if (fixed_ws != nullptr) {
+      if (need > fixed_ws_bytes) return DG_ERR_SCRATCH_LIMIT;
+      args.ws = fixed_ws;
+    } else {
+      args.ws = workspace(need, s);
+      if (!args.ws) return DG_ERR_CUDA;
+    }
   }
 
   const int ga = (LAYOUT == dg::kMasked) ? p.groups : 1;
@@ -304,6 +313,56 @@ dg_status dg_fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const
   Problem p{a, sfa, b, sfb, c, d, nullptr, nullptr, m, n, k, 1, 0};
   return run_gemm<false, dg::kDense>(p, static_cast<cudaStream_t>(stream));
 }
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- no-alloc
+//
+// Scratch of dg_fp8_gemm_nt_noalloc: one fixed array per device, part of
+// this library's device image, so it exists on every GPU that loads the
+// library until the process exits.  All calls on a device share it.
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+}  // namespace
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+namespace {
+std::mutex g_noalloc_mutex;
+float* g_noalloc_addr[64] = {};
+
+// Device address of g_noalloc_scratch on the current device.  Host code
+// only holds a stand-in symbol for the array, so the address is looked up
+// once per device, with that device current, and cached.
+dg_status noalloc_scratch(float** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DG_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return DG_ERR_CUDA;
+    g_noalloc_addr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_addr[dev];
+  return DG_OK;
+}
+}  // namespace
+
+extern "C" {
+
+dg_status dg_fp8_gemm_nt_noalloc(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                                 const void* c, void* d, int m, int n, int k, void* stream) {
+  if (m < 0) return DG_ERR_INVALID_ARG;
+  dg_status st = check_common(a, sfa, b, sfb, c, d, n, k);
+  if (st != DG_OK) return st;
+  if (m == 0) return DG_OK;
+  float* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != DG_OK) return st;
+  Problem p{a, sfa, b, sfb, c, d, nullptr, nullptr, m, n, k, 1, 0};
+  return run_gemm<false, dg::kDense>(p, static_cast<cudaStream_t>(stream), scratch, kNoAllocScratchBytes);
+}
+
+size_t dg_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
 
 dg_status dg_fp8_fp4_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, const void* c,
                              void* d, int m, int n, int k, void* stream) {
@@ -439,6 +498,7 @@ const char* dg_status_string(int status) {
     case DG_ERR_CUDA: return "DG_ERR_CUDA";
     case DG_ERR_TIMEOUT: return "DG_ERR_TIMEOUT";
     case DG_ERR_BAD_METADATA: return "DG_ERR_BAD_METADATA";
+    case DG_ERR_SCRATCH_LIMIT: return "DG_ERR_SCRATCH_LIMIT";
     default: return "DG_ERR_UNKNOWN";
   }
 }
