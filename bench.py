@@ -6,7 +6,10 @@ shapes: M in {64, 128, 4096} x (N, K) in {(2112,7168), (24576,1536),
 (32768,512), (7168,16384), (4096,7168), (7168,2048)}, A/B ~ N(0,1) quantised
 with 1x128 / 128x128 UE8M0 scales, C ~ N(0,1) bf16 (synthetic, seeded).
 Each GEMM call is timed with CUDA events on its stream after an L2 flush (a
-256 MB write), so no call reads its inputs from a warm L2.
+256 MB write followed by a 256 MB read, so L2 holds clean unrelated lines),
+so no call reads its inputs from a warm L2; each step is
+enqueued behind a short device-side sleep so that no timed call waits for the
+host to launch it.
 
   value   = total FLOPs of the sweep (all ranks) / device time (max over ranks)
   e2e     = the same sweep through the C ABI from pinned HOST buffers, the
@@ -42,6 +45,7 @@ UNIT = "TFLOPS"
 DENSE_NK = [(2112, 7168), (24576, 1536), (32768, 512), (7168, 16384), (4096, 7168), (7168, 2048)]
 DENSE_M = [64, 128, 4096]
 FLUSH_BYTES = 256 << 20
+HOLD_CYCLES = 6_000_000  # ~3 ms at 2 GHz: longer than the host needs to enqueue one step
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_PER_BF16 = 2.0  # nominal dense FP8 : BF16 tensor throughput (4.5 : 2.25 PFLOP/s)
 
@@ -292,6 +296,14 @@ def main():
     gen.manual_seed(1234 + rank)
     inputs = [make_inputs(dg, torch, m, n, k, gen) for (m, n, k) in shapes]
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush_rd = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
+
+    def flush_l2():
+        # write 256 MB (> 126 MB L2), then read another 256 MB so that L2 ends
+        # up holding clean lines of unrelated data: no input of the timed call
+        # is cached and no dirty line of the flush is written back inside it
+        flush.zero_()
+        flush_rd.max()
     stream = torch.cuda.current_stream()
     torch.cuda.synchronize()
 
@@ -299,8 +311,11 @@ def main():
         dg.dg_fp8_gemm_nt(x["a"], x["sfa"], x["b"], x["sfb"], x["c"], x["d"], stream=stream)
 
     def sweep(events):
+        # Hold the stream in a short device-side sleep while the host enqueues
+        # the whole step, so no timed call waits for the host to launch it.
+        torch.cuda._sleep(HOLD_CYCLES)
         for i, x in enumerate(inputs):
-            flush.zero_()
+            flush_l2()
             if events is not None:
                 events[i][0].record(stream)
             call(x)
@@ -427,7 +442,7 @@ def main():
                                     if not args.shape else f"dense NT FP8 {args.shape}"),
                        "shapes": len(shapes), "accumulate": "f32 (TMEM)", "out": "bf16", "c": "N(0,1) bf16",
                        "scales": "UE8M0 1x128 (A), 128x128 (B)",
-                       "l2": "flushed before every timed GEMM call (256 MB write, not timed)",
+                       "l2": "flushed before every timed GEMM call: 256 MB write then 256 MB read, not timed",
                        "parallelism": f"replicas x{world}", "wall_s_timed_region": round(wall, 3)},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
             "clocks": clocks, "per_shape": per_shape,

@@ -198,6 +198,17 @@ int64_t dg_packed_sf_words(int rows, int num_sf_cols);
 int dg_get_num_sms(void);
 dg_status dg_set_num_sms(int num_sms);
 
+/* Programmatic dependent launch (default on): every kernel of this library
+ * is launched as a programmatic dependent of the preceding work on its
+ * stream, so its launch and prologue (barrier set-up, TMEM allocation,
+ * descriptor prefetch) overlap the previous kernel's tail; it touches no
+ * global memory before that work has completed.  dg_set_pdl(0) launches
+ * plainly.  Source: "DeepGEMM：统一高性能张量核心 GEMM 计算库编译与使用指南"
+ * (zhouruolin.cn), section "工具函数" (set_pdl), and "DeepSeek 发布 DeepGEMM
+ * 重大更新" (linlog.top), section "其他更新" (PDL). */
+dg_status dg_set_pdl(int enable);
+int dg_get_pdl(void);
+
 /* Row alignment of groups in the contiguous layout: 128. */
 int dg_get_mk_alignment_for_contiguous_layout(void);
 

@@ -21,7 +21,7 @@ __all__ = [
     "DGError", "lib", "dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
     "dg_m_grouped_fp8_gemm_nt_masked", "dg_fp8_gemm_nt_noalloc", "dg_noalloc_scratch_bytes", "dg_fp8_fp4_gemm_nt", "dg_m_grouped_fp8_fp4_gemm_nt_contiguous",
     "dg_quantize_fp8", "dg_quantize_fp4", "dg_pack_sf", "dg_packed_sf_words", "dg_get_num_sms",
-    "dg_set_num_sms", "dg_get_mk_alignment_for_contiguous_layout", "dg_get_last_error",
+    "dg_set_num_sms", "dg_set_pdl", "dg_get_pdl", "dg_get_mk_alignment_for_contiguous_layout", "dg_get_last_error",
     "dg_debug_starved_wait", "dg_launch_count", "dg_query_dense_config", "dg_num_tiles", "dg_shutdown",
     "SYMBOLS",
 ]
@@ -51,6 +51,8 @@ SYMBOLS = {
     "dg_get_num_sms": (_INT, []),
     "dg_set_num_sms": (_INT, [_INT]),
     "dg_get_mk_alignment_for_contiguous_layout": (_INT, []),
+    "dg_set_pdl": (_INT, [_INT]),
+    "dg_get_pdl": (_INT, []),
     "dg_get_last_error": (_INT, [_VP]),
     "dg_debug_starved_wait": (_INT, [ctypes.c_uint, _VP]),
     "dg_status_string": (ctypes.c_char_p, [_INT]),
@@ -204,6 +206,14 @@ def dg_get_num_sms() -> int:
 
 def dg_set_num_sms(n: int) -> None:
     _check(lib().dg_set_num_sms(int(n)), "dg_set_num_sms")
+
+
+def dg_set_pdl(enable: bool) -> None:
+    _check(lib().dg_set_pdl(int(bool(enable))), "dg_set_pdl")
+
+
+def dg_get_pdl() -> bool:
+    return bool(lib().dg_get_pdl())
 
 
 def dg_get_mk_alignment_for_contiguous_layout() -> int:

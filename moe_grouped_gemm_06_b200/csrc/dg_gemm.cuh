@@ -13,15 +13,17 @@
 // M-grouped contiguous and masked layouts); "DeepSeek 发布 DeepGEMM 重大更新"
 // (linlog.top), section "FP4 精度支持" (FP8 x FP4).
 //
-// Roles (192 threads, one CTA per SM, persistent over work units):
+// Roles (320 threads, one CTA per SM, persistent over work units):
 //   warp 0      TMA producer: A/B tiles (128-byte swizzle) and packed scale
 //               words into a STAGES-deep shared-memory ring.
 //   warp 1      allocates TMEM; one lane issues tcgen05.cp (scales -> TMEM)
 //               and tcgen05.mma.kind::mxf8f6f4.block_scale into a
 //               double-buffered FP32 accumulator.
-//   warps 2..5  epilogue: tcgen05.ld -> (+C) -> bf16 -> swizzled smem -> TMA
-//               store; rows past a masked group's count are never written.
-//               With split-K they write FP32 partials instead.
+//   warps 2..9  epilogue, two warps per TMEM sub-partition (one column half
+//               each): C prefetched into registers, tcgen05.ld -> (+C) ->
+//               bf16 -> swizzled smem -> TMA store; rows past a masked
+//               group's count are never written.  With split-K they write
+//               FP32 partials, summed by splitk_reduce_kernel.
 //
 // The scales are applied inside the MMA: the UE8M0 code of a 1x128 group is
 // used for each of the four K=32 steps of its 128-wide block (the instruction
@@ -35,7 +37,8 @@ namespace dg {
 
 constexpr int kBM = 128;           // rows of A per tile (= TMEM lanes)
 constexpr int kBK = 128;           // K per pipeline stage (= one scale block)
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;       // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
+constexpr int kEpiWarps = 8;
 constexpr int kEpiCols = 32;       // columns per epilogue store box
 constexpr int kTmemCols = 512;
 constexpr int kMaxMaskedGroups = 1024;
@@ -74,15 +77,16 @@ struct Cfg {
   // a tile starts 0 or 64 rows into its first chunk.
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
   static constexpr int kSfbChunks = 3;                       // 128-row scale chunks a tile can touch
-  static constexpr int kAccBufs = (BN <= 224) ? 2 : 1;
-  // accumulator buffers start at TMEM columns 0 and 256
+  // FP32 accumulator buffers in TMEM: three of 128 columns (BN = 128), two at
+  // columns 0 and 256 (BN = 192), one (BN = 256); scale factors after them.
+  static constexpr int kAccBufs = (BN <= 128) ? 3 : (BN <= 224 ? 2 : 1);
   static constexpr int kABytes = kBM * kBK;                  // 16 KB
   static constexpr int kBBytes = BN * kBK;                   // smem bytes (FP4 lands padded to 1 B/elt)
   static constexpr int kBTxBytes = FP4 ? BN * kBK / 2 : BN * kBK;  // bytes the TMA copy reports (packed)
   static constexpr int kSfaBytes = 512;
   static constexpr int kSfbBytes = kSfbChunks * 512;
   static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
-  static constexpr int kEpiBytes = 4 * 2 * 32 * 64;          // 4 warps x 2 buffers x (32 rows x 64 B)
+  static constexpr int kEpiBytes = kEpiWarps * 32 * 64;        // one 32 x 64 B staging box per epilogue warp
   static constexpr int kMaskBytes = ((kMaxMaskedGroups + 1) * 4 + 15) / 16 * 16;
   static constexpr int kBarBytes = 256;
   static constexpr int kBudget = 232448 - 1024;              // 227 KB minus alignment slack
@@ -91,8 +95,8 @@ struct Cfg {
   static_assert(kStages >= 2, "stages");
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kEpiBytes + kMaskBytes + kBarBytes;
   static constexpr uint32_t kColAcc = 0;
-  static constexpr uint32_t kAccStride = 256;
-  static constexpr uint32_t kColSfa = (kAccBufs == 2) ? 256 + BN : BN;   // even, 4-column aligned
+  static constexpr uint32_t kAccStride = (BN <= 128) ? 128 : 256;
+  static constexpr uint32_t kColSfa = (kAccBufs - 1) * kAccStride + BN;  // even, 4-column aligned
   static constexpr uint32_t kColSfb = kColSfa + 4;
   static_assert(kColSfb + 4 * kSfbChunks <= kTmemCols, "TMEM columns");
   // Instruction descriptor of kind::mxf8f6f4 with block scaling: A = E4M3,
@@ -163,9 +167,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* full = bars;
   uint64_t* empty = bars + S;
   uint64_t* tfull = bars + 2 * S;
-  uint64_t* tempty = bars + 2 * S + 2;
-  uint64_t* drain = bars + 2 * S + 4;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+  uint64_t* tempty = bars + 2 * S + 3;
+  uint64_t* drain = bars + 2 * S + 6;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 * S + 7);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
 
   const int warp = threadIdx.x / 32;
@@ -177,9 +181,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < 3; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+      mbar_init(&tempty[b], kEpiWarps);
     }
     mbar_init(drain, 1);
     *s_abort = 0;
@@ -194,6 +198,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(s_tmem, kTmemCols);
     tmem_relinquish();
   }
+  // Prologue above touches no global memory; with programmatic dependent
+  // launch it overlaps the previous kernel's tail.  Everything below may
+  // read inputs the previous kernel wrote.
+  pdl_wait();
+  pdl_launch_dependents();
   int num_units;
   if (LAYOUT == kMasked) {
     // tiles per group, read from device memory (so the call stays
@@ -313,8 +322,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n0 = u.nb * BN;
         const int nchunks = (min(n0 + BN, a.n) - 1) / 128 - n0 / 128 + 1;
         const uint32_t sfb_t = tmem_base + C::kColSfb + (uint32_t)((n0 % 128) / 32);
-        const int buf = (C::kAccBufs == 2) ? (local & 1) : 0;
-        const uint32_t use = (C::kAccBufs == 2) ? (uint32_t)(local >> 1) : (uint32_t)local;
+        const int buf = local % C::kAccBufs;
+        const uint32_t use = (uint32_t)(local / C::kAccBufs);
         if (!dg_wait(&tempty[buf], (use & 1) ^ 1, s_abort, limit)) {
           ok = false;
           break;
@@ -362,87 +371,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM sub-partition of this warp: lanes 32q..32q+31
-    uint8_t* stg0 = s_epi + (warp - 2) * (2 * 32 * 64);
+    // Two warps per TMEM sub-partition: warp w reads lanes 32*(w%4).. and the
+    // column half (w-2)/4 of the tile.  All C loads of a tile are issued into
+    // registers before waiting for its accumulator, so they overlap the MMAs.
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    constexpr int kCols = BN / 2;                 // columns of this warp
+    constexpr int kChunks = kCols / kEpiCols;     // 32-column chunks of this warp
+    uint8_t* stg = s_epi + (warp - 2) * (32 * 64);
     int local = 0;
-    uint32_t store_seq = 0;
     for (int t = blockIdx.x; t < num_units; t += gridDim.x) {
       Unit u = decode_unit<LAYOUT>(t, a, s_prefix);
       if (LAYOUT == kContig && !u.valid) continue;
-      const int buf = (C::kAccBufs == 2) ? (local & 1) : 0;
-      const uint32_t use = (C::kAccBufs == 2) ? (uint32_t)(local >> 1) : (uint32_t)local;
-      int ok = 1;
-      if (lane == 0) ok = dg_wait(&tfull[buf], use & 1, s_abort, limit) ? 1 : 0;
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      tc_fence_after();
+      const int buf = local % C::kAccBufs;
+      const uint32_t use = (uint32_t)(local / C::kAccBufs);
       const int r0 = u.mb * kBM + q * 32;  // first row of this warp (within the group for masked)
       int limit_rows = a.rows;
       if (LAYOUT == kMasked) limit_rows = min(max(__ldg(a.masked_m + u.g), 0), a.rows);
       const int vr = min(32, limit_rows - r0);
       const int row = r0 + (int)lane;
       const long long grow = (LAYOUT == kMasked) ? (long long)u.g * a.rows + row : row;
-      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + C::kColAcc + buf * C::kAccStride;
-#pragma unroll 1
-      for (int j = 0; j < BN / kEpiCols; ++j) {
-        const int col0 = u.nb * BN + j * kEpiCols;
-        if (vr <= 0 || col0 >= a.n) break;
-        // C for this thread's row segment, fetched before the TMEM read
-        float cv[kEpiCols];
+      const int colw = u.nb * BN + half * kCols;  // first column of this warp
+
+      uint4 creg[kChunks][4];
+      const bool load_c = a.c != nullptr && a.splits == 1;
 #pragma unroll
-        for (int i = 0; i < kEpiCols; ++i) cv[i] = 0.f;
-        if (a.c != nullptr && a.splits == 1 && (int)lane < vr &&
-            DG_CHECK(((reinterpret_cast<uintptr_t>(a.c + grow * a.n + col0) & 15) == 0) && row < a.rows &&
-                         grow >= 0, 1)) {
-          const uint4* src = reinterpret_cast<const uint4*>(a.c + grow * a.n + col0);
+      for (int j = 0; j < kChunks; ++j)
 #pragma unroll
-          for (int v = 0; v < kEpiCols / 8; ++v) {
-            if (col0 + 8 * v < a.n) {
-              uint4 w = __ldg(src + v);
-              const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        for (int v = 0; v < 4; ++v) creg[j][v] = make_uint4(0u, 0u, 0u, 0u);
+      if (load_c && (int)lane < vr &&
+          DG_CHECK(((reinterpret_cast<uintptr_t>(a.c + grow * a.n + colw) & 15) == 0) && row < a.rows && grow >= 0,
+                   1)) {
+        const uint4* src = reinterpret_cast<const uint4*>(a.c + grow * a.n + colw);
 #pragma unroll
-              for (int h = 0; h < 4; ++h) {
-                cv[8 * v + 2 * h] = __uint_as_float(ww[h] << 16);
-                cv[8 * v + 2 * h + 1] = __uint_as_float(ww[h] & 0xFFFF0000u);
-              }
-            }
-          }
-        }
-        uint32_t acc[kEpiCols];
-        DG_CHECK(((t_row & 0xFFFF) + j * kEpiCols + kEpiCols <= (uint32_t)kTmemCols) &&
-                     ((t_row >> 16) & 0xFFFF) == (uint32_t)(q * 32) + (tmem_base >> 16) && (warp & 3) == q,
-                 8);
-        tc_ld_32x32b_x32(t_row + j * kEpiCols, acc);
-        tc_wait_ld_regs(acc);
-        if (a.splits > 1) {
-          // FP32 partials of this K slice: ws[split][row][col]
-          if ((int)lane < vr &&
-              DG_CHECK(a.ws != nullptr && u.split < a.splits && row < a.rows &&
-                           (reinterpret_cast<uintptr_t>(a.ws + ((long long)u.split * a.rows + row) * a.n + col0) & 15) == 0,
-                       3)) {
-            float4* dst = reinterpret_cast<float4*>(a.ws + ((long long)u.split * a.rows + row) * a.n + col0);
+        for (int j = 0; j < kChunks; ++j)
 #pragma unroll
-            for (int v = 0; v < kEpiCols / 4; ++v)
-              if (col0 + 4 * v < a.n)
-                dst[v] = make_float4(__uint_as_float(acc[4 * v]), __uint_as_float(acc[4 * v + 1]),
-                                     __uint_as_float(acc[4 * v + 2]), __uint_as_float(acc[4 * v + 3]));
-          }
-          continue;
-        }
-        uint32_t packed[kEpiCols / 2];
-#pragma unroll
-        for (int i = 0; i < kEpiCols / 2; ++i) {
-          __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(acc[2 * i]) + cv[2 * i],
-                                                   __uint_as_float(acc[2 * i + 1]) + cv[2 * i + 1]);
-          packed[i] = *reinterpret_cast<uint32_t*>(&h);
-        }
+          for (int v = 0; v < 4; ++v)
+            if (colw + j * kEpiCols + 8 * v < a.n) creg[j][v] = __ldg(src + j * 4 + v);
+      }
+
+      int ok = 1;
+      if (lane == 0) ok = dg_wait(&tfull[buf], use & 1, s_abort, limit) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + C::kColAcc + buf * C::kAccStride +
+                             (uint32_t)(half * kCols);
+
+      // bf16 result of one 32-column chunk of this warp's rows -> D
+      auto store_chunk = [&](int col0, const uint32_t (&packed)[kEpiCols / 2]) {
         if (vr == 32) {
           // full 32-row box: swizzled staging (64-byte rows) + TMA store
-          uint8_t* stg = stg0 + (store_seq & 1) * (32 * 64);
           DG_CHECK((smem_u32(stg) & 1023) == 0 && stg >= s_epi && stg + 2048 <= s_epi + C::kEpiBytes &&
                        (col0 % 8) == 0 && r0 + 32 <= (LAYOUT == kMasked ? limit_rows : a.rows),
                    7);
-          if (lane == 0) bulk_wait_group_read<1>();
+          if (lane == 0) bulk_wait_group_read<0>();
           __syncwarp();
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
@@ -456,7 +439,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_store_3d(&tm_d, stg, col0, r0, (LAYOUT == kMasked) ? u.g : 0);
             bulk_commit_group();
           }
-          ++store_seq;
         } else if ((int)lane < vr &&
                    DG_CHECK((reinterpret_cast<uintptr_t>(a.d + grow * a.n + col0) & 15) == 0 && row < limit_rows,
                             2)) {
@@ -466,6 +448,64 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int v = 0; v < kEpiCols / 8; ++v)
             if (col0 + 8 * v < a.n)
               dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+        }
+      };
+
+      if (a.splits > 1) {
+        // ---- split-K: this slice's FP32 partials; splitk_reduce_kernel sums
+        // the slices in slice order (+C) and writes D
+#pragma unroll
+        for (int j = 0; j < kChunks; ++j) {
+          const int col0 = colw + j * kEpiCols;
+          if (vr > 0 && col0 < a.n) {
+            uint32_t acc[kEpiCols];
+            tc_ld_32x32b_x32(t_row + j * kEpiCols, acc);
+            tc_wait_ld_regs(acc);
+            if ((int)lane < vr &&
+                DG_CHECK(a.ws != nullptr && u.split < a.splits && row < a.rows &&
+                             (reinterpret_cast<uintptr_t>(a.ws + ((long long)u.split * a.rows + row) * a.n + col0) &
+                              15) == 0,
+                         3)) {
+              float4* dst = reinterpret_cast<float4*>(a.ws + ((long long)u.split * a.rows + row) * a.n + col0);
+#pragma unroll
+              for (int v = 0; v < kEpiCols / 4; ++v)
+                if (col0 + 4 * v < a.n)
+                  dst[v] = make_float4(__uint_as_float(acc[4 * v]), __uint_as_float(acc[4 * v + 1]),
+                                       __uint_as_float(acc[4 * v + 2]), __uint_as_float(acc[4 * v + 3]));
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[buf]);
+        ++local;
+        continue;
+      }
+
+#pragma unroll
+      for (int j = 0; j < kChunks; ++j) {
+        const int col0 = colw + j * kEpiCols;
+        if (vr > 0 && col0 < a.n) {
+          uint32_t acc[kEpiCols];
+          DG_CHECK(((t_row & 0xFFFF) + j * kEpiCols + kEpiCols <= (uint32_t)kTmemCols) &&
+                       ((t_row >> 16) & 0xFFFF) == (uint32_t)(q * 32) + (tmem_base >> 16) && (warp & 3) == q,
+                   8);
+          tc_ld_32x32b_x32(t_row + j * kEpiCols, acc);
+          tc_wait_ld_regs(acc);
+          uint32_t packed[kEpiCols / 2];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint32_t cw[4] = {creg[j][v].x, creg[j][v].y, creg[j][v].z, creg[j][v].w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const int i = 4 * v + h;
+              __nv_bfloat162 bv = __floats2bfloat162_rn(__uint_as_float(acc[2 * i]) + __uint_as_float(cw[h] << 16),
+                                                        __uint_as_float(acc[2 * i + 1]) +
+                                                            __uint_as_float(cw[h] & 0xFFFF0000u));
+              packed[i] = *reinterpret_cast<uint32_t*>(&bv);
+            }
+          }
+          store_chunk(col0, packed);
         }
       }
       tc_fence_before();
@@ -485,39 +525,42 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Split-K reduction: D = bf16(sum_s ws[s] + C), 8 columns per thread.
+// Split-K reduction: D = bf16(sum_s ws[s] + C) with the slices summed in
+// slice order (deterministic).  4 columns per thread; the loads of all
+// slices are issued before the first add (at most kMaxSplits slices).
+constexpr int kMaxSplits = 16;
 __global__ void splitk_reduce_kernel(const float* __restrict__ ws, const uint16_t* __restrict__ c,
                                      uint16_t* __restrict__ d, int rows, int n, int splits) {
-  const long long units = (long long)rows * (n / 8);
+  pdl_wait();
+  const long long units = (long long)rows * (n / 4);
   for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < units;
        u += (long long)gridDim.x * blockDim.x) {
-    const long long r = u / (n / 8);
-    const int col = (int)(u - r * (n / 8)) * 8;
-    float acc[8];
+    const long long r = u / (n / 4);
+    const int col = (int)(u - r * (n / 4)) * 4;
+    const float4* p = reinterpret_cast<const float4*>(ws + r * n + col);
+    const long long slice = (long long)rows * n / 4;  // float4 stride between slices
+    float4 part[kMaxSplits];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    for (int s = 0; s < splits; ++s) {
-      const float4* p = reinterpret_cast<const float4*>(ws + ((long long)s * rows + r) * n + col);
-      float4 x = __ldg(p), y = __ldg(p + 1);
-      acc[0] += x.x; acc[1] += x.y; acc[2] += x.z; acc[3] += x.w;
-      acc[4] += y.x; acc[5] += y.y; acc[6] += y.z; acc[7] += y.w;
+    for (int s = 0; s < kMaxSplits; ++s)
+      part[s] = (s < splits) ? __ldg(p + s * slice) : make_float4(0.f, 0.f, 0.f, 0.f);
+    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+#pragma unroll
+    for (int s = 0; s < kMaxSplits; ++s) {
+      acc0 += part[s].x;
+      acc1 += part[s].y;
+      acc2 += part[s].z;
+      acc3 += part[s].w;
     }
     if (c != nullptr) {
-      uint4 w = __ldg(reinterpret_cast<const uint4*>(c + r * n + col));
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        acc[2 * h] += __uint_as_float(ww[h] << 16);
-        acc[2 * h + 1] += __uint_as_float(ww[h] & 0xFFFF0000u);
-      }
+      const uint2 w = __ldg(reinterpret_cast<const uint2*>(c + r * n + col));
+      acc0 += __uint_as_float(w.x << 16);
+      acc1 += __uint_as_float(w.x & 0xFFFF0000u);
+      acc2 += __uint_as_float(w.y << 16);
+      acc3 += __uint_as_float(w.y & 0xFFFF0000u);
     }
-    uint32_t o[4];
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * h], acc[2 * h + 1]);
-      o[h] = *reinterpret_cast<uint32_t*>(&b);
-    }
-    *reinterpret_cast<uint4*>(d + r * n + col) = make_uint4(o[0], o[1], o[2], o[3]);
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc0, acc1), hi = __floats2bfloat162_rn(acc2, acc3);
+    *reinterpret_cast<uint2*>(d + r * n + col) =
+        make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
   }
 }
 

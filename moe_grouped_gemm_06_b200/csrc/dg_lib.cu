@@ -18,6 +18,24 @@ namespace {
 
 std::atomic<uint64_t> g_launches{0};
 int g_num_sms_override = 0;
+std::atomic<int> g_pdl{1};  // programmatic dependent launch on (dg_set_pdl)
+
+// Launches a kernel on `s`, as a programmatic dependent of the previous work
+// on the stream when PDL is enabled.
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = g_pdl.load() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -103,13 +121,27 @@ long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
 // overhead of 4 K-blocks), with a 3% surcharge per extra split-K slice for
 // the partial-sum round trip.  Minimised over the instantiated block sizes;
 // ties keep fewer slices, then the larger block.
+// DG_BLOCK_N (one of kBlockNs) restricts the search to that block width.
+int forced_block_n() {
+  static int v = [] {
+    const char* e = std::getenv("DG_BLOCK_N");
+    if (!e) return 0;
+    const int b = std::atoi(e);
+    for (int bn : kBlockNs)
+      if (bn == b) return b;
+    return 0;
+  }();
+  return v;
+}
+
 Plan plan_gemm(long long m_blocks, int n, int k, int sms, bool allow_split) {
   Plan best;
   double best_cost = 1e300;
   const int kb = k / 128;
   for (int bn : kBlockNs) {
+    if (forced_block_n() && bn != forced_block_n()) continue;
     const long long tiles = m_blocks * ceil_div(n, bn);
-    const int max_s = allow_split ? std::max(1, std::min(16, kb / 2)) : 1;
+    const int max_s = allow_split ? std::max(1, std::min(dg::kMaxSplits, kb / 2)) : 1;
     for (int s = 1; s <= max_s; ++s) {
       const int kbps = (int)ceil_div(kb, s);
       const int s_eff = (int)ceil_div(kb, kbps);
@@ -140,6 +172,8 @@ struct Workspace {
 std::mutex g_ws_mutex;
 std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
 
+// Split-K FP32 partials of this (device, stream), allocated stream-ordered on
+// first use and grown on demand.
 float* workspace(size_t bytes, cudaStream_t s) {
   int dev = 0;
   cudaGetDevice(&dev);
@@ -171,8 +205,8 @@ dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
       return DG_ERR_CUDA;
     attr_set_mask.fetch_or(bit);
   }
-  kern<<<grid, dg::kThreads, C::kSmemBytes, s>>>(ta, tb, td, args);
-  if (cudaGetLastError() != cudaSuccess) return DG_ERR_CUDA;
+  if (launch(kern, dim3(grid), dim3(dg::kThreads), C::kSmemBytes, s, ta, tb, td, args) != cudaSuccess)
+    return DG_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return DG_OK;
 }
@@ -282,11 +316,12 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
   dg_status st = dispatch<FP4, LAYOUT>(plan.bn, ta, tb, td, args, plan.grid, s);
   if (st != DG_OK || plan.splits == 1) return st;
 
-  const long long units = (long long)p.rows * (p.n / 8);
+  const long long units = (long long)p.rows * (p.n / 4);
   const int threads = 256;
   const int blocks = (int)std::min<long long>(ceil_div(units, threads), (long long)sms * 8);
-  dg::splitk_reduce_kernel<<<blocks, threads, 0, s>>>(args.ws, args.c, args.d, p.rows, p.n, plan.splits);
-  if (cudaGetLastError() != cudaSuccess) return DG_ERR_CUDA;
+  if (launch(dg::splitk_reduce_kernel, dim3(blocks), dim3(threads), 0, s, (const float*)args.ws, args.c, args.d,
+             p.rows, p.n, plan.splits) != cudaSuccess)
+    return DG_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return DG_OK;
 }
@@ -471,6 +506,13 @@ dg_status dg_set_num_sms(int n) {
 }
 
 int dg_get_mk_alignment_for_contiguous_layout(void) { return dg::kBM; }
+
+dg_status dg_set_pdl(int enable) {
+  g_pdl.store(enable ? 1 : 0);
+  return DG_OK;
+}
+
+int dg_get_pdl(void) { return g_pdl.load(); }
 
 dg_status dg_get_last_error(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DG_ERR_CUDA;

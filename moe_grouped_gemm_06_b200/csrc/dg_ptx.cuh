@@ -88,6 +88,20 @@ __device__ __forceinline__ bool dg_wait(uint64_t* bar, uint32_t parity, volatile
   }
 }
 
+// ------------------------------------------- programmatic dependent launch
+
+// Block until the grids this one depends on (launched before it on the
+// stream) have completed and their memory is visible.  A no-op when the
+// kernel was not launched as a programmatic dependent.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Allow the next grid on the stream (if launched as a programmatic
+// dependent) to begin launching; it still waits for this grid's completion
+// before touching memory.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
