@@ -209,6 +209,13 @@ dg_status dg_set_num_sms(int num_sms);
 dg_status dg_set_pdl(int enable);
 int dg_get_pdl(void);
 
+/* Restricts the tile heuristic to one configuration: block_n in {128, 192,
+ * 256} (0 = any) and ctas 1 (single-CTA 128-row tiles) or 0 (any); ctas = 2
+ * (CTA-pair tiles) returns DG_ERR_UNSUPPORTED in this version.  Meant for
+ * tuning and tests; the default (0, 0) is the heuristic.  The environment
+ * variable DG_BLOCK_N sets the initial block width. */
+dg_status dg_set_tile_config(int block_n, int ctas);
+
 /* Row alignment of groups in the contiguous layout: 128. */
 int dg_get_mk_alignment_for_contiguous_layout(void);
 
@@ -228,8 +235,9 @@ const char* dg_status_string(int status);
 uint64_t dg_launch_count(void);
 
 /* Configuration the dense heuristic picks for (m, n, k): block_n, split-K
- * slices, work units and grid size (any pointer may be NULL). */
-dg_status dg_query_dense_config(int m, int n, int k, int* block_n, int* splits, int* units, int* grid);
+ * slices, work units (tiles x slices), grid size in CTAs and CTAs per tile
+ * (1 or 2) (any pointer may be NULL). */
+dg_status dg_query_dense_config(int m, int n, int k, int* block_n, int* splits, int* units, int* grid, int* ctas);
 
 /* Output tiles of an m x n problem cut into block_m x block_n tiles (the
  * count the heuristic balances against the SM count; "DeepSeek 开源第三弹 ...

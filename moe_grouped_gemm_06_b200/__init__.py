@@ -21,7 +21,7 @@ __all__ = [
     "DGError", "lib", "dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
     "dg_m_grouped_fp8_gemm_nt_masked", "dg_fp8_gemm_nt_noalloc", "dg_noalloc_scratch_bytes", "dg_fp8_fp4_gemm_nt", "dg_m_grouped_fp8_fp4_gemm_nt_contiguous",
     "dg_quantize_fp8", "dg_quantize_fp4", "dg_pack_sf", "dg_packed_sf_words", "dg_get_num_sms",
-    "dg_set_num_sms", "dg_set_pdl", "dg_get_pdl", "dg_get_mk_alignment_for_contiguous_layout", "dg_get_last_error",
+    "dg_set_num_sms", "dg_set_pdl", "dg_get_pdl", "dg_set_tile_config", "dg_get_mk_alignment_for_contiguous_layout", "dg_get_last_error",
     "dg_debug_starved_wait", "dg_launch_count", "dg_query_dense_config", "dg_num_tiles", "dg_shutdown",
     "SYMBOLS",
 ]
@@ -52,12 +52,13 @@ SYMBOLS = {
     "dg_set_num_sms": (_INT, [_INT]),
     "dg_get_mk_alignment_for_contiguous_layout": (_INT, []),
     "dg_set_pdl": (_INT, [_INT]),
+    "dg_set_tile_config": (_INT, [_INT, _INT]),
     "dg_get_pdl": (_INT, []),
     "dg_get_last_error": (_INT, [_VP]),
     "dg_debug_starved_wait": (_INT, [ctypes.c_uint, _VP]),
     "dg_status_string": (ctypes.c_char_p, [_INT]),
     "dg_launch_count": (ctypes.c_uint64, []),
-    "dg_query_dense_config": (_INT, [_INT, _INT, _INT, _VP, _VP, _VP, _VP]),
+    "dg_query_dense_config": (_INT, [_INT, _INT, _INT, _VP, _VP, _VP, _VP, _VP]),
     "dg_num_tiles": (_I64, [_INT, _INT, _INT, _INT]),
     "dg_shutdown": (None, []),
 }
@@ -212,6 +213,10 @@ def dg_set_pdl(enable: bool) -> None:
     _check(lib().dg_set_pdl(int(bool(enable))), "dg_set_pdl")
 
 
+def dg_set_tile_config(block_n: int = 0, ctas: int = 0) -> None:
+    _check(lib().dg_set_tile_config(int(block_n), int(ctas)), "dg_set_tile_config")
+
+
 def dg_get_pdl() -> bool:
     return bool(lib().dg_get_pdl())
 
@@ -234,9 +239,9 @@ def dg_launch_count() -> int:
 
 
 def dg_query_dense_config(m: int, n: int, k: int) -> dict:
-    vals = [ctypes.c_int(0) for _ in range(4)]
+    vals = [ctypes.c_int(0) for _ in range(5)]
     _check(lib().dg_query_dense_config(m, n, k, *[ctypes.byref(v) for v in vals]), "dg_query_dense_config")
-    return dict(zip(("block_n", "splits", "units", "grid"), (v.value for v in vals)))
+    return dict(zip(("block_n", "splits", "units", "grid", "ctas"), (v.value for v in vals)))
 
 
 def dg_num_tiles(m: int, n: int, block_m: int, block_n: int) -> int:

@@ -68,7 +68,7 @@ struct GemmArgs {
   long long sfa_words, sfb_words;      // total packed words (self-check bounds)
 };
 
-template <int BN, bool FP4>
+template <int BN, bool FP4, int CTAS = 1>
 struct Cfg {
   // The scale-factor operand of the MMA is addressed in TMEM columns of 32
   // rows (a 128-row chunk spans 4 columns), and that address must be even:
@@ -81,8 +81,9 @@ struct Cfg {
   // columns 0 and 256 (BN = 192), one (BN = 256); scale factors after them.
   static constexpr int kAccBufs = (BN <= 128) ? 3 : (BN <= 224 ? 2 : 1);
   static constexpr int kABytes = kBM * kBK;                  // 16 KB
-  static constexpr int kBBytes = BN * kBK;                   // smem bytes (FP4 lands padded to 1 B/elt)
-  static constexpr int kBTxBytes = FP4 ? BN * kBK / 2 : BN * kBK;  // bytes the TMA copy reports (packed)
+  static constexpr int kBRows = BN / CTAS;                   // B rows each CTA of a pair loads
+  static constexpr int kBBytes = kBRows * kBK;               // smem bytes (FP4 lands padded to 1 B/elt)
+  static constexpr int kBTxBytes = FP4 ? kBBytes / 2 : kBBytes;  // bytes the TMA copy reports (packed)
   static constexpr int kSfaBytes = 512;
   static constexpr int kSfbBytes = kSfbChunks * 512;
   static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
@@ -100,9 +101,10 @@ struct Cfg {
   static constexpr uint32_t kColSfb = kColSfa + 4;
   static_assert(kColSfb + 4 * kSfbChunks <= kTmemCols, "TMEM columns");
   // Instruction descriptor of kind::mxf8f6f4 with block scaling: A = E4M3,
-  // B = E4M3 (0) or E2M1 (5), both K-major, UE8M0 scales, M = 128, N = BN.
+  // B = E4M3 (0) or E2M1 (5), both K-major, UE8M0 scales, M = 128 per CTA
+  // (256 for a CTA pair), N = BN.
   static constexpr uint32_t kIdesc = (0u << 7) | ((FP4 ? 5u : 0u) << 10) | ((uint32_t)(BN >> 3) << 17) |
-                                     (1u << 23) | ((uint32_t)(kBM >> 4) << 24);
+                                     (1u << 23) | ((uint32_t)((kBM * CTAS) >> 4) << 24);
 };
 
 struct Unit {
@@ -142,18 +144,25 @@ __device__ __forceinline__ Unit decode_unit(int t, const GemmArgs& a, const int*
   u.nb = rem / band_rows;
   u.g = 0;
   if (LAYOUT == kContig) {
-    int g = __ldg(a.m_indices + (long long)u.mb * kBM);
+    int g = __ldg(a.m_indices + (long long)u.mb * kBM);  // 1-CTA tiles only
     u.g = g;
     u.valid = (g >= 0 && g < a.num_groups);
   }
   return u;
 }
 
-template <int BN, bool FP4, int LAYOUT>
+// CTAS = 2: a cluster of two CTAs computes 256 x BN tiles (dense layout only);
+// tm_sfa / tm_sfb view the packed scale words as rows of 512 bytes so that
+// the peer's scale loads can complete on the leader's barrier.
+template <int BN, bool FP4, int LAYOUT, int CTAS>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                const __grid_constant__ CUtensorMap tm_d, const GemmArgs args) {
-  using C = Cfg<BN, FP4>;
+                const __grid_constant__ CUtensorMap tm_d, const __grid_constant__ CUtensorMap tm_sfa,
+                const __grid_constant__ CUtensorMap tm_sfb, const GemmArgs args) {
+  static_assert(CTAS == 1 || (CTAS == 2 && LAYOUT == kDense), "CTA pairs serve the dense layout");
+  using C = Cfg<BN, FP4, CTAS>;
+  constexpr bool kPair = (CTAS == 2);
+  constexpr int kTileM = kBM * CTAS;
   constexpr int S = C::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -175,6 +184,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x / 32;
   const uint32_t lane = lane_id();
   const GemmArgs& a = args;
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;   // 0 = leader (issues the MMAs)
+  const int unit0 = blockIdx.x / CTAS, unit_step = gridDim.x / CTAS;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -183,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 3; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], kEpiWarps);
+      mbar_init(&tempty[b], kEpiWarps * CTAS);  // the pair's epilogues release the leader
     }
     mbar_init(drain, 1);
     *s_abort = 0;
@@ -193,10 +204,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_b);
     prefetch_tmap(&tm_d);
+    if constexpr (kPair) {
+      prefetch_tmap(&tm_sfa);
+      prefetch_tmap(&tm_sfb);
+    }
   }
   if (warp == 1) {
-    tmem_alloc(s_tmem, kTmemCols);
-    tmem_relinquish();
+    if constexpr (kPair) {
+      tmem_alloc_pair(s_tmem, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(s_tmem, kTmemCols);
+      tmem_relinquish();
+    }
   }
   // Prologue above touches no global memory; with programmatic dependent
   // launch it overlaps the previous kernel's tail.  Everything below may
@@ -220,7 +240,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (kPair)
+    cluster_sync_all();  // both CTAs' barriers initialised before any cross-CTA arrival
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
   if (LAYOUT == kMasked)
@@ -238,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t filled_phase[8];
       uint32_t filled_mask = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < num_units && ok; t += gridDim.x) {
+      for (int t = unit0; t < num_units && ok; t += unit_step) {
         Unit u = decode_unit<LAYOUT>(t, a, s_prefix);
         if (LAYOUT == kContig && !u.valid) {
           if (u.g >= a.num_groups) record_error(-5);
@@ -250,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int c0 = n0 / 128;
         const int c1 = (min(n0 + BN, a.n) - 1) / 128;
         const int nchunks = c1 - c0 + 1;
-        const int a_row = u.mb * kBM;
+        const int a_row = u.mb * kTileM + (int)rank * kBM;
         const int a_grp = (LAYOUT == kMasked) ? u.g : 0;
         const int b_grp = (LAYOUT == kDense) ? 0 : u.g;
         const int32_t* sfa_g = a.sfa + (LAYOUT == kMasked ? (long long)u.g * a.sfa_group_words : 0);
@@ -268,6 +291,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           DG_CHECK(((smem_u32(s_a + stage * C::kABytes) | smem_u32(s_b + stage * C::kBBytes)) & 1023) == 0 &&
                        u.mb < a.num_m_blocks && u.nb < a.num_n_blocks && kb < a.kb_total,
                    6);
+          if constexpr (kPair) {
+            // both CTAs' loads complete on the leader's barrier, which expects
+            // the bytes of both.  A cta_group::2 copy names its barrier by this
+            // CTA's shared address with the peer bit (bit 24) cleared.
+            const uint32_t bar = smem_u32(&full[stage]) & kPeerBitMask;
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], bytes * CTAS);
+            tma_load_3d_pair(s_a + stage * C::kABytes, &tm_a, bar, kb * kBK, a_row, 0);
+            tma_load_3d_pair(s_b + stage * C::kBBytes, &tm_b, bar, kb * kBK, n0 + (int)rank * C::kBRows, 0);
+            if (new_sfa) tma_load_2d_pair(s_sfa + stage * C::kSfaBytes, &tm_sfa, bar, 0,
+                                          (kb >> 2) * a.sfa_chunks + a_row / 128);
+            if (new_sfb) {
+              const int q = FP4 ? kb : (kb >> 2);
+              for (int ch = 0; ch < nchunks; ++ch)
+                tma_load_2d_pair(s_sfb + stage * C::kSfbBytes + ch * 512, &tm_sfb, bar, 0, q * a.sfb_chunks + c0 + ch);
+            }
+            filled_phase[stage] = phase;
+            filled_mask |= 1u << stage;
+            if (++stage == S) {
+              stage = 0;
+              phase ^= 1;
+            }
+            continue;
+          }
           mbar_arrive_expect_tx(&full[stage], bytes);
           tma_load_3d(s_a + stage * C::kABytes, &tm_a, &full[stage], kb * kBK, a_row, a_grp);
           tma_load_3d(s_b + stage * C::kBBytes, &tm_b, &full[stage], kb * kBK, n0, b_grp);
@@ -295,9 +341,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (!ok) {
+      if (!ok && rank == 0) {
         // never leave copies in flight into shared memory: wait (bounded) for
-        // the last fill of every stage
+        // the last fill of every stage (a pair's fills all count on the
+        // leader's barriers; the final cluster barrier holds the peer)
         for (int s = 0; s < S; ++s)
           if (filled_mask & (1u << s)) {
             uint64_t t0 = global_timer_ns();
@@ -308,13 +355,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
       const uint32_t sfa_t = tmem_base + C::kColSfa;
-      for (int t = blockIdx.x; t < num_units && ok; t += gridDim.x) {
+      for (int t = unit0; t < num_units && ok; t += unit_step) {
         Unit u = decode_unit<LAYOUT>(t, a, s_prefix);
         if (LAYOUT == kContig && !u.valid) continue;
         const int kb0 = u.split * a.kb_per_split;
@@ -338,11 +385,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const bool new_sfa = ((kb & 3) == 0) || kb == kb0;
           const bool new_sfb = FP4 || new_sfa;
-          if (new_sfa) tc_cp_32x128b_x4(sfa_t, sdesc_sf_32x16(s_sfa + stage * C::kSfaBytes));
+          if (new_sfa) {
+            if constexpr (kPair)
+              tc_cp_32x128b_x4_pair(sfa_t, sdesc_sf_32x16(s_sfa + stage * C::kSfaBytes));
+            else
+              tc_cp_32x128b_x4(sfa_t, sdesc_sf_32x16(s_sfa + stage * C::kSfaBytes));
+          }
           if (new_sfb)
-            for (int ch = 0; ch < nchunks; ++ch)
-              tc_cp_32x128b_x4(tmem_base + C::kColSfb + 4 * ch,
-                               sdesc_sf_32x16(s_sfb + stage * C::kSfbBytes + ch * 512));
+            for (int ch = 0; ch < nchunks; ++ch) {
+              const uint64_t sd = sdesc_sf_32x16(s_sfb + stage * C::kSfbBytes + ch * 512);
+              if constexpr (kPair)
+                tc_cp_32x128b_x4_pair(tmem_base + C::kColSfb + 4 * ch, sd);
+              else
+                tc_cp_32x128b_x4(tmem_base + C::kColSfb + 4 * ch, sd);
+            }
           const uint64_t adesc = sdesc_k_sw128(s_a + stage * C::kABytes);
           const uint64_t bdesc = sdesc_k_sw128(s_b + stage * C::kBBytes);
           const uint32_t ida = (uint32_t)(kb & 3);
@@ -350,21 +406,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int ks = 0; ks < kBK / 32; ++ks) {
             const uint32_t idb = FP4 ? (uint32_t)ks : ida;
             const uint32_t idesc = C::kIdesc | (ida << 29) | (idb << 4);
-            tc_mma_mxf8f6f4(d_t, adesc + (uint64_t)(ks * 2), bdesc + (uint64_t)(ks * 2), idesc,
-                            sfa_t | (ida << 30), sfb_t | (idb << 30), (kb > kb0 || ks > 0) ? 1u : 0u);
+            if constexpr (kPair)
+              tc_mma_mxf8f6f4_pair(d_t, adesc + (uint64_t)(ks * 2), bdesc + (uint64_t)(ks * 2), idesc,
+                                   sfa_t | (ida << 30), sfb_t | (idb << 30), (kb > kb0 || ks > 0) ? 1u : 0u);
+            else
+              tc_mma_mxf8f6f4(d_t, adesc + (uint64_t)(ks * 2), bdesc + (uint64_t)(ks * 2), idesc,
+                              sfa_t | (ida << 30), sfb_t | (idb << 30), (kb > kb0 || ks > 0) ? 1u : 0u);
           }
-          tc_commit(&empty[stage]);
+          if constexpr (kPair)
+            tc_commit_pair_mc(&empty[stage], 0x3);  // frees the stage in both CTAs
+          else
+            tc_commit(&empty[stage]);
           if (++stage == S) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        tc_commit(&tfull[buf]);
+        if constexpr (kPair)
+          tc_commit_pair_mc(&tfull[buf], 0x3);  // both CTAs' epilogues may read
+        else
+          tc_commit(&tfull[buf]);
         ++local;
       }
       // all tcgen05 work of this thread complete before TMEM is released
-      tc_commit(drain);
+      if constexpr (kPair)
+        tc_commit_pair(drain);
+      else
+        tc_commit(drain);
       uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < limit) {
       }
@@ -380,12 +449,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kChunks = kCols / kEpiCols;     // 32-column chunks of this warp
     uint8_t* stg = s_epi + (warp - 2) * (32 * 64);
     int local = 0;
-    for (int t = blockIdx.x; t < num_units; t += gridDim.x) {
+    // where this warp releases an accumulator buffer: the leader's barrier
+    auto release_acc = [&](int b) {
+      if constexpr (kPair)
+        mbar_arrive_cluster(mapa_shared(&tempty[b], 0));
+      else
+        mbar_arrive(&tempty[b]);
+    };
+    for (int t = unit0; t < num_units; t += unit_step) {
       Unit u = decode_unit<LAYOUT>(t, a, s_prefix);
       if (LAYOUT == kContig && !u.valid) continue;
       const int buf = local % C::kAccBufs;
       const uint32_t use = (uint32_t)(local / C::kAccBufs);
-      const int r0 = u.mb * kBM + q * 32;  // first row of this warp (within the group for masked)
+      const int r0 = u.mb * kTileM + (int)rank * kBM + q * 32;  // first row of this warp (in the group if masked)
       int limit_rows = a.rows;
       if (LAYOUT == kMasked) limit_rows = min(max(__ldg(a.masked_m + u.g), 0), a.rows);
       const int vr = min(32, limit_rows - r0);
@@ -477,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[buf]);
+        if (lane == 0) release_acc(buf);
         ++local;
         continue;
       }
@@ -510,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[buf]);
+      if (lane == 0) release_acc(buf);
       ++local;
     }
     if (lane == 0) bulk_wait_group_all();
@@ -518,10 +594,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  if constexpr (kPair)
+    cluster_sync_all();  // the leader's MMAs (which also write the peer's TMEM) have drained
+  else
+    __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if constexpr (kPair)
+      tmem_dealloc_pair(tmem_base, kTmemCols);
+    else
+      tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 

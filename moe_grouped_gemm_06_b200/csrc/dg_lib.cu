@@ -23,17 +23,29 @@ std::atomic<int> g_pdl{1};  // programmatic dependent launch on (dg_set_pdl)
 // Launches a kernel on `s`, as a programmatic dependent of the previous work
 // on the stream when PDL is enabled.
 template <typename... KArgs, typename... Args>
-cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args&&... args) {
+cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, int cluster,
+                   Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (g_pdl.load()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = g_pdl.load() ? 1 : 0;
+  cfg.numAttrs = n;
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
@@ -108,6 +120,7 @@ constexpr int kBlockNs[] = {128, 192, 256};  // multiples of 64 (see Cfg in dg_g
 
 struct Plan {
   int bn = 128;
+  int ctas = 1;  // 2: a cluster of two CTAs computes 256-row tiles
   int splits = 1;
   int kb_per_split = 1;
   long long units = 0;
@@ -121,24 +134,53 @@ long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
 // overhead of 4 K-blocks), with a 3% surcharge per extra split-K slice for
 // the partial-sum round trip.  Minimised over the instantiated block sizes;
 // ties keep fewer slices, then the larger block.
-// DG_BLOCK_N (one of kBlockNs) restricts the search to that block width.
-int forced_block_n() {
-  static int v = [] {
-    const char* e = std::getenv("DG_BLOCK_N");
-    if (!e) return 0;
-    const int b = std::atoi(e);
-    for (int bn : kBlockNs)
-      if (bn == b) return b;
-    return 0;
-  }();
-  return v;
+// Tile-configuration override (dg_set_tile_config; initial values from the
+// environment variables DG_BLOCK_N and DG_CTAS): restricts the heuristic's
+// search to one block width and/or to single CTAs (1) or CTA pairs (2).
+int env_int(const char* name) {
+  const char* e = std::getenv(name);
+  return e ? std::atoi(e) : 0;
+}
+std::atomic<int> g_force_bn{env_int("DG_BLOCK_N")};
+std::atomic<int> g_force_ctas{env_int("DG_CTAS") == 1 ? 1 : 0};
+
+int forced_ctas() {
+  const int c = g_force_ctas.load();
+  return (c == 1 || c == 2) ? c : 0;
 }
 
-Plan plan_gemm(long long m_blocks, int n, int k, int sms, bool allow_split) {
+int forced_block_n() {
+  const int b = g_force_bn.load();
+  for (int bn : kBlockNs)
+    if (bn == b) return b;
+  return 0;
+}
+
+// CTA pairs (dense only, allow_pair) are costed per cluster: half the SMs,
+// tiles of 256 rows, no split-K, and 0.85x the per-unit time for staging half
+// of B per SM.
+Plan plan_gemm(long long m_blocks, int n, int k, int sms, bool allow_split, bool allow_pair = false) {
   Plan best;
   double best_cost = 1e300;
   const int kb = k / 128;
+  if (allow_pair && m_blocks >= 2 && forced_ctas() != 1) {
+    for (int bn : kBlockNs) {
+      if (bn < 192 || (forced_block_n() && bn != forced_block_n())) continue;
+      const long long units = ((m_blocks + 1) / 2) * ceil_div(n, bn);
+      const double waves = (double)ceil_div(units, sms / 2);
+      const double cost = waves * (double)bn * (kb + 4) * 0.85;
+      if (cost < best_cost * (1 - 1e-9)) {
+        best_cost = cost;
+        best.bn = bn;
+        best.ctas = 2;
+        best.splits = 1;
+        best.kb_per_split = kb;
+        best.units = units;
+      }
+    }
+  }
   for (int bn : kBlockNs) {
+    if (forced_ctas() == 2 && best.ctas == 2) break;
     if (forced_block_n() && bn != forced_block_n()) continue;
     const long long tiles = m_blocks * ceil_div(n, bn);
     const int max_s = allow_split ? std::max(1, std::min(dg::kMaxSplits, kb / 2)) : 1;
@@ -152,14 +194,17 @@ Plan plan_gemm(long long m_blocks, int n, int k, int sms, bool allow_split) {
       if (cost < best_cost * (1 - 1e-9)) {
         best_cost = cost;
         best.bn = bn;
+        best.ctas = 1;
         best.splits = s;
         best.kb_per_split = kbps;
         best.units = units;
       }
     }
   }
-  best.grid = (int)std::min<long long>(best.units, sms);
-  if (best.grid < 1) best.grid = 1;
+  if (best.ctas == 2)
+    best.grid = 2 * (int)std::max<long long>(1, std::min<long long>(best.units, sms / 2));
+  else
+    best.grid = (int)std::max<long long>(1, std::min<long long>(best.units, sms));
   return best;
 }
 
@@ -191,11 +236,11 @@ float* workspace(size_t bytes, cudaStream_t s) {
 
 // ------------------------------------------------------------ launches
 
-template <int BN, bool FP4, int LAYOUT>
-dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td, const dg::GemmArgs& args,
-                      int grid, cudaStream_t s) {
-  using C = dg::Cfg<BN, FP4>;
-  auto kern = dg::gemm_kernel<BN, FP4, LAYOUT>;
+template <int BN, bool FP4, int LAYOUT, int CTAS>
+dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td, const CUtensorMap& tsfa,
+                      const CUtensorMap& tsfb, const dg::GemmArgs& args, int grid, cudaStream_t s) {
+  using C = dg::Cfg<BN, FP4, CTAS>;
+  auto kern = dg::gemm_kernel<BN, FP4, LAYOUT, CTAS>;
   static std::atomic<uint64_t> attr_set_mask{0};  // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
@@ -205,19 +250,24 @@ dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
       return DG_ERR_CUDA;
     attr_set_mask.fetch_or(bit);
   }
-  if (launch(kern, dim3(grid), dim3(dg::kThreads), C::kSmemBytes, s, ta, tb, td, args) != cudaSuccess)
+  if (launch(kern, dim3(grid), dim3(dg::kThreads), C::kSmemBytes, s, CTAS, ta, tb, td, tsfa, tsfb, args) !=
+      cudaSuccess)
     return DG_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return DG_OK;
 }
 
 template <bool FP4, int LAYOUT>
-dg_status dispatch(int bn, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
-                   const dg::GemmArgs& args, int grid, cudaStream_t s) {
+dg_status dispatch(int bn, int ctas, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
+                   const CUtensorMap& tsfa, const CUtensorMap& tsfb, const dg::GemmArgs& args, int grid,
+                   cudaStream_t s) {
+  // CTA-pair (cta_group::2) kernels are not launched: on B200 they stopped
+  // with "illegal instruction" and the cause is not yet known.
+  if (ctas != 1) return DG_ERR_UNSUPPORTED;
   switch (bn) {
-    case 128: return launch_gemm<128, FP4, LAYOUT>(ta, tb, td, args, grid, s);
-    case 192: return launch_gemm<192, FP4, LAYOUT>(ta, tb, td, args, grid, s);
-    case 256: return launch_gemm<256, FP4, LAYOUT>(ta, tb, td, args, grid, s);
+    case 128: return launch_gemm<128, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
+    case 192: return launch_gemm<192, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
+    case 256: return launch_gemm<256, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
     default: return DG_ERR_UNSUPPORTED;
   }
 }
@@ -252,7 +302,7 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
     plan.grid = (int)std::min<long long>((long long)p.groups * m_blocks * ceil_div(p.n, plan.bn), sms);
   } else {
     const bool allow_split = (LAYOUT == dg::kDense) && p.rows <= 1024;
-    plan = plan_gemm(m_blocks, p.n, p.k, sms, allow_split);
+    plan = plan_gemm(m_blocks, p.n, p.k, sms, allow_split, /*allow_pair=*/false);
   }
 
   dg::GemmArgs args{};
@@ -267,7 +317,7 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
   args.n = p.n;
   args.k = p.k;
   args.num_groups = p.groups;
-  args.num_m_blocks = (int)m_blocks;
+  args.num_m_blocks = (int)(plan.ctas == 2 ? ceil_div(p.rows, 2 * dg::kBM) : m_blocks);
   args.num_n_blocks = (int)ceil_div(p.n, plan.bn);
   args.kb_total = p.k / 128;
   args.splits = plan.splits;
@@ -301,25 +351,38 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
                      (uint64_t)p.rows * p.k, 128, dg::kBM, CU_TENSOR_MAP_SWIZZLE_128B);
   if (FP4)
     ok = ok && make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, p.b, p.k, p.n, gb, (uint64_t)p.k / 2,
-                        (uint64_t)p.n * p.k / 2, 128, plan.bn, CU_TENSOR_MAP_SWIZZLE_128B);
+                        (uint64_t)p.n * p.k / 2, 128, plan.bn / plan.ctas, CU_TENSOR_MAP_SWIZZLE_128B);
   else
     ok = ok && make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.b, p.k, p.n, gb, (uint64_t)p.k, (uint64_t)p.n * p.k,
-                        128, plan.bn, CU_TENSOR_MAP_SWIZZLE_128B);
+                        128, plan.bn / plan.ctas, CU_TENSOR_MAP_SWIZZLE_128B);
+  // packed scale words as rows of 128 words (one 128-row chunk per row): the
+  // CTA-pair kernel loads them with tiled copies that can complete on the
+  // leader's barrier; single-CTA kernels use plain bulk copies instead
+  CUtensorMap tsfa = ta, tsfb = ta;
+  if (plan.ctas == 2) {
+    const uint64_t rows_a = (uint64_t)args.sfa_q * args.sfa_chunks;
+    const uint64_t rows_b = (uint64_t)args.sfb_q * args.sfb_chunks;
+    ok = ok && make_map(&tsfa, CU_TENSOR_MAP_DATA_TYPE_INT32, p.sfa, 128, rows_a, 1, 512, rows_a * 512, 128, 1,
+                        CU_TENSOR_MAP_SWIZZLE_NONE);
+    ok = ok && make_map(&tsfb, CU_TENSOR_MAP_DATA_TYPE_INT32, p.sfb, 128, rows_b, 1, 512, rows_b * 512, 128, 1,
+                        CU_TENSOR_MAP_SWIZZLE_NONE);
+  }
   ok = ok && make_map(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.d, p.n, p.rows, ga, (uint64_t)p.n * 2,
                       (uint64_t)p.rows * p.n * 2, dg::kEpiCols, 32, CU_TENSOR_MAP_SWIZZLE_64B);
   if (!ok) return DG_ERR_CUDA;
 
   if (log_enabled())
-    std::fprintf(stderr, "[dg] layout=%d fp4=%d rows=%d n=%d k=%d groups=%d -> block_n=%d splits=%d units=%lld grid=%d\n",
-                 LAYOUT, (int)FP4, p.rows, p.n, p.k, p.groups, plan.bn, plan.splits, plan.units, plan.grid);
+    std::fprintf(stderr,
+                 "[dg] layout=%d fp4=%d rows=%d n=%d k=%d groups=%d -> block_n=%d ctas=%d splits=%d units=%lld grid=%d\n",
+                 LAYOUT, (int)FP4, p.rows, p.n, p.k, p.groups, plan.bn, plan.ctas, plan.splits, plan.units, plan.grid);
 
-  dg_status st = dispatch<FP4, LAYOUT>(plan.bn, ta, tb, td, args, plan.grid, s);
+  dg_status st = dispatch<FP4, LAYOUT>(plan.bn, plan.ctas, ta, tb, td, tsfa, tsfb, args, plan.grid, s);
   if (st != DG_OK || plan.splits == 1) return st;
 
   const long long units = (long long)p.rows * (p.n / 4);
   const int threads = 256;
   const int blocks = (int)std::min<long long>(ceil_div(units, threads), (long long)sms * 8);
-  if (launch(dg::splitk_reduce_kernel, dim3(blocks), dim3(threads), 0, s, (const float*)args.ws, args.c, args.d,
+  if (launch(dg::splitk_reduce_kernel, dim3(blocks), dim3(threads), 0, s, 1, (const float*)args.ws, args.c, args.d,
              p.rows, p.n, plan.splits) != cudaSuccess)
     return DG_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -514,6 +577,19 @@ dg_status dg_set_pdl(int enable) {
 
 int dg_get_pdl(void) { return g_pdl.load(); }
 
+dg_status dg_set_tile_config(int block_n, int ctas) {
+  if (block_n != 0) {
+    bool known = false;
+    for (int bn : kBlockNs) known = known || (bn == block_n);
+    if (!known) return DG_ERR_INVALID_ARG;
+  }
+  if (ctas != 0 && ctas != 1 && ctas != 2) return DG_ERR_INVALID_ARG;
+  if (ctas == 2) return DG_ERR_UNSUPPORTED;  // CTA pairs are not launched (see dispatch)
+  g_force_bn.store(block_n);
+  g_force_ctas.store(ctas);
+  return DG_OK;
+}
+
 dg_status dg_get_last_error(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DG_ERR_CUDA;
   int v = 0;
@@ -547,15 +623,16 @@ const char* dg_status_string(int status) {
 
 uint64_t dg_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
-dg_status dg_query_dense_config(int m, int n, int k, int* block_n, int* splits, int* units, int* grid) {
+dg_status dg_query_dense_config(int m, int n, int k, int* block_n, int* splits, int* units, int* grid, int* ctas) {
   if (m <= 0 || n <= 0 || k <= 0 || k % 128 != 0) return DG_ERR_INVALID_ARG;
   const int sms = num_sms();
   if (sms <= 0) return DG_ERR_CUDA;
-  Plan p = plan_gemm(ceil_div(m, dg::kBM), n, k, sms, m <= 1024);
+  Plan p = plan_gemm(ceil_div(m, dg::kBM), n, k, sms, m <= 1024, /*allow_pair=*/false);
   if (block_n) *block_n = p.bn;
   if (splits) *splits = p.splits;
   if (units) *units = (int)p.units;
   if (grid) *grid = p.grid;
+  if (ctas) *ctas = p.ctas;
   return DG_OK;
 }
 

@@ -133,3 +133,18 @@ def test_heuristic_large_m_has_no_split(dg):
         dg.dg_set_num_sms(0)
     assert cfg["splits"] == 1 and cfg["grid"] == 148
     assert small["splits"] > 1 and small["units"] <= 148
+
+
+def test_tile_config_override_and_pairs_refused(dg):
+    assert dg.lib().dg_set_tile_config(96, 0) == -1          # not an instantiated width
+    assert dg.lib().dg_set_tile_config(0, 2) == -2           # CTA pairs are not launched
+    dg.dg_set_num_sms(148)
+    try:
+        dg.dg_set_tile_config(256, 1)
+        assert dg.dg_query_dense_config(4096, 7168, 16384)["block_n"] == 256
+        dg.dg_set_tile_config(0, 0)
+        for shape in [(4096, 7168, 16384), (4096, 2112, 7168), (256, 7168, 7168)]:
+            assert dg.dg_query_dense_config(*shape)["ctas"] == 1
+    finally:
+        dg.dg_set_tile_config(0, 0)
+        dg.dg_set_num_sms(0)
