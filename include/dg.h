@@ -48,10 +48,11 @@
  * past its time limit, group metadata out of range) are recorded in a
  * device-side error word and reported later by dg_get_last_error().
  *
- * Scratch memory.  The split-K path of the dense calls (chosen by the host
- * heuristic for small M) keeps an FP32 workspace per (device, stream),
- * allocated stream-ordered on first use and grown on demand; dg_shutdown()
- * releases it.  No other call allocates device memory.
+ * Scratch memory.  When the host heuristic shares the K-iterations of some
+ * tiles out over several CTAs (stream-K: small M, or the last partial wave of
+ * tiles), dg_fp8_gemm_nt keeps their FP32 partial sums in a workspace per
+ * (device, stream), allocated stream-ordered on first use and grown on
+ * demand; dg_shutdown() releases it.  No other call allocates device memory.
  */
 #ifndef DG_H_
 #define DG_H_
@@ -72,8 +73,10 @@ typedef enum {
                                 dg_get_last_error)                            */
   DG_ERR_BAD_METADATA = -5,  /* masked_m outside [0, max_m] or m_indices >=
                                 num_groups, seen on the device                */
-  DG_ERR_SCRATCH_LIMIT = -6  /* dg_fp8_gemm_nt_noalloc: the problem needs more
-                                split-K scratch than the fixed array holds    */
+  DG_ERR_SCRATCH_LIMIT = -6  /* reserved: a plan needing more scratch than
+                                the fixed no-alloc array (not returned by this
+                                version, whose no-alloc planner keeps within
+                                the array)                                    */
 } dg_status;
 
 /* ---------------------------------------------------------------- GEMMs */
@@ -129,14 +132,15 @@ dg_status dg_m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa, con
  * own rule forbids cudaMalloc/cudaFree on the hot path (they can synchronise
  * the device and they fail when memory is exhausted).
  *
- * Arguments, results and errors are those of dg_fp8_gemm_nt.  When the host
- * heuristic splits K (small m), the FP32 partial sums go to one fixed device
- * array of dg_noalloc_scratch_bytes() = 32 MiB that is part of this library's
- * device image: every GPU that loads the library holds it until the process
- * exits.  A problem whose split needs more than that (splits * m * n * 4
- * bytes) returns DG_ERR_SCRATCH_LIMIT before anything is launched.  Nothing
- * in the array has to start at zero: every partial that is read is first
- * written by the same call.
+ * Arguments, results and errors are those of dg_fp8_gemm_nt.  Stream-K
+ * partial sums go to one fixed device array of dg_noalloc_scratch_bytes() =
+ * 32 MiB that is part of this library's device image: every GPU that loads
+ * the library holds it until the process exits.  The heuristic only picks
+ * plans whose partials fit in it (whole tiles need none), so the plan -- and
+ * the rounding of the result -- can differ from dg_fp8_gemm_nt's for
+ * problems whose best stream-K split needs more; dg_query_dense_config with
+ * that cap shows the plan.  Nothing in the array has to start at zero: every
+ * partial that is read is first written by the same call.
  *
  * All calls on a device share the array and it keeps the last call's
  * contents, so two calls whose kernels overlap on the GPU (different streams,
@@ -209,12 +213,16 @@ dg_status dg_set_num_sms(int num_sms);
 dg_status dg_set_pdl(int enable);
 int dg_get_pdl(void);
 
-/* Restricts the tile heuristic to one configuration: block_n in {128, 192,
- * 256} (0 = any) and ctas 1 (single-CTA 128-row tiles) or 0 (any); ctas = 2
- * (CTA-pair tiles) returns DG_ERR_UNSUPPORTED in this version.  Meant for
- * tuning and tests; the default (0, 0) is the heuristic.  The environment
- * variable DG_BLOCK_N sets the initial block width. */
-dg_status dg_set_tile_config(int block_n, int ctas);
+/* Restricts the tile heuristic (all later calls, all threads): block_n in
+ * {128, 160, 192, 224, 256} (0 = the heuristic's choice among 128, 192, 256;
+ * 160 and 224 are only used when forced) and schedule 0 (heuristic), 1
+ * (whole tiles only), 2 (the last tiles cut into per-tile K-slices, one per
+ * CTA) or 3 (stream-K: the last tiles' K-iterations shared evenly over the
+ * grid); 2 and 3 apply to the dense calls whenever such a split exists.
+ * Anything else returns DG_ERR_INVALID_ARG and changes nothing.  Meant for
+ * tuning and tests.  The environment variables DG_BLOCK_N and DG_SCHEDULE set
+ * the initial values. */
+dg_status dg_set_tile_config(int block_n, int schedule);
 
 /* Row alignment of groups in the contiguous layout: 128. */
 int dg_get_mk_alignment_for_contiguous_layout(void);
@@ -234,17 +242,25 @@ const char* dg_status_string(int status);
 /* Kernels this library has launched in this process (all devices). */
 uint64_t dg_launch_count(void);
 
-/* Configuration the dense heuristic picks for (m, n, k): block_n, split-K
- * slices, work units (tiles x slices), grid size in CTAs and CTAs per tile
- * (1 or 2) (any pointer may be NULL). */
-dg_status dg_query_dense_config(int m, int n, int k, int* block_n, int* splits, int* units, int* grid, int* ctas);
+/* Plan the dense heuristic picks for (m, n, k) with at most workspace_cap
+ * bytes of workspace (0: no cap, the plan of dg_fp8_gemm_nt;
+ * dg_noalloc_scratch_bytes(): the plan of dg_fp8_gemm_nt_noalloc): block_n,
+ * tiles computed whole (dp_tiles), tiles after them whose K-blocks are
+ * shared over several CTAs (sk_tiles, 0 = none), how: sk_split > 0 = each
+ * cut into that many equal K-slices, 0 = stream-K (even shares of all their
+ * K-blocks over the grid), workspace slots per shared tile, grid size in CTAs
+ * and workspace bytes.  Any output pointer may be NULL.  DG_ERR_INVALID_ARG
+ * for m, n <= 0, k not a positive multiple of 128 or a negative cap. */
+dg_status dg_query_dense_config(int m, int n, int k, int64_t workspace_cap, int* block_n, int* dp_tiles,
+                                int* sk_tiles, int* sk_split, int* max_segments, int* grid,
+                                int64_t* workspace_bytes);
 
 /* Output tiles of an m x n problem cut into block_m x block_n tiles (the
  * count the heuristic balances against the SM count; "DeepSeek 开源第三弹 ...
  * DeepGEMM" (app.myzaker.com), section "非对齐块大小"). */
 int64_t dg_num_tiles(int m, int n, int block_m, int block_n);
 
-/* Releases the split-K workspaces of all devices (synchronises each). */
+/* Releases the stream-K workspaces of all devices (synchronises each). */
 void dg_shutdown(void);
 
 #ifdef __cplusplus

@@ -58,7 +58,7 @@ SYMBOLS = {
     "dg_debug_starved_wait": (_INT, [ctypes.c_uint, _VP]),
     "dg_status_string": (ctypes.c_char_p, [_INT]),
     "dg_launch_count": (ctypes.c_uint64, []),
-    "dg_query_dense_config": (_INT, [_INT, _INT, _INT, _VP, _VP, _VP, _VP, _VP]),
+    "dg_query_dense_config": (_INT, [_INT, _INT, _INT, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "dg_num_tiles": (_I64, [_INT, _INT, _INT, _INT]),
     "dg_shutdown": (None, []),
 }
@@ -213,8 +213,9 @@ def dg_set_pdl(enable: bool) -> None:
     _check(lib().dg_set_pdl(int(bool(enable))), "dg_set_pdl")
 
 
-def dg_set_tile_config(block_n: int = 0, ctas: int = 0) -> None:
-    _check(lib().dg_set_tile_config(int(block_n), int(ctas)), "dg_set_tile_config")
+def dg_set_tile_config(block_n: int = 0, schedule: int = 0) -> None:
+    """block_n: 0 = heuristic; schedule: 0 heuristic, 1 whole tiles, 2 per-tile K-slices, 3 stream-K."""
+    _check(lib().dg_set_tile_config(int(block_n), int(schedule)), "dg_set_tile_config")
 
 
 def dg_get_pdl() -> bool:
@@ -238,10 +239,12 @@ def dg_launch_count() -> int:
     return int(lib().dg_launch_count())
 
 
-def dg_query_dense_config(m: int, n: int, k: int) -> dict:
-    vals = [ctypes.c_int(0) for _ in range(5)]
-    _check(lib().dg_query_dense_config(m, n, k, *[ctypes.byref(v) for v in vals]), "dg_query_dense_config")
-    return dict(zip(("block_n", "splits", "units", "grid", "ctas"), (v.value for v in vals)))
+def dg_query_dense_config(m: int, n: int, k: int, workspace_cap: int = 0) -> dict:
+    vals = [ctypes.c_int(0) for _ in range(6)] + [ctypes.c_int64(0)]
+    _check(lib().dg_query_dense_config(m, n, k, int(workspace_cap), *[ctypes.byref(v) for v in vals]),
+           "dg_query_dense_config")
+    keys = ("block_n", "dp_tiles", "sk_tiles", "sk_split", "max_segments", "grid", "workspace_bytes")
+    return dict(zip(keys, (v.value for v in vals)))
 
 
 def dg_num_tiles(m: int, n: int, block_m: int, block_n: int) -> int:

@@ -22,8 +22,8 @@
 //   warps 2..9  epilogue, two warps per TMEM sub-partition (one column half
 //               each): C prefetched into registers, tcgen05.ld -> (+C) ->
 //               bf16 -> swizzled smem -> TMA store; rows past a masked
-//               group's count are never written.  With split-K they write
-//               FP32 partials, summed by splitk_reduce_kernel.
+//               group's count are never written.  Stream-K pieces go to
+//               FP32 workspace slots, summed by sk_reduce_kernel.
 //
 // The scales are applied inside the MMA: the UE8M0 code of a 1x128 group is
 // used for each of the four K=32 steps of its 128-wide block (the instruction
@@ -50,7 +50,7 @@ struct GemmArgs {
   const int32_t* sfb;        // packed scale words of B
   const uint16_t* c;         // bf16 bits [rows][n] or nullptr
   uint16_t* d;               // bf16 bits (predicated-store path)
-  float* ws;                 // split-K partials [splits][rows][n]
+  float* ws;                 // stream-K partials [sk_tiles][max_seg][kBM][BN] (FP32)
   const int32_t* m_indices;  // contiguous: group of each row (-1 = padding)
   const int32_t* masked_m;   // masked: valid rows per group
   int rows;                  // dense: M; contiguous: M_total; masked: max_m
@@ -59,7 +59,17 @@ struct GemmArgs {
   int num_m_blocks;          // per group for masked
   int num_n_blocks;
   int kb_total;              // k / 128
-  int splits, kb_per_split;
+  // dense schedule: the first dp_tiles tiles (raster order) are computed
+  // whole, round robin over the CTAs; the K-iterations of the sk_tiles tiles
+  // after them are shared out:
+  //   sk_split = s > 0: tile j's K-blocks cut into s equal slices, slice t on
+  //                     CTA j*s + t (one piece per CTA, slot t);
+  //   sk_split = 0:     stream-K: sk_iters = sk_tiles x kb_total iterations,
+  //                     CTA c taking [c sk_iters / G, (c + 1) sk_iters / G),
+  //                     slot = CTA - first CTA of the tile.
+  // A tile's pieces land in its max_seg workspace slots.
+  int dp_tiles, sk_tiles, max_seg, sk_split;
+  long long sk_iters;
   int sfa_chunks, sfb_chunks;          // ceil(rows/128), ceil(n/128)
   long long sfa_group_words, sfb_group_words;
   int sfa_q, sfb_q;                    // packed groups along K
@@ -71,22 +81,27 @@ struct GemmArgs {
 template <int BN, bool FP4, int CTAS = 1>
 struct Cfg {
   // The scale-factor operand of the MMA is addressed in TMEM columns of 32
-  // rows (a 128-row chunk spans 4 columns), and that address must be even:
-  // a tile starting 32 or 96 rows into a chunk (odd column) faults with a
-  // misaligned-address error.  Block widths are therefore multiples of 64, so
-  // a tile starts 0 or 64 rows into its first chunk.
-  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
-  static constexpr int kSfbChunks = 3;                       // 128-row scale chunks a tile can touch
+  // rows (a 128-row chunk spans 4 columns), and that address must be even: a
+  // tile starting 32 or 96 rows into a chunk (odd column) faults with a
+  // misaligned-address error.  Tiles of a width that is not a multiple of 64
+  // therefore have their B scale words re-based in shared memory (kRebase) so
+  // that the MMA reads them from column offset 0.
+  static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "BN");
+  static constexpr int kMaxOffRows = (BN % 128 == 0) ? 0 : (BN % 64 == 0 ? 64 : 96);
+  static constexpr int kSfbChunks = (kMaxOffRows + BN + 127) / 128;  // 128-row scale chunks a tile can touch
+  static constexpr bool kRebase = (BN % 64 != 0);
+  static constexpr int kSfrChunks = (BN + 127) / 128;                // re-based chunks (tile rows only)
+  static constexpr int kSfrBytes = kRebase ? kSfrChunks * 512 : 0;
   // FP32 accumulator buffers in TMEM: three of 128 columns (BN = 128), two at
   // columns 0 and 256 (BN = 192), one (BN = 256); scale factors after them.
-  static constexpr int kAccBufs = (BN <= 128) ? 3 : (BN <= 224 ? 2 : 1);
+  static constexpr int kAccBufs = (BN <= 128) ? 3 : (BN <= 240 ? 2 : 1);
   static constexpr int kABytes = kBM * kBK;                  // 16 KB
   static constexpr int kBRows = BN / CTAS;                   // B rows each CTA of a pair loads
   static constexpr int kBBytes = kBRows * kBK;               // smem bytes (FP4 lands padded to 1 B/elt)
   static constexpr int kBTxBytes = FP4 ? kBBytes / 2 : kBBytes;  // bytes the TMA copy reports (packed)
   static constexpr int kSfaBytes = 512;
   static constexpr int kSfbBytes = kSfbChunks * 512;
-  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes + kSfrBytes;
   static constexpr int kEpiBytes = kEpiWarps * 32 * 64;        // one 32 x 64 B staging box per epilogue warp
   static constexpr int kMaskBytes = ((kMaxMaskedGroups + 1) * 4 + 15) / 16 * 16;
   static constexpr int kBarBytes = 256;
@@ -108,48 +123,111 @@ struct Cfg {
 };
 
 struct Unit {
-  int g, mb, nb, split;
+  int g, mb, nb;
+  int kb0, kb1;   // K-blocks of this unit
+  int slot;       // stream-K workspace slot, -1: the whole tile (result to D)
+  int sk;         // stream-K tile index (slot >= 0)
   bool valid;
 };
 
-// Work-unit order: split-K slice slowest, then L2-rasterised (m, n) tiles in
-// bands of `raster` m-blocks (m fastest inside a band), so that the CTAs
-// running at the same time share the A rows and B columns of one band.
-// Masked: group by group, n-blocks, m-blocks fastest (m-blocks of a group
-// share its B tiles).
-template <int LAYOUT>
-__device__ __forceinline__ Unit decode_unit(int t, const GemmArgs& a, const int* s_prefix) {
-  Unit u;
-  u.valid = true;
-  if (LAYOUT == kMasked) {
-    int g = 0;
-    while (s_prefix[g + 1] <= t) ++g;
-    int local = t - s_prefix[g];
-    int valid_rows = min(max(__ldg(a.masked_m + g), 0), a.rows);
-    int mcount = (valid_rows + kBM - 1) / kBM;
-    u.g = g;
-    u.nb = local / mcount;
-    u.mb = local % mcount;
-    u.split = 0;
-    return u;
-  }
-  int tiles = a.num_m_blocks * a.num_n_blocks;
-  u.split = t / tiles;
-  int tl = t - u.split * tiles;
-  int band_tiles = a.raster * a.num_n_blocks;
-  int band = tl / band_tiles;
-  int rem = tl - band * band_tiles;
-  int band_rows = min(a.raster, a.num_m_blocks - band * a.raster);
-  u.mb = band * a.raster + rem % band_rows;
-  u.nb = rem / band_rows;
-  u.g = 0;
-  if (LAYOUT == kContig) {
-    int g = __ldg(a.m_indices + (long long)u.mb * kBM);  // 1-CTA tiles only
-    u.g = g;
-    u.valid = (g >= 0 && g < a.num_groups);
-  }
-  return u;
+// Stream-K bookkeeping (host and device): the CTA whose share of the G-way
+// even split of `iters` iterations contains iteration x, and the first
+// iteration of CTA c.  Valid for iters >= G (every share non-empty).
+__host__ __device__ __forceinline__ int sk_cta_of(long long x, int G, long long iters) {
+  return (int)(((x + 1) * G - 1) / iters);
 }
+__host__ __device__ __forceinline__ long long sk_begin(int c, int G, long long iters) {
+  return (long long)c * iters / G;
+}
+
+// (m-block, n-block) of tile tl in raster order: bands of `raster` m-blocks,
+// m fastest inside a band, so that the CTAs running at the same time share
+// the A rows and B columns of one band.
+__host__ __device__ __forceinline__ void raster_tile(int tl, int raster, int num_m_blocks, int num_n_blocks,
+                                                     int& mb, int& nb) {
+  const int band_tiles = raster * num_n_blocks;
+  const int band = tl / band_tiles;
+  const int rem = tl - band * band_tiles;
+  const int band_rows = min(raster, num_m_blocks - band * raster);
+  mb = band * raster + rem % band_rows;
+  nb = rem / band_rows;
+}
+
+// Work units of one CTA, in the order all three roles walk them.
+// Dense: the whole tiles t = cta, cta + G, ... below dp_tiles, then this
+// CTA's stream-K share cut at tile boundaries.  Contiguous: every tile of the
+// raster order round robin (a tile's group from its first row).  Masked:
+// group by group, n-blocks, m-blocks fastest (m-blocks of a group share its B
+// tiles).
+template <int LAYOUT>
+struct WorkIter {
+  int t, step, cta;
+  long long x, x_end;  // stream-K iterations of this CTA still to walk
+
+  __device__ __forceinline__ WorkIter(const GemmArgs& a, int cta_, int G) : t(cta_), step(G), cta(cta_) {
+    x = x_end = 0;
+    if (LAYOUT == kDense && a.sk_tiles > 0) {
+      if (a.sk_split > 0) {
+        x_end = (cta_ < a.sk_tiles * a.sk_split) ? 1 : 0;  // one piece
+      } else {
+        x = sk_begin(cta_, G, a.sk_iters);
+        x_end = sk_begin(cta_ + 1, G, a.sk_iters);
+      }
+    }
+  }
+
+  __device__ __forceinline__ bool next(const GemmArgs& a, const int* s_prefix, int num_units, Unit& u) {
+    u.valid = true;
+    u.g = 0;
+    u.slot = -1;
+    u.sk = 0;
+    u.kb0 = 0;
+    u.kb1 = a.kb_total;
+    if (t < num_units) {
+      if (LAYOUT == kMasked) {
+        int g = 0;
+        while (s_prefix[g + 1] <= t) ++g;
+        const int local = t - s_prefix[g];
+        const int valid_rows = min(max(__ldg(a.masked_m + g), 0), a.rows);
+        const int mcount = (valid_rows + kBM - 1) / kBM;
+        u.g = g;
+        u.nb = local / mcount;
+        u.mb = local % mcount;
+      } else {
+        raster_tile(t, a.raster, a.num_m_blocks, a.num_n_blocks, u.mb, u.nb);
+        if (LAYOUT == kContig) {
+          const int g = __ldg(a.m_indices + (long long)u.mb * kBM);  // 1-CTA tiles only
+          u.g = g;
+          u.valid = (g >= 0 && g < a.num_groups);
+        }
+      }
+      t += step;
+      return true;
+    }
+    if (LAYOUT != kDense || x >= x_end) return false;
+    const int kbt = a.kb_total;
+    if (a.sk_split > 0) {
+      const int j = cta / a.sk_split;
+      const int t = cta - j * a.sk_split;
+      u.sk = j;
+      u.slot = t;
+      u.kb0 = (int)((long long)t * kbt / a.sk_split);
+      u.kb1 = (int)((long long)(t + 1) * kbt / a.sk_split);
+      raster_tile(a.dp_tiles + j, a.raster, a.num_m_blocks, a.num_n_blocks, u.mb, u.nb);
+      x = x_end;
+      return true;
+    }
+    const int j = (int)(x / kbt);
+    u.sk = j;
+    u.kb0 = (int)(x - (long long)j * kbt);
+    const long long left = x_end - x;
+    u.kb1 = (left < (long long)(kbt - u.kb0)) ? u.kb0 + (int)left : kbt;
+    u.slot = cta - sk_cta_of((long long)j * kbt, step, a.sk_iters);
+    raster_tile(a.dp_tiles + j, a.raster, a.num_m_blocks, a.num_n_blocks, u.mb, u.nb);
+    x += u.kb1 - u.kb0;
+    return true;
+  }
+};
 
 // CTAS = 2: a cluster of two CTAs computes 256 x BN tiles (dense layout only);
 // tm_sfa / tm_sfb view the packed scale words as rows of 512 bytes so that
@@ -170,7 +248,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* s_b = s_a + S * C::kABytes;
   uint8_t* s_sfa = s_b + S * C::kBBytes;
   uint8_t* s_sfb = s_sfa + S * C::kSfaBytes;
-  uint8_t* s_epi = s_sfb + S * C::kSfbBytes;
+  uint8_t* s_sfr = s_sfb + S * C::kSfbBytes;   // re-based B scale words (kRebase only)
+  uint8_t* s_epi = s_sfr + S * C::kSfrBytes;
   int* s_prefix = reinterpret_cast<int*>(s_epi + C::kEpiBytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(s_prefix) + C::kMaskBytes);
   uint64_t* full = bars;
@@ -185,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t lane = lane_id();
   const GemmArgs& a = args;
   const uint32_t rank = kPair ? cluster_ctarank() : 0u;   // 0 = leader (issues the MMAs)
-  const int unit0 = blockIdx.x / CTAS, unit_step = gridDim.x / CTAS;
+  const int cta_id = blockIdx.x / CTAS, num_ctas = gridDim.x / CTAS;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -248,8 +327,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *s_tmem;
   if (LAYOUT == kMasked)
     num_units = s_prefix[a.num_groups];
+  else if (LAYOUT == kDense)
+    num_units = a.dp_tiles;
   else
-    num_units = a.num_m_blocks * a.num_n_blocks * a.splits;
+    num_units = a.num_m_blocks * a.num_n_blocks;
 
   const uint64_t limit = a.timeout_ns;
 
@@ -261,14 +342,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t filled_phase[8];
       uint32_t filled_mask = 0;
       bool ok = true;
-      for (int t = unit0; t < num_units && ok; t += unit_step) {
-        Unit u = decode_unit<LAYOUT>(t, a, s_prefix);
+      WorkIter<LAYOUT> it(a, cta_id, num_ctas);
+      Unit u;
+      while (ok && it.next(a, s_prefix, num_units, u)) {
         if (LAYOUT == kContig && !u.valid) {
           if (u.g >= a.num_groups) record_error(-5);
           continue;
         }
-        const int kb0 = u.split * a.kb_per_split;
-        const int kb1 = min(a.kb_total, kb0 + a.kb_per_split);
+        const int kb0 = u.kb0;
+        const int kb1 = u.kb1;
         const int n0 = u.nb * BN;
         const int c0 = n0 / 128;
         const int c1 = (min(n0 + BN, a.n) - 1) / 128;
@@ -355,20 +437,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // One lane waits on the barriers and issues every tcgen05 operation (a
+    // warp-wide loop with per-K-block warp synchronisation measured 1.8x
+    // slower).  It also re-bases the B scale words when a tile starts an odd
+    // number of 32-row groups into its first scale chunk.
     if (lane == 0 && rank == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
       const uint32_t sfa_t = tmem_base + C::kColSfa;
-      for (int t = unit0; t < num_units && ok; t += unit_step) {
-        Unit u = decode_unit<LAYOUT>(t, a, s_prefix);
+      WorkIter<LAYOUT> it(a, cta_id, num_ctas);
+      Unit u;
+      while (ok && it.next(a, s_prefix, num_units, u)) {
         if (LAYOUT == kContig && !u.valid) continue;
-        const int kb0 = u.split * a.kb_per_split;
-        const int kb1 = min(a.kb_total, kb0 + a.kb_per_split);
+        const int kb0 = u.kb0;
+        const int kb1 = u.kb1;
         const int n0 = u.nb * BN;
         const int nchunks = (min(n0 + BN, a.n) - 1) / 128 - n0 / 128 + 1;
-        const uint32_t sfb_t = tmem_base + C::kColSfb + (uint32_t)((n0 % 128) / 32);
+        const int off = (n0 % 128) / 32;  // 32-row groups into the first scale chunk
+        const bool rebase = C::kRebase && (off & 1);
+        const uint32_t sfb_t = tmem_base + C::kColSfb + (uint32_t)(rebase ? 0 : off);
         const int buf = local % C::kAccBufs;
         const uint32_t use = (uint32_t)(local / C::kAccBufs);
         if (!dg_wait(&tempty[buf], (use & 1) ^ 1, s_abort, limit)) {
@@ -385,20 +474,48 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const bool new_sfa = ((kb & 3) == 0) || kb == kb0;
           const bool new_sfb = FP4 || new_sfa;
+          const uint8_t* sfb_src = s_sfb + stage * C::kSfbBytes;
+          uint8_t* sfb_reb = s_sfr + stage * C::kSfrBytes;
+          if (C::kRebase && rebase && new_sfb) {
+            // word w of line l of re-based chunk v = word (off + w) % 4 of line
+            // l of loaded chunk v + (off + w) / 4 (chunks past the loaded range
+            // only feed rows outside the tile)
+            for (int l = 0; l < 32; ++l) {
+              uint4 ld[C::kSfbChunks];
+#pragma unroll
+              for (int c = 0; c < C::kSfbChunks; ++c)
+                ld[c] = *reinterpret_cast<const uint4*>(sfb_src + c * 512 + l * 16);
+#pragma unroll
+              for (int v = 0; v < C::kSfrChunks; ++v) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                  const int j = off + w;
+                  const uint4 q4 = ld[min(v + (j >> 2), C::kSfbChunks - 1)];
+                  const int e = j & 3;
+                  w4[w] = e == 0 ? q4.x : (e == 1 ? q4.y : (e == 2 ? q4.z : q4.w));
+                }
+                *reinterpret_cast<uint4*>(sfb_reb + v * 512 + l * 16) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+              }
+            }
+            fence_proxy_async_smem();
+          }
           if (new_sfa) {
             if constexpr (kPair)
               tc_cp_32x128b_x4_pair(sfa_t, sdesc_sf_32x16(s_sfa + stage * C::kSfaBytes));
             else
               tc_cp_32x128b_x4(sfa_t, sdesc_sf_32x16(s_sfa + stage * C::kSfaBytes));
           }
-          if (new_sfb)
-            for (int ch = 0; ch < nchunks; ++ch) {
-              const uint64_t sd = sdesc_sf_32x16(s_sfb + stage * C::kSfbBytes + ch * 512);
+          if (new_sfb) {
+            const int ncp = rebase ? C::kSfrChunks : nchunks;
+            for (int ch = 0; ch < ncp; ++ch) {
+              const uint64_t sd = sdesc_sf_32x16((rebase ? sfb_reb : sfb_src) + ch * 512);
               if constexpr (kPair)
                 tc_cp_32x128b_x4_pair(tmem_base + C::kColSfb + 4 * ch, sd);
               else
                 tc_cp_32x128b_x4(tmem_base + C::kColSfb + 4 * ch, sd);
             }
+          }
           const uint64_t adesc = sdesc_k_sw128(s_a + stage * C::kABytes);
           const uint64_t bdesc = sdesc_k_sw128(s_b + stage * C::kBBytes);
           const uint32_t ida = (uint32_t)(kb & 3);
@@ -445,19 +562,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     // registers before waiting for its accumulator, so they overlap the MMAs.
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
-    constexpr int kCols = BN / 2;                 // columns of this warp
-    constexpr int kChunks = kCols / kEpiCols;     // 32-column chunks of this warp
+    constexpr int kNch = BN / kEpiCols;           // 32-column chunks of the tile
+    constexpr int kChunks = (kNch + 1) / 2;       // chunks of the first half; the second has kNch - kChunks
+    constexpr int kCols = kChunks * kEpiCols;     // column offset of the second half
+    const int nch_w = half ? (kNch - kChunks) : kChunks;  // chunks of this warp
     uint8_t* stg = s_epi + (warp - 2) * (32 * 64);
     int local = 0;
     // where this warp releases an accumulator buffer: the leader's barrier
+    // C of one unit for this warp's 32 rows x kCols columns (zeros where there
+    // is no C or no row), read row-wise into registers
+    auto load_c_rows = [&](uint4 (&dst)[kChunks][4], const Unit& uu, bool want) {
+#pragma unroll
+      for (int j = 0; j < kChunks; ++j)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) dst[j][v] = make_uint4(0u, 0u, 0u, 0u);
+      const int rr0 = uu.mb * kTileM + (int)rank * kBM + q * 32;
+      int lim = a.rows;
+      if (LAYOUT == kMasked) lim = min(max(__ldg(a.masked_m + uu.g), 0), a.rows);
+      const int rrow = rr0 + (int)lane;
+      const long long rg = (LAYOUT == kMasked) ? (long long)uu.g * a.rows + rrow : rrow;
+      const int cw = uu.nb * BN + half * kCols;
+      if (want && rrow < lim &&
+          DG_CHECK(((reinterpret_cast<uintptr_t>(a.c + rg * a.n + cw) & 15) == 0) && rrow < a.rows && rg >= 0, 1)) {
+        const uint4* src = reinterpret_cast<const uint4*>(a.c + rg * a.n + cw);
+#pragma unroll
+        for (int j = 0; j < kChunks; ++j)
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            if (j < nch_w && cw + j * kEpiCols + 8 * v < a.n) dst[j][v] = __ldg(src + j * 4 + v);
+      }
+    };
+    // one unit of look-ahead for C where registers allow
+    constexpr bool kPrefetchC = (kChunks <= 3);
+    uint4 cnext[kChunks][4];
+    bool have_next_c = false;  // cnext holds C of the next unit this warp drains
+    (void)cnext;
     auto release_acc = [&](int b) {
       if constexpr (kPair)
         mbar_arrive_cluster(mapa_shared(&tempty[b], 0));
       else
         mbar_arrive(&tempty[b]);
     };
-    for (int t = unit0; t < num_units; t += unit_step) {
-      Unit u = decode_unit<LAYOUT>(t, a, s_prefix);
+    WorkIter<LAYOUT> it(a, cta_id, num_ctas);
+    Unit u;
+    while (it.next(a, s_prefix, num_units, u)) {
       if (LAYOUT == kContig && !u.valid) continue;
       const int buf = local % C::kAccBufs;
       const uint32_t use = (uint32_t)(local / C::kAccBufs);
@@ -470,20 +618,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int colw = u.nb * BN + half * kCols;  // first column of this warp
 
       uint4 creg[kChunks][4];
-      const bool load_c = a.c != nullptr && a.splits == 1;
+      const bool load_c = a.c != nullptr && u.slot < 0;
+      if constexpr (kPrefetchC) {
+        if (have_next_c) {
+          // C of this unit was loaded while the previous unit was stored
 #pragma unroll
-      for (int j = 0; j < kChunks; ++j)
+          for (int j = 0; j < kChunks; ++j)
 #pragma unroll
-        for (int v = 0; v < 4; ++v) creg[j][v] = make_uint4(0u, 0u, 0u, 0u);
-      if (load_c && (int)lane < vr &&
-          DG_CHECK(((reinterpret_cast<uintptr_t>(a.c + grow * a.n + colw) & 15) == 0) && row < a.rows && grow >= 0,
-                   1)) {
-        const uint4* src = reinterpret_cast<const uint4*>(a.c + grow * a.n + colw);
-#pragma unroll
-        for (int j = 0; j < kChunks; ++j)
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            if (colw + j * kEpiCols + 8 * v < a.n) creg[j][v] = __ldg(src + j * 4 + v);
+            for (int v = 0; v < 4; ++v) creg[j][v] = cnext[j][v];
+        } else {
+          load_c_rows(creg, u, load_c);
+        }
+        // issue the loads of the next unit's C now, so that they arrive while
+        // this unit is drained and stored
+        have_next_c = false;
+        if (a.c != nullptr) {
+          WorkIter<LAYOUT> peek = it;
+          Unit un;
+          if (peek.next(a, s_prefix, num_units, un) && un.valid && un.slot < 0) {
+            load_c_rows(cnext, un, true);
+            have_next_c = true;
+          }
+        }
+      } else {
+        load_c_rows(creg, u, load_c);
       }
 
       int ok = 1;
@@ -527,22 +685,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
 
-      if (a.splits > 1) {
-        // ---- split-K: this slice's FP32 partials; splitk_reduce_kernel sums
-        // the slices in slice order (+C) and writes D
+      if (u.slot >= 0) {
+        // ---- stream-K piece: FP32 partial sums of kb0..kb1 into the tile's
+        // workspace slot; sk_reduce_kernel adds the slots in K order (+C)
+        // and writes D
+        float* tile_ws = a.ws + ((long long)u.sk * a.max_seg + u.slot) * (kBM * BN);
 #pragma unroll
         for (int j = 0; j < kChunks; ++j) {
           const int col0 = colw + j * kEpiCols;
-          if (vr > 0 && col0 < a.n) {
+          if (j < nch_w && vr > 0 && col0 < a.n) {
             uint32_t acc[kEpiCols];
             tc_ld_32x32b_x32(t_row + j * kEpiCols, acc);
             tc_wait_ld_regs(acc);
+            float* dst_row = tile_ws + (q * 32 + (int)lane) * BN + (col0 - u.nb * BN);
             if ((int)lane < vr &&
-                DG_CHECK(a.ws != nullptr && u.split < a.splits && row < a.rows &&
-                             (reinterpret_cast<uintptr_t>(a.ws + ((long long)u.split * a.rows + row) * a.n + col0) &
-                              15) == 0,
+                DG_CHECK(!kPair && a.ws != nullptr && u.sk < a.sk_tiles && u.slot < a.max_seg && row < a.rows &&
+                             (reinterpret_cast<uintptr_t>(dst_row) & 15) == 0,
                          3)) {
-              float4* dst = reinterpret_cast<float4*>(a.ws + ((long long)u.split * a.rows + row) * a.n + col0);
+              float4* dst = reinterpret_cast<float4*>(dst_row);
 #pragma unroll
               for (int v = 0; v < kEpiCols / 4; ++v)
                 if (col0 + 4 * v < a.n)
@@ -561,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int j = 0; j < kChunks; ++j) {
         const int col0 = colw + j * kEpiCols;
-        if (vr > 0 && col0 < a.n) {
+        if (j < nch_w && vr > 0 && col0 < a.n) {
           uint32_t acc[kEpiCols];
           DG_CHECK(((t_row & 0xFFFF) + j * kEpiCols + kEpiCols <= (uint32_t)kTmemCols) &&
                        ((t_row >> 16) & 0xFFFF) == (uint32_t)(q * 32) + (tmem_base >> 16) && (warp & 3) == q,
@@ -607,41 +767,66 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Split-K reduction: D = bf16(sum_s ws[s] + C) with the slices summed in
-// slice order (deterministic).  4 columns per thread; the loads of all
-// slices are issued before the first add (at most kMaxSplits slices).
-constexpr int kMaxSplits = 16;
-__global__ void splitk_reduce_kernel(const float* __restrict__ ws, const uint16_t* __restrict__ c,
-                                     uint16_t* __restrict__ d, int rows, int n, int splits) {
+// Stream-K fix-up: for every stream-K tile, D = bf16(sum of its workspace
+// slots in slot (= K) order + C), so the result does not depend on timing.
+// One thread per 4 columns of a tile row; the slots are loaded 8 at a time
+// before they are added.
+struct SkReduceArgs {
+  const float* ws;
+  const uint16_t* c;
+  uint16_t* d;
+  int rows, n, bn;
+  int kb_total, dp_tiles, sk_tiles, max_seg, sk_split, ctas;
+  long long sk_iters;
+  int raster, num_m_blocks, num_n_blocks;
+};
+
+__global__ void __launch_bounds__(256) sk_reduce_kernel(const SkReduceArgs r) {
   pdl_wait();
-  const long long units = (long long)rows * (n / 4);
-  for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < units;
-       u += (long long)gridDim.x * blockDim.x) {
-    const long long r = u / (n / 4);
-    const int col = (int)(u - r * (n / 4)) * 4;
-    const float4* p = reinterpret_cast<const float4*>(ws + r * n + col);
-    const long long slice = (long long)rows * n / 4;  // float4 stride between slices
-    float4 part[kMaxSplits];
-#pragma unroll
-    for (int s = 0; s < kMaxSplits; ++s)
-      part[s] = (s < splits) ? __ldg(p + s * slice) : make_float4(0.f, 0.f, 0.f, 0.f);
-    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-#pragma unroll
-    for (int s = 0; s < kMaxSplits; ++s) {
-      acc0 += part[s].x;
-      acc1 += part[s].y;
-      acc2 += part[s].z;
-      acc3 += part[s].w;
+  const int q4 = r.bn / 4;
+  const int per_tile = kBM * q4;
+  const long long items = (long long)r.sk_tiles * per_tile;
+  const long long slot4 = (long long)kBM * r.bn / 4;  // float4s between slots
+  for (long long it = blockIdx.x * (long long)blockDim.x + threadIdx.x; it < items;
+       it += (long long)gridDim.x * blockDim.x) {
+    const int j = (int)(it / per_tile);
+    const int rem = (int)(it - (long long)j * per_tile);
+    const int lr = rem / q4;
+    const int lc = (rem - lr * q4) * 4;
+    int mb, nb;
+    raster_tile(r.dp_tiles + j, r.raster, r.num_m_blocks, r.num_n_blocks, mb, nb);
+    const int row = mb * kBM + lr;
+    const int col = nb * r.bn + lc;
+    if (row >= r.rows || col >= r.n) continue;
+    int nseg = r.sk_split;
+    if (nseg == 0) {
+      const long long x0 = (long long)j * r.kb_total;
+      nseg = sk_cta_of(x0 + r.kb_total - 1, r.ctas, r.sk_iters) - sk_cta_of(x0, r.ctas, r.sk_iters) + 1;
     }
-    if (c != nullptr) {
-      const uint2 w = __ldg(reinterpret_cast<const uint2*>(c + r * n + col));
+    const float4* p = reinterpret_cast<const float4*>(r.ws + ((long long)j * r.max_seg * kBM + lr) * r.bn + lc);
+    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+    for (int s0 = 0; s0 < nseg; s0 += 8) {
+      float4 part[8];
+#pragma unroll
+      for (int s = 0; s < 8; ++s)
+        part[s] = (s0 + s < nseg) ? __ldcg(p + (s0 + s) * slot4) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        acc0 += part[s].x;
+        acc1 += part[s].y;
+        acc2 += part[s].z;
+        acc3 += part[s].w;
+      }
+    }
+    if (r.c != nullptr) {
+      const uint2 w = __ldg(reinterpret_cast<const uint2*>(r.c + (long long)row * r.n + col));
       acc0 += __uint_as_float(w.x << 16);
       acc1 += __uint_as_float(w.x & 0xFFFF0000u);
       acc2 += __uint_as_float(w.y << 16);
       acc3 += __uint_as_float(w.y & 0xFFFF0000u);
     }
     __nv_bfloat162 lo = __floats2bfloat162_rn(acc0, acc1), hi = __floats2bfloat162_rn(acc2, acc3);
-    *reinterpret_cast<uint2*>(d + r * n + col) =
+    *reinterpret_cast<uint2*>(r.d + (long long)row * r.n + col) =
         make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
   }
 }

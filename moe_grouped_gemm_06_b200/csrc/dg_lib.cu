@@ -116,95 +116,168 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t
 
 // ------------------------------------------------------------ heuristic
 
-constexpr int kBlockNs[] = {128, 192, 256};  // multiples of 64 (see Cfg in dg_gemm.cuh)
-
 struct Plan {
   int bn = 128;
-  int ctas = 1;  // 2: a cluster of two CTAs computes 256-row tiles
-  int splits = 1;
-  int kb_per_split = 1;
-  long long units = 0;
+  int ctas = 1;           // 2: a cluster of two CTAs computes 256-row tiles (not launched)
+  long long dp_tiles = 0; // tiles computed whole (all tiles when sk_tiles = 0)
+  int sk_tiles = 0;       // stream-K tiles after them (dense only)
+  int max_seg = 0;        // workspace slots per stream-K tile
+  int sk_split = 0;       // > 0: each stream-K tile cut into this many K-slices
+  long long sk_iters = 0;
   int grid = 0;
+  double cost = 0;        // estimated microseconds
+  size_t ws_bytes() const { return (size_t)sk_tiles * max_seg * dg::kBM * bn * sizeof(float); }
 };
 
 long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
 
-// Estimated critical path (per SM) in units of "B rows x K-blocks" streamed
-// through the tensor core: waves x (BN x K-blocks per unit + a per-unit
-// overhead of 4 K-blocks), with a 3% surcharge per extra split-K slice for
-// the partial-sum round trip.  Minimised over the instantiated block sizes;
-// ties keep fewer slices, then the larger block.
+// Per-tile time of each instantiated block width on B200, fitted to measured
+// dense sweeps (M = 4096, K from 512 to 16384; microseconds at the SM clock
+// under load):
+//   tile = max(K-blocks x per_kb + per_tile, epilogue)
+// With two or three accumulator buffers the epilogue of one tile overlaps the
+// main loop of the next, so a tile costs the slower of the two; at 256
+// columns there is one buffer and the epilogue is inside per_tile.  Widths 160
+// and 224 re-base their scale words on the MMA-issuing thread, which costs
+// more than they gain; they are available through dg_set_tile_config but
+// never chosen automatically.
+struct WidthCost {
+  int bn;
+  double per_kb, per_tile, epilogue;
+  bool automatic;
+};
+constexpr WidthCost kWidthCosts[] = {
+    {128, 0.2305, 1.9, 2.94, true}, {160, 0.32, 2.4, 3.6, false}, {192, 0.368, 1.6, 3.97, true},
+    {224, 0.41, 3.0, 4.6, false},   {256, 0.4236, 4.34, 0.0, true},
+};
+
 // Tile-configuration override (dg_set_tile_config; initial values from the
-// environment variables DG_BLOCK_N and DG_CTAS): restricts the heuristic's
-// search to one block width and/or to single CTAs (1) or CTA pairs (2).
+// environment variables DG_BLOCK_N and DG_SCHEDULE): one block width, and/or
+// one schedule: whole tiles (1), tail cut into per-tile K-slices (2) or
+// stream-K tail (3).
 int env_int(const char* name) {
   const char* e = std::getenv(name);
   return e ? std::atoi(e) : 0;
 }
 std::atomic<int> g_force_bn{env_int("DG_BLOCK_N")};
-std::atomic<int> g_force_ctas{env_int("DG_CTAS") == 1 ? 1 : 0};
-
-int forced_ctas() {
-  const int c = g_force_ctas.load();
-  return (c == 1 || c == 2) ? c : 0;
-}
+std::atomic<int> g_force_schedule{(env_int("DG_SCHEDULE") >= 1 && env_int("DG_SCHEDULE") <= 3) ? env_int("DG_SCHEDULE")
+                                                                                             : 0};
 
 int forced_block_n() {
   const int b = g_force_bn.load();
-  for (int bn : kBlockNs)
-    if (bn == b) return b;
+  for (const WidthCost& wc : kWidthCosts)
+    if (wc.bn == b) return b;
   return 0;
 }
 
-// CTA pairs (dense only, allow_pair) are costed per cluster: half the SMs,
-// tiles of 256 rows, no split-K, and 0.85x the per-unit time for staging half
-// of B per SM.
-Plan plan_gemm(long long m_blocks, int n, int k, int sms, bool allow_split, bool allow_pair = false) {
+double tile_time(const WidthCost& wc, int kb) { return std::max(kb * wc.per_kb + wc.per_tile, wc.epilogue); }
+
+// Stream-K split of the last sk_tiles tiles over G CTAs: exact slots per
+// tile (CTAs whose shares meet the tile), 0 when some share would be empty.
+int sk_max_segments(int sk_tiles, int kb, int G) {
+  const long long iters = (long long)sk_tiles * kb;
+  if (sk_tiles <= 0 || iters < G) return 0;
+  int mx = 0;
+  for (int j = 0; j < sk_tiles; ++j) {
+    const long long x0 = (long long)j * kb;
+    mx = std::max(mx, dg::sk_cta_of(x0 + kb - 1, G, iters) - dg::sk_cta_of(x0, G, iters) + 1);
+  }
+  return mx;
+}
+
+// Chooses the block width and the schedule minimising the estimated time
+// (microseconds; constants measured on B200):
+//   whole tiles:  ceil(tiles / SMs) x tile time
+//   tail split:   q full waves of whole tiles (q = the number of full waves,
+//                 or one less), then the remaining r tiles shared over the
+//                 SMs, either each cut into s = SMs / r equal K-slices (one
+//                 piece per CTA), or as stream-K (even shares of all their
+//                 K-iterations, pieces crossing tiles; at one accumulator
+//                 buffer a CTA's pieces run one after the other); plus the
+//                 fix-up kernel (7.5 us for slices, 9.5 us for stream-K, of
+//                 launch, partial writes and reads, + the partial bytes at
+//                 ~5 TB/s) and, after full waves, the HBM reads of the shared
+//                 tiles' A and B rows (pieces of different K ranges do not
+//                 reuse each other's tiles in L2).
+// Every plan is at least the time to move the unique bytes of A, B, C and D
+// through HBM (~5.5 TB/s), and at small M (at most two 128-row blocks, where
+// B streams from HBM in 128-byte rows) at least the time to stream B at
+// ~4 TB/s and the time one SM needs to stream its share (~63 GB/s per SM);
+// among plans at the floor the one with the least estimated SM time wins.  Sharing is offered for the dense layout only
+// (allow_sk) and only within ws_cap bytes of workspace (0: no cap).  Ties
+// keep whole tiles.
+Plan plan_gemm(long long m_blocks, int n, int k, int sms, bool allow_sk, size_t ws_cap = 0) {
   Plan best;
-  double best_cost = 1e300;
+  best.cost = 1e300;
   const int kb = k / 128;
-  if (allow_pair && m_blocks >= 2 && forced_ctas() != 1) {
-    for (int bn : kBlockNs) {
-      if (bn < 192 || (forced_block_n() && bn != forced_block_n())) continue;
-      const long long units = ((m_blocks + 1) / 2) * ceil_div(n, bn);
-      const double waves = (double)ceil_div(units, sms / 2);
-      const double cost = waves * (double)bn * (kb + 4) * 0.85;
-      if (cost < best_cost * (1 - 1e-9)) {
-        best_cost = cost;
-        best.bn = bn;
-        best.ctas = 2;
-        best.splits = 1;
-        best.kb_per_split = kb;
-        best.units = units;
-      }
-    }
-  }
-  for (int bn : kBlockNs) {
-    if (forced_ctas() == 2 && best.ctas == 2) break;
-    if (forced_block_n() && bn != forced_block_n()) continue;
+  const int sched = g_force_schedule.load();
+  const double rows = (double)m_blocks * dg::kBM;
+  const bool streams_b = m_blocks <= 2;
+  const double hbm_floor = std::max((rows * k + (double)n * k + 4.0 * rows * n) / 5.5e6,
+                                    streams_b ? (double)n * k / 4.0e6 : 0.0);
+  for (const WidthCost& wc : kWidthCosts) {
+    const int bn = wc.bn;
+    if (forced_block_n() ? bn != forced_block_n() : !wc.automatic) continue;
     const long long tiles = m_blocks * ceil_div(n, bn);
-    const int max_s = allow_split ? std::max(1, std::min(dg::kMaxSplits, kb / 2)) : 1;
-    for (int s = 1; s <= max_s; ++s) {
-      const int kbps = (int)ceil_div(kb, s);
-      const int s_eff = (int)ceil_div(kb, kbps);
-      if (s_eff != s) continue;
-      const long long units = tiles * s;
-      const double waves = (double)ceil_div(units, sms);
-      const double cost = waves * (double)bn * (kbps + 4) * (1.0 + 0.03 * (s - 1));
-      if (cost < best_cost * (1 - 1e-9)) {
-        best_cost = cost;
-        best.bn = bn;
-        best.ctas = 1;
-        best.splits = s;
-        best.kb_per_split = kbps;
-        best.units = units;
+    auto consider = [&](const Plan& p) {
+      if (p.cost < best.cost * (1 - 1e-9)) best = p;
+    };
+    // time for one CTA to stream kbs K-blocks of B from HBM (small M only)
+    auto stream_b = [&](long long kbs) { return streams_b ? (double)kbs * bn * 128.0 / 6.3e4 : 0.0; };
+    Plan dp;
+    dp.bn = bn;
+    dp.dp_tiles = tiles;
+    dp.grid = (int)std::max<long long>(1, std::min<long long>(tiles, sms));
+    const long long waves = ceil_div(tiles, sms);
+    // at the floor, the plan with less work on the SMs wins (5% of it counts)
+    auto floored = [&](double t) { return std::max(t, hbm_floor) + 0.05 * t; };
+    dp.cost = floored(std::max((double)waves * tile_time(wc, kb), waves * stream_b(kb))) * (sched >= 2 ? 1e6 : 1.0);
+    consider(dp);
+    if (!allow_sk || sched == 1) continue;
+    const long long full_waves = tiles / sms;
+    for (long long q = full_waves; q >= std::max(0LL, full_waves - 1); --q) {
+      const long long sk = tiles - q * sms;
+      if (sk <= 0 || sk > 4 * (long long)sms) continue;
+      const double shared_reads = q > 0 ? (double)sk * (dg::kBM + bn) * k / 6e6 : 0.0;
+      Plan p;
+      p.bn = bn;
+      p.dp_tiles = q * sms;
+      p.sk_tiles = (int)sk;
+      // (a) each remaining tile cut into s K-slices
+      const long long s_split = std::min<long long>(sms / sk, kb);
+      if (s_split >= 2 && sched != 3) {
+        Plan ps = p;
+        ps.sk_split = (int)s_split;
+        ps.max_seg = (int)s_split;
+        ps.grid = (int)(q > 0 ? sms : sk * s_split);
+        const long long kbs = ceil_div(kb, s_split);
+        const double piece = std::max(tile_time(wc, (int)kbs), stream_b(kbs)) + shared_reads;
+        const double fixup = 7.5 + (double)sk * s_split * dg::kBM * bn * 4.0 / 5e6;
+        ps.cost = floored((double)q * tile_time(wc, kb) + piece + fixup);
+        if (ws_cap == 0 || ps.ws_bytes() <= ws_cap) consider(ps);
       }
+      // (b) stream-K over all SMs
+      if (sched == 2) continue;
+      const long long iters = sk * kb;
+      const int G = (int)std::min<long long>(sms, iters);
+      if (G < 2 || (q > 0 && G != sms)) continue;
+      const int max_seg = sk_max_segments((int)sk, kb, G);
+      if (max_seg == 0 || max_seg > 64) continue;
+      p.max_seg = max_seg;
+      p.sk_iters = iters;
+      p.grid = G;
+      if (ws_cap != 0 && p.ws_bytes() > ws_cap) continue;
+      const long long share = ceil_div(iters, G);
+      const long long pieces = std::min<long long>(share, ceil_div(share, kb) + 1);
+      const double compute = (wc.epilogue > 0.0)
+                                 ? std::max(share * wc.per_kb + pieces * wc.per_tile, pieces * wc.epilogue)
+                                 : share * wc.per_kb + pieces * wc.per_tile;
+      const double piece = std::max(compute, stream_b(share)) + shared_reads;
+      const double fixup = 9.5 + (double)(sk + G) * dg::kBM * bn * 4.0 / 5e6;
+      p.cost = floored((double)q * tile_time(wc, kb) + piece + fixup);
+      consider(p);
     }
   }
-  if (best.ctas == 2)
-    best.grid = 2 * (int)std::max<long long>(1, std::min<long long>(best.units, sms / 2));
-  else
-    best.grid = (int)std::max<long long>(1, std::min<long long>(best.units, sms));
   return best;
 }
 
@@ -217,7 +290,7 @@ struct Workspace {
 std::mutex g_ws_mutex;
 std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
 
-// Split-K FP32 partials of this (device, stream), allocated stream-ordered on
+// Stream-K partial sums of this (device, stream), allocated stream-ordered on
 // first use and grown on demand.
 float* workspace(size_t bytes, cudaStream_t s) {
   int dev = 0;
@@ -266,7 +339,9 @@ dg_status dispatch(int bn, int ctas, const CUtensorMap& ta, const CUtensorMap& t
   if (ctas != 1) return DG_ERR_UNSUPPORTED;
   switch (bn) {
     case 128: return launch_gemm<128, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
+    case 160: return launch_gemm<160, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
     case 192: return launch_gemm<192, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
+    case 224: return launch_gemm<224, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
     case 256: return launch_gemm<256, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
     default: return DG_ERR_UNSUPPORTED;
   }
@@ -287,9 +362,10 @@ struct Problem {
   int expected_m;  // masked hint
 };
 
-// fixed_ws / fixed_ws_bytes: when given, split-K partials go to this caller-
-// provided device buffer instead of the per-stream workspace, and a plan that
-// needs more than fixed_ws_bytes is rejected with DG_ERR_SCRATCH_LIMIT.
+// fixed_ws / fixed_ws_bytes: when given, stream-K partials go to this
+// caller-provided device buffer instead of the per-stream workspace, and the
+// planner only considers plans that fit in fixed_ws_bytes (whole tiles
+// always do).
 template <bool FP4, int LAYOUT>
 dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, size_t fixed_ws_bytes = 0) {
   const int sms = num_sms();
@@ -301,8 +377,7 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
     plan = plan_gemm((long long)p.groups * ceil_div(em, dg::kBM), p.n, p.k, sms, false);
     plan.grid = (int)std::min<long long>((long long)p.groups * m_blocks * ceil_div(p.n, plan.bn), sms);
   } else {
-    const bool allow_split = (LAYOUT == dg::kDense) && p.rows <= 1024;
-    plan = plan_gemm(m_blocks, p.n, p.k, sms, allow_split, /*allow_pair=*/false);
+    plan = plan_gemm(m_blocks, p.n, p.k, sms, LAYOUT == dg::kDense, fixed_ws != nullptr ? fixed_ws_bytes : 0);
   }
 
   dg::GemmArgs args{};
@@ -320,8 +395,11 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
   args.num_m_blocks = (int)(plan.ctas == 2 ? ceil_div(p.rows, 2 * dg::kBM) : m_blocks);
   args.num_n_blocks = (int)ceil_div(p.n, plan.bn);
   args.kb_total = p.k / 128;
-  args.splits = plan.splits;
-  args.kb_per_split = plan.kb_per_split;
+  args.dp_tiles = (int)plan.dp_tiles;
+  args.sk_tiles = plan.sk_tiles;
+  args.max_seg = plan.max_seg;
+  args.sk_split = plan.sk_split;
+  args.sk_iters = plan.sk_iters;
   args.sfa_chunks = (int)ceil_div(p.rows, 128);
   args.sfb_chunks = (int)ceil_div(p.n, 128);
   args.sfa_q = (int)ceil_div(p.k / 128, 4);
@@ -333,8 +411,8 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
   args.sfa_words = args.sfa_group_words * ((LAYOUT == dg::kMasked) ? p.groups : 1);
   args.sfb_words = args.sfb_group_words * ((LAYOUT == dg::kDense) ? 1 : p.groups);
 
-  if (plan.splits > 1) {
-    const size_t need = (size_t)plan.splits * p.rows * p.n * sizeof(float);
+  if (plan.sk_tiles > 0) {
+    const size_t need = plan.ws_bytes();
     if (fixed_ws != nullptr) {
       if (need > fixed_ws_bytes) return DG_ERR_SCRATCH_LIMIT;
       args.ws = fixed_ws;
@@ -373,18 +451,35 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
 
   if (log_enabled())
     std::fprintf(stderr,
-                 "[dg] layout=%d fp4=%d rows=%d n=%d k=%d groups=%d -> block_n=%d ctas=%d splits=%d units=%lld grid=%d\n",
-                 LAYOUT, (int)FP4, p.rows, p.n, p.k, p.groups, plan.bn, plan.ctas, plan.splits, plan.units, plan.grid);
+                 "[dg] layout=%d fp4=%d rows=%d n=%d k=%d groups=%d -> block_n=%d dp_tiles=%lld sk_tiles=%d "
+                 "split=%d max_seg=%d grid=%d est=%.1fus\n",
+                 LAYOUT, (int)FP4, p.rows, p.n, p.k, p.groups, plan.bn, plan.dp_tiles, plan.sk_tiles, plan.sk_split,
+                 plan.max_seg, plan.grid, plan.cost);
 
   dg_status st = dispatch<FP4, LAYOUT>(plan.bn, plan.ctas, ta, tb, td, tsfa, tsfb, args, plan.grid, s);
-  if (st != DG_OK || plan.splits == 1) return st;
+  if (st != DG_OK || plan.sk_tiles == 0) return st;
 
-  const long long units = (long long)p.rows * (p.n / 4);
+  dg::SkReduceArgs r{};
+  r.ws = args.ws;
+  r.c = args.c;
+  r.d = args.d;
+  r.rows = p.rows;
+  r.n = p.n;
+  r.bn = plan.bn;
+  r.kb_total = args.kb_total;
+  r.dp_tiles = args.dp_tiles;
+  r.sk_tiles = plan.sk_tiles;
+  r.max_seg = plan.max_seg;
+  r.sk_split = plan.sk_split;
+  r.ctas = plan.grid;
+  r.sk_iters = plan.sk_iters;
+  r.raster = args.raster;
+  r.num_m_blocks = args.num_m_blocks;
+  r.num_n_blocks = args.num_n_blocks;
+  const long long items = (long long)plan.sk_tiles * dg::kBM * (plan.bn / 4);
   const int threads = 256;
-  const int blocks = (int)std::min<long long>(ceil_div(units, threads), (long long)sms * 8);
-  if (launch(dg::splitk_reduce_kernel, dim3(blocks), dim3(threads), 0, s, 1, (const float*)args.ws, args.c, args.d,
-             p.rows, p.n, plan.splits) != cudaSuccess)
-    return DG_ERR_CUDA;
+  const int blocks = (int)std::min<long long>(ceil_div(items, threads), (long long)sms * 8);
+  if (launch(dg::sk_reduce_kernel, dim3(blocks), dim3(threads), 0, s, 1, r) != cudaSuccess) return DG_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return DG_OK;
 }
@@ -577,16 +672,15 @@ dg_status dg_set_pdl(int enable) {
 
 int dg_get_pdl(void) { return g_pdl.load(); }
 
-dg_status dg_set_tile_config(int block_n, int ctas) {
+dg_status dg_set_tile_config(int block_n, int schedule) {
   if (block_n != 0) {
     bool known = false;
-    for (int bn : kBlockNs) known = known || (bn == block_n);
+    for (const WidthCost& wc : kWidthCosts) known = known || (wc.bn == block_n);
     if (!known) return DG_ERR_INVALID_ARG;
   }
-  if (ctas != 0 && ctas != 1 && ctas != 2) return DG_ERR_INVALID_ARG;
-  if (ctas == 2) return DG_ERR_UNSUPPORTED;  // CTA pairs are not launched (see dispatch)
+  if (schedule < 0 || schedule > 3) return DG_ERR_INVALID_ARG;
   g_force_bn.store(block_n);
-  g_force_ctas.store(ctas);
+  g_force_schedule.store(schedule);
   return DG_OK;
 }
 
@@ -623,16 +717,20 @@ const char* dg_status_string(int status) {
 
 uint64_t dg_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
-dg_status dg_query_dense_config(int m, int n, int k, int* block_n, int* splits, int* units, int* grid, int* ctas) {
-  if (m <= 0 || n <= 0 || k <= 0 || k % 128 != 0) return DG_ERR_INVALID_ARG;
+dg_status dg_query_dense_config(int m, int n, int k, int64_t workspace_cap, int* block_n, int* dp_tiles,
+                                int* sk_tiles, int* sk_split, int* max_segments, int* grid,
+                                int64_t* workspace_bytes) {
+  if (m <= 0 || n <= 0 || k <= 0 || k % 128 != 0 || workspace_cap < 0) return DG_ERR_INVALID_ARG;
   const int sms = num_sms();
   if (sms <= 0) return DG_ERR_CUDA;
-  Plan p = plan_gemm(ceil_div(m, dg::kBM), n, k, sms, m <= 1024, /*allow_pair=*/false);
+  Plan p = plan_gemm(ceil_div(m, dg::kBM), n, k, sms, true, (size_t)workspace_cap);
   if (block_n) *block_n = p.bn;
-  if (splits) *splits = p.splits;
-  if (units) *units = (int)p.units;
+  if (dp_tiles) *dp_tiles = (int)p.dp_tiles;
+  if (sk_tiles) *sk_tiles = p.sk_tiles;
+  if (sk_split) *sk_split = p.sk_split;
+  if (max_segments) *max_segments = p.max_seg;
   if (grid) *grid = p.grid;
-  if (ctas) *ctas = p.ctas;
+  if (workspace_bytes) *workspace_bytes = (int64_t)p.ws_bytes();
   return DG_OK;
 }
 

@@ -107,44 +107,115 @@ def test_tile_count_matches_pages_worked_example(dg):
         assert dg.dg_num_tiles(m, n, bm, bn) == tiles
 
 
-def test_heuristic_in_the_pages_example(dg):
+def test_stream_k_keeps_more_sms_busy_than_the_pages_fix(dg):
     # The page's unaligned BLOCK_N=112 keeps 128 of 132 SMs busy for M=256,
     # N=7168 where 128x128 tiles keep 112.  Block widths here are multiples of
-    # 64 (the scale-factor operand's TMEM address must be even), so the
-    # heuristic has {128, 192, 256} x split-K; it must never do worse than the
-    # page's aligned baseline and must fill whole waves.
-    (m, n, _, _, base, sms), _ = _golden_rows()
+    # 32 (one TMEM column of scale factors), so 112 is not available; the
+    # stream-K schedule instead shares the K-iterations of the 112 tiles over
+    # all 132 SMs.  The heuristic keeps at least the page's baseline busy.
+    (m, n, _, _, base, sms), (_, _, _, _, best, _) = _golden_rows()
     dg.dg_set_num_sms(sms)
     try:
-        cfg = dg.dg_query_dense_config(m, n, 7168)
+        auto = dg.dg_query_dense_config(m, n, 7168)
+        dg.dg_set_tile_config(0, 3)
+        sk = dg.dg_query_dense_config(m, n, 7168)
     finally:
+        dg.dg_set_tile_config(0, 0)
         dg.dg_set_num_sms(0)
-    assert cfg["block_n"] % 64 == 0
-    assert cfg["grid"] >= base
-    assert cfg["units"] <= sms or cfg["units"] % cfg["grid"] == 0
+    assert auto["block_n"] % 32 == 0 and auto["grid"] >= base
+    assert sk["sk_tiles"] > 0 and sk["sk_split"] == 0 and sk["grid"] == sms > best > base
 
 
-def test_heuristic_large_m_has_no_split(dg):
+def test_heuristic_shares_k_only_where_waves_are_short(dg):
     dg.dg_set_num_sms(148)
     try:
-        cfg = dg.dg_query_dense_config(4096, 7168, 16384)
-        small = dg.dg_query_dense_config(64, 2112, 7168)
+        big = dg.dg_query_dense_config(4096, 7168, 16384)
+        small = dg.dg_query_dense_config(64, 7168, 16384)
     finally:
         dg.dg_set_num_sms(0)
-    assert cfg["splits"] == 1 and cfg["grid"] == 148
-    assert small["splits"] > 1 and small["units"] <= 148
+    # large M: whole tiles for all full waves, the 8 tiles of the partial
+    # wave cut into K-slices over the SMs
+    assert big["dp_tiles"] == 6 * 148 and big["sk_tiles"] == 8 and big["sk_split"] == 148 // 8
+    # small M, long K: 56 tiles would leave 92 SMs idle; each is cut in two
+    assert small["dp_tiles"] == 0 and small["sk_tiles"] == 56 and small["sk_split"] == 2
+    assert small["grid"] == 112
 
 
-def test_tile_config_override_and_pairs_refused(dg):
+def _brute_force_segments(sk_tiles, kb, grid):
+    """Slots per stream-K tile by walking every CTA's share of the
+    sk_tiles x kb iterations (CTA c: [c*I//G, (c+1)*I//G))."""
+    iters = sk_tiles * kb
+    owners = [set() for _ in range(sk_tiles)]
+    covered = 0
+    for c in range(grid):
+        lo, hi = c * iters // grid, (c + 1) * iters // grid
+        assert hi > lo                         # no CTA without work
+        covered += hi - lo
+        for x in range(lo, hi):
+            owners[x // kb].add(c)
+    assert covered == iters
+    for o in owners:                            # a tile's CTAs are consecutive
+        assert max(o) - min(o) + 1 == len(o)
+    return max(len(o) for o in owners)
+
+
+@pytest.mark.parametrize("schedule", [2, 3])
+@pytest.mark.parametrize("sms", [148, 132, 7])
+@pytest.mark.parametrize("m,n,k", [(64, 2112, 7168), (4096, 7168, 16384), (300, 1000, 1024), (1100, 520, 512),
+                                   (4096, 4096, 128), (128, 256, 384)])
+def test_shared_tail_plan_partition(dg, schedule, sms, m, n, k):
+    dg.dg_set_num_sms(sms)
+    dg.dg_set_tile_config(0, schedule)
+    try:
+        cfg = dg.dg_query_dense_config(m, n, k)
+    finally:
+        dg.dg_set_tile_config(0, 0)
+        dg.dg_set_num_sms(0)
+    tiles = -(-m // 128) * -(-n // cfg["block_n"])
+    kb = k // 128
+    assert cfg["dp_tiles"] + cfg["sk_tiles"] == tiles
+    if cfg["sk_tiles"] == 0:                    # no such split exists
+        assert cfg["grid"] == min(tiles, sms) and cfg["workspace_bytes"] == 0
+        return
+    assert cfg["grid"] <= sms and cfg["dp_tiles"] % cfg["grid"] == 0
+    assert cfg["dp_tiles"] == 0 or cfg["grid"] == sms
+    if schedule == 2:
+        # one piece per CTA: sk_tiles x s CTAs, each slice at least one K-block
+        s = cfg["sk_split"]
+        assert 2 <= s <= kb and cfg["sk_tiles"] * s <= cfg["grid"] and cfg["max_segments"] == s
+    else:
+        assert cfg["sk_split"] == 0
+        assert cfg["max_segments"] == _brute_force_segments(cfg["sk_tiles"], kb, cfg["grid"])
+    assert cfg["workspace_bytes"] == cfg["sk_tiles"] * cfg["max_segments"] * 128 * cfg["block_n"] * 4
+
+
+def test_workspace_cap_limits_the_plan(dg):
+    dg.dg_set_num_sms(148)
+    try:
+        free = dg.dg_query_dense_config(64, 7168, 16384)
+        capped = dg.dg_query_dense_config(64, 7168, 16384, workspace_cap=free["workspace_bytes"] - 1)
+        none = dg.dg_query_dense_config(64, 7168, 16384, workspace_cap=1)
+    finally:
+        dg.dg_set_num_sms(0)
+    assert free["workspace_bytes"] > 0
+    assert 0 < capped["workspace_bytes"] < free["workspace_bytes"] or capped["sk_tiles"] == 0
+    assert none["sk_tiles"] == 0 and none["workspace_bytes"] == 0
+    assert dg.lib().dg_query_dense_config(64, 2112, 7168, -1, None, None, None, None, None, None, None) == -1
+
+
+def test_tile_config_override(dg):
     assert dg.lib().dg_set_tile_config(96, 0) == -1          # not an instantiated width
-    assert dg.lib().dg_set_tile_config(0, 2) == -2           # CTA pairs are not launched
+    assert dg.lib().dg_set_tile_config(0, 4) == -1           # no such schedule
     dg.dg_set_num_sms(148)
     try:
         dg.dg_set_tile_config(256, 1)
-        assert dg.dg_query_dense_config(4096, 7168, 16384)["block_n"] == 256
+        cfg = dg.dg_query_dense_config(4096, 7168, 16384)
+        assert cfg["block_n"] == 256 and cfg["sk_tiles"] == 0
+        dg.dg_set_tile_config(224, 0)
+        assert dg.dg_query_dense_config(4096, 7168, 16384)["block_n"] == 224
         dg.dg_set_tile_config(0, 0)
         for shape in [(4096, 7168, 16384), (4096, 2112, 7168), (256, 7168, 7168)]:
-            assert dg.dg_query_dense_config(*shape)["ctas"] == 1
+            assert dg.dg_query_dense_config(*shape)["block_n"] in (128, 192, 256)
     finally:
         dg.dg_set_tile_config(0, 0)
         dg.dg_set_num_sms(0)

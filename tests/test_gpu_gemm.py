@@ -83,7 +83,7 @@ def test_pack_sf_bit_exact(dg, rows, ng, row_div):
     (128, 512, 1024, False),    # the small worked configuration (C = 0)
     (200, 328, 384, True),      # ragged M and N tails, K of three blocks
     (1100, 520, 512, True),     # several m-blocks, no split-K, ragged tails
-    (64, 2112, 7168, True),     # split-K path
+    (64, 2112, 7168, True),     # stream-K over all SMs (17 tiles)
     (3, 64, 256, True),         # tiny M
 ])
 def test_dense_matches_oracle(dg, M, N, K, with_c):
@@ -91,6 +91,91 @@ def test_dense_matches_oracle(dg, M, N, K, with_c):
     d = p.run(dg)
     stats = check_close(d, p.ref(), f"dense {M}x{N}x{K}")
     assert stats["n"] == M * N
+
+
+@pytest.mark.parametrize("schedule", [2, 3])
+@pytest.mark.parametrize("sms", [0, 7])
+@pytest.mark.parametrize("bn", [128, 192, 256])
+@pytest.mark.parametrize("M,N,K,with_c,fp4", [
+    (1100, 520, 512, True, False),     # ragged M and N tails, 4 K-blocks
+    (300, 1000, 1536, True, False),    # pieces that start and end inside tiles
+    (128, 512, 128, False, False),     # one K-block: every piece is a whole tile
+    (200, 904, 1024, True, True),      # FP8 x FP4
+])
+def test_dense_shared_tail_matches_oracle(dg, schedule, sms, bn, M, N, K, with_c, fp4):
+    # Forced per-tile K-slices (2) or stream-K (3).  With 7 "SMs" the small
+    # problems run waves of whole tiles before the shared K-blocks of the last
+    # tiles, as large problems do on 148 SMs.
+    dg.dg_set_num_sms(sms)
+    dg.dg_set_tile_config(bn, schedule)
+    try:
+        cfg = dg.dg_query_dense_config(M, N, K)
+        assert cfg["block_n"] == bn
+        if cfg["sk_tiles"] == 0:
+            pytest.skip(f"no split of this kind: {cfg}")
+        assert (cfg["sk_split"] > 0) == (schedule == 2)
+        p = Dense(2400 + M + bn + sms, M, N, K, with_c=with_c, fp4=fp4).upload()
+        check_close(p.run(dg), p.ref(), f"schedule {schedule} bn={bn} sms={sms} {M}x{N}x{K} {cfg}")
+        assert dg.dg_get_last_error() == 0
+    finally:
+        dg.dg_set_tile_config(0, 0)
+        dg.dg_set_num_sms(0)
+
+
+def test_dense_shared_tail_is_deterministic_and_agrees_with_whole_tiles(dg):
+    M, N, K = 1100, 2112, 2048
+    p = Dense(2500, M, N, K, with_c=True).upload()
+    outs = {}
+    dg.dg_set_num_sms(30)          # 153 tiles: 5 waves + 3 shared tiles
+    try:
+        for sched in (1, 2, 2, 3, 3):
+            dg.dg_set_tile_config(128, sched)
+            assert (dg.dg_query_dense_config(M, N, K)["sk_tiles"] > 0) == (sched > 1)
+            outs.setdefault(sched, []).append(p.run(dg))
+    finally:
+        dg.dg_set_tile_config(0, 0)
+        dg.dg_set_num_sms(0)
+    for sched in (2, 3):
+        assert np.array_equal(outs[sched][0], outs[sched][1])   # slots summed in K order
+        check_close(outs[sched][0], outs[1][0], f"schedule {sched} vs whole tiles")
+        check_close(outs[sched][0], p.ref(), f"schedule {sched} vs oracle")
+
+
+@pytest.mark.parametrize("bn", [160, 224])
+@pytest.mark.parametrize("M,N,K,fp4", [(300, 1000, 1024, False), (1100, 2112, 512, False), (200, 904, 512, True)])
+def test_dense_rebased_scale_widths(dg, bn, M, N, K, fp4):
+    # widths that start tiles 32 or 96 rows into a 128-row scale chunk: the B
+    # scale words are re-based in shared memory before the TMEM copy
+    dg.dg_set_tile_config(bn, 1)
+    try:
+        assert dg.dg_query_dense_config(M, N, K)["block_n"] == bn
+        p = Dense(2600 + M + bn, M, N, K, with_c=True, fp4=fp4).upload()
+        check_close(p.run(dg), p.ref(), f"bn={bn} {M}x{N}x{K} fp4={fp4}")
+    finally:
+        dg.dg_set_tile_config(0, 0)
+
+
+@pytest.mark.parametrize("bn", [160, 224])
+def test_grouped_rebased_scale_widths(dg, bn):
+    dg.dg_set_tile_config(bn, 1)
+    try:
+        N, K = 1000, 512
+        cs = _contiguous_case(2700 + bn, 3, 60, 200, N, K)
+        d = _run_contiguous(dg, cs, N)
+        ref = oracle.gemm_contiguous(cs["qa"], cs["ea"], cs["qb"], cs["eb"], cs["mi"], c=cs["c"])
+        valid = cs["mi"] >= 0
+        check_close(d[valid], ref[valid], f"contiguous bn={bn}")
+        G, max_m = 3, 256
+        mm = np.array([5, 256, 130], np.int32)
+        qa, ea, sfa, qb, eb, sfb = _masked_case(2800 + bn, G, max_m, N, K, mm)
+        dm = _run_masked(dg, G, max_m, N, qa, sfa, qb, sfb, mm)
+        refm = oracle.gemm_masked(qa, ea, qb, eb, mm)
+        ddm = bf16_dev_to_f64(dm)
+        for g in range(G):
+            check_close(ddm[g, :mm[g]], refm[g, :mm[g]], f"masked bn={bn} g={g}")
+            assert np.all(host(dm).view(np.uint16)[g, mm[g]:] == SENTINEL)
+    finally:
+        dg.dg_set_tile_config(0, 0)
 
 
 def test_dense_long_k_accumulation(dg):
