@@ -57,6 +57,9 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--shape", default=None, help="run one M,N,K shape instead of the sweep")
+    ap.add_argument("--workload", default="dense", choices=["dense", "contiguous", "masked", "fp4"],
+                    help="dense: the DeepSeek-V3 dense sweep (default); contiguous / masked / fp4: the "
+                         "M-grouped prefill, masked decode and FP8 x FP4 cases, one JSON line each")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -192,6 +195,182 @@ def make_inputs(dg, torch, m, n, k, gen):
     return {"a": a, "sfa": sfa, "b": b, "sfb": sfb, "c": c, "d": d}
 
 
+# ---------------------------------------------------------------- grouped / FP4 cases
+
+GROUPED_NK = [(4096, 7168), (7168, 2048)]
+CONTIG_GROUPS, CONTIG_ROWS = 8, (6000, 10000)
+MASKED_GROUPS, MASKED_MAX_M, MASKED_EXPECTED = 32, 256, (16, 64, 128)
+
+
+def quant_a_dev(dg, torch, rows, k, gen, groups=1):
+    """e4m3 A [groups*rows, k] with 1x128 scales, packed per group."""
+    x = torch.randn((groups * rows, k), generator=gen, device="cuda", dtype=torch.float32)
+    a = torch.empty((groups * rows, k), dtype=torch.uint8, device="cuda")
+    ea = torch.empty((groups * rows, k // 128), dtype=torch.uint8, device="cuda")
+    dg.dg_quantize_fp8(x, a, ea, 1)
+    del x
+    words = dg.dg_packed_sf_words(rows, k // 128)
+    sfa = torch.empty(groups * words, dtype=torch.int32, device="cuda")
+    for g in range(groups):
+        dg.dg_pack_sf(ea[g * rows:(g + 1) * rows], rows, sfa[g * words:(g + 1) * words], row_div=1)
+    return a, sfa
+
+
+def quant_b_dev(dg, torch, groups, n, k, gen, fp4=False):
+    """B [groups, n, k] e4m3 with 128x128 scales, or e2m1 [groups, n, k/2]
+    with 1x32 scales; scale words packed per group."""
+    b = torch.empty((groups, n, k // 2 if fp4 else k), dtype=torch.uint8, device="cuda")
+    cols = k // 32 if fp4 else k // 128
+    words = dg.dg_packed_sf_words(n, cols)
+    sfb = torch.empty(groups * words, dtype=torch.int32, device="cuda")
+    for g in range(groups):
+        x = torch.randn((n, k), generator=gen, device="cuda", dtype=torch.float32)
+        if fp4:
+            e = torch.empty((n, cols), dtype=torch.uint8, device="cuda")
+            dg.dg_quantize_fp4(x, b[g], e)
+            dg.dg_pack_sf(e, n, sfb[g * words:(g + 1) * words], row_div=1)
+        else:
+            e = torch.empty(((n + 127) // 128, cols), dtype=torch.uint8, device="cuda")
+            dg.dg_quantize_fp8(x, b[g], e, 128)
+            dg.dg_pack_sf(e, n, sfb[g * words:(g + 1) * words], row_div=128)
+        del x, e
+    return b, sfb
+
+
+def grouped_cases(dg, torch, workload, gen, seed):
+    """[(name, call, flops, algorithmic bytes)] for the grouped / FP4 configs:
+    contiguous (MoE prefill, 8 groups of U[6000,10000] rows padded to 128),
+    masked (MoE decode, 32 groups, max_m 256, masked_m ~ U[0, 2 expected_m]),
+    fp4 (dense M=4096 and contiguous with e2m1 weights)."""
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    cases = []
+
+    def contiguous(n, k, fp4):
+        rows = rng.integers(CONTIG_ROWS[0], CONTIG_ROWS[1] + 1, CONTIG_GROUPS)
+        mi = np.concatenate([np.concatenate([np.full(r, g, np.int32), np.full(-r % 128, -1, np.int32)])
+                             for g, r in enumerate(rows)])
+        m_total, valid = mi.size, int(rows.sum())
+        a, sfa = quant_a_dev(dg, torch, m_total, k, gen)
+        b, sfb = quant_b_dev(dg, torch, CONTIG_GROUPS, n, k, gen, fp4)
+        d = torch.empty((m_total, n), dtype=torch.bfloat16, device="cuda")
+        t_mi = torch.from_numpy(mi).cuda()
+        fn = dg.dg_m_grouped_fp8_fp4_gemm_nt_contiguous if fp4 else dg.dg_m_grouped_fp8_gemm_nt_contiguous
+        bb = CONTIG_GROUPS * n * k // (2 if fp4 else 1)
+        by = valid * k + bb + 2 * valid * n + (sfa.numel() + sfb.numel()) * 4 + 4 * m_total
+        name = f"contiguous{'-fp4' if fp4 else ''} G={CONTIG_GROUPS} M={m_total} ({valid} valid) N={n} K={k}"
+        cases.append((name, lambda: fn(a, sfa, b, sfb, None, d, t_mi), 2.0 * valid * n * k, by))
+
+    if workload == "contiguous":
+        for (n, k) in GROUPED_NK:
+            contiguous(n, k, False)
+    elif workload == "masked":
+        G, max_m = MASKED_GROUPS, MASKED_MAX_M
+        for (n, k) in GROUPED_NK:
+            b, sfb = quant_b_dev(dg, torch, G, n, k, gen)
+            for em in MASKED_EXPECTED:
+                mm = np.minimum(rng.integers(0, 2 * em + 1, G), max_m).astype(np.int32)
+                a, sfa = quant_a_dev(dg, torch, max_m, k, gen, groups=G)
+                a = a.view(G, max_m, k)
+                d = torch.empty((G, max_m, n), dtype=torch.bfloat16, device="cuda")
+                t_mm = torch.from_numpy(mm).cuda()
+                valid = int(mm.sum())
+                by = valid * k + G * n * k + 2 * valid * n + (valid * (k // 128)) + sfb.numel() * 4
+                name = f"masked G={G} max_m={max_m} expected_m={em} ({valid} valid rows) N={n} K={k}"
+                cases.append((name, (lambda a=a, sfa=sfa, b=b, sfb=sfb, d=d, t_mm=t_mm, em=em:
+                                     dg.dg_m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, t_mm, expected_m=em)),
+                              2.0 * valid * n * k, by))
+    elif workload == "fp4":
+        for (n, k) in GROUPED_NK:
+            m = 4096
+            a, sfa = quant_a_dev(dg, torch, m, k, gen)
+            b, sfb = quant_b_dev(dg, torch, 1, n, k, gen, fp4=True)
+            b = b[0]
+            d = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+            by = m * k + n * k // 2 + 2 * m * n + (sfa.numel() + sfb.numel()) * 4
+            cases.append((f"dense-fp4 M={m} N={n} K={k}",
+                          (lambda a=a, sfa=sfa, b=b, sfb=sfb, d=d: dg.dg_fp8_fp4_gemm_nt(a, sfa, b, sfb, None, d)),
+                          2.0 * m * n * k, by))
+        for (n, k) in GROUPED_NK:
+            contiguous(n, k, True)
+    return cases
+
+
+def run_grouped(args, dg, torch, rank, world, use_dist, local_rank):
+    """--workload contiguous | masked | fp4: each case timed alone (L2
+    flushed before every call), one JSON line with per-case TFLOPS, GB/s
+    and roofline fraction."""
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(4321 + rank)
+    cases = grouped_cases(dg, torch, args.workload, gen, 99 + rank)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush_rd = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(events):
+        torch.cuda._sleep(HOLD_CYCLES)
+        for i, (_, call, _, _) in enumerate(cases):
+            flush.zero_()
+            flush_rd.max()
+            if events is not None:
+                events[i][0].record(stream)
+            call()
+            if events is not None:
+                events[i][1].record(stream)
+
+    for _ in range(max(args.warmup, 1)):
+        step(None)
+    assert dg.dg_get_last_error() == 0, "device error during warm-up"
+    events = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in cases]
+              for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank)
+    if use_dist:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    launches0 = dg.dg_launch_count()
+    for s_ in range(args.steps):
+        step(events[s_])
+    torch.cuda.synchronize()
+    launches = dg.dg_launch_count() - launches0
+    clocks = sampler.stop()
+    assert dg.dg_get_last_error() == 0, "device error during timing"
+    ms = [sum(events[s_][i][0].elapsed_time(events[s_][i][1]) for s_ in range(args.steps)) / args.steps
+          for i in range(len(cases))]
+    t = torch.tensor([sum(ms)], dtype=torch.float64, device="cuda")
+    if use_dist:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    peaks, peak_kind = load_peaks()
+    fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
+    hbm = peaks["hbm_gbs"]
+    ridge = fp8_peak * 1e12 / (hbm * 1e9)
+    per_case = []
+    for (name, _, f, by), m_ in zip(cases, ms):
+        tf, gbs = f / (m_ * 1e-3) / 1e12, by / (m_ * 1e-3) / 1e9
+        bound = "tensor" if f / by >= ridge else "hbm"
+        per_case.append({"case": name, "us": round(m_ * 1e3, 2), "tflops": round(tf, 1), "gbs": round(gbs, 1),
+                         "bound": bound, "frac": round(tf / fp8_peak if bound == "tensor" else gbs / hbm, 4)})
+    dom = max(range(len(cases)), key=lambda i: ms[i])
+    pc = per_case[dom]
+    roofline = {"bound": pc["bound"], "achieved": pc["tflops"] if pc["bound"] == "tensor" else pc["gbs"],
+                "peak": round(fp8_peak, 1) if pc["bound"] == "tensor" else hbm,
+                "unit": "TFLOP/s" if pc["bound"] == "tensor" else "GB/s", "frac": pc["frac"], "traffic": None,
+                "kernel": f"gemm_kernel on {pc['case']}",
+                "peak_source": f"{peak_kind}: FP8 = bf16 burst {peaks['bf16_tflops']} x {FP8_PER_BF16}; HBM {hbm} GB/s"}
+    if rank == 0:
+        value = world * sum(c[2] for c in cases) / (float(t.item()) * 1e-3) / 1e12
+        line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(float(t.item()), 4), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+                "config": {"workload": args.workload, "cases": len(cases),
+                           "l2": "flushed before every timed call: 256 MB write then 256 MB read, not timed",
+                           "parallelism": f"replicas x{world}"},
+                "roofline": roofline, "cpu_baseline": None, "e2e": None, "gpu_launches": int(launches),
+                "clocks": clocks, "per_case": per_case}
+        print(json.dumps(line), flush=True)
+
+
 # ---------------------------------------------------------------- CPU oracle
 
 def oracle_prepare(shapes, seed=0):
@@ -290,6 +469,13 @@ def main():
     if use_dist:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
+
+    if args.workload != "dense":
+        run_grouped(args, dg, torch, rank, world, use_dist, local_rank)
+        if use_dist:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
 
     shapes = shapes_from(args)
     gen = torch.Generator(device="cuda")
