@@ -656,7 +656,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto store_chunk = [&](int col0, const uint32_t (&packed)[kEpiCols / 2]) {
         if (vr == 32) {
           // full 32-row box: swizzled staging (64-byte rows) + TMA store
-          DG_CHECK((smem_u32(stg) & 1023) == 0 && stg >= s_epi && stg + 2048 <= s_epi + C::kEpiBytes &&
+          // 64-byte swizzle: the pattern XORs address bits 7-8 into 4-5, so the
+          // staging box needs 512-byte alignment
+          DG_CHECK((smem_u32(stg) & 511) == 0 && stg >= s_epi && stg + 2048 <= s_epi + C::kEpiBytes &&
                        (col0 % 8) == 0 && r0 + 32 <= (LAYOUT == kMasked ? limit_rows : a.rows),
                    7);
           if (lane == 0) bulk_wait_group_read<0>();

@@ -24,6 +24,15 @@ def dg():
     assert dg.dg_get_last_error() == 0
 
 
+@pytest.fixture(autouse=True)
+def no_device_error_left(dg):
+    # every test leaves the device error word clear (tests that provoke an
+    # error read and clear it themselves), so a kernel self-check that fires
+    # is reported by the test that triggered it
+    yield
+    assert dg.dg_get_last_error() == 0, "device error recorded during this test"
+
+
 # ------------------------------------------------------------------ prep
 
 @pytest.mark.parametrize("rows,cols", [(1, 128), (300, 512)])
