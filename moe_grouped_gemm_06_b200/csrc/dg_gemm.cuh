@@ -569,28 +569,49 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* stg = s_epi + (warp - 2) * (32 * 64);
     int local = 0;
     // where this warp releases an accumulator buffer: the leader's barrier
-    // C of one unit for this warp's 32 rows x kCols columns (zeros where there
-    // is no C or no row), read row-wise into registers
+    // C of one unit for this warp's 32 rows x kCols columns, loaded
+    // coalesced: in load i the four lanes 4r..4r+3 read the four 16-byte
+    // pieces of row 8i + r of each 32-column chunk, so one warp load covers 8
+    // rows x 64 contiguous bytes (zeros where there is no C or no row).
+    // dst[j][i] is piece (lane & 3) of row 8i + (lane >> 2) of chunk j;
+    // stage_c() hands each lane its own row through the staging box.
     auto load_c_rows = [&](uint4 (&dst)[kChunks][4], const Unit& uu, bool want) {
 #pragma unroll
       for (int j = 0; j < kChunks; ++j)
 #pragma unroll
-        for (int v = 0; v < 4; ++v) dst[j][v] = make_uint4(0u, 0u, 0u, 0u);
+        for (int i = 0; i < 4; ++i) dst[j][i] = make_uint4(0u, 0u, 0u, 0u);
+      if (!want) return;
       const int rr0 = uu.mb * kTileM + (int)rank * kBM + q * 32;
       int lim = a.rows;
       if (LAYOUT == kMasked) lim = min(max(__ldg(a.masked_m + uu.g), 0), a.rows);
-      const int rrow = rr0 + (int)lane;
-      const long long rg = (LAYOUT == kMasked) ? (long long)uu.g * a.rows + rrow : rrow;
       const int cw = uu.nb * BN + half * kCols;
-      if (want && rrow < lim &&
-          DG_CHECK(((reinterpret_cast<uintptr_t>(a.c + rg * a.n + cw) & 15) == 0) && rrow < a.rows && rg >= 0, 1)) {
-        const uint4* src = reinterpret_cast<const uint4*>(a.c + rg * a.n + cw);
+      const int seg = (int)(lane & 3);
 #pragma unroll
-        for (int j = 0; j < kChunks; ++j)
+      for (int i = 0; i < 4; ++i) {
+        const int rrow = rr0 + 8 * i + (int)(lane >> 2);
+        const long long rg = (LAYOUT == kMasked) ? (long long)uu.g * a.rows + rrow : rrow;
+        if (rrow < lim &&
+            DG_CHECK(((reinterpret_cast<uintptr_t>(a.c + rg * a.n + cw) & 15) == 0) && rrow < a.rows && rg >= 0, 1)) {
+          const uint4* src = reinterpret_cast<const uint4*>(a.c + rg * a.n + cw) + seg;
 #pragma unroll
-          for (int v = 0; v < 4; ++v)
-            if (j < nch_w && cw + j * kEpiCols + 8 * v < a.n) dst[j][v] = __ldg(src + j * 4 + v);
+          for (int j = 0; j < kChunks; ++j)
+            if (j < nch_w && cw + j * kEpiCols + 8 * seg < a.n) dst[j][i] = __ldg(src + j * 4);
+        }
       }
+    };
+    // C of chunk j (as loaded by load_c_rows) into the staging box, in the
+    // swizzled layout the D store uses; each lane then reads its own row's
+    // pieces back while converting, and the bf16 result overwrites them
+    auto stage_c = [&](const uint4 (&cj)[4]) {
+      if (lane == 0) bulk_wait_group_read<0>();  // the previous TMA store has read the box
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int rw = 8 * i + (int)(lane >> 2);
+        const int pos = (int)(lane & 3) ^ ((rw >> 1) & 3);
+        *reinterpret_cast<uint4*>(stg + rw * 64 + pos * 16) = cj[i];
+      }
+      __syncwarp();
     };
     // one unit of look-ahead for C where registers allow
     constexpr bool kPrefetchC = (kChunks <= 3);
@@ -729,11 +750,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                        ((t_row >> 16) & 0xFFFF) == (uint32_t)(q * 32) + (tmem_base >> 16) && (warp & 3) == q,
                    8);
           tc_ld_32x32b_x32(t_row + j * kEpiCols, acc);
+          if (load_c) stage_c(creg[j]);
           tc_wait_ld_regs(acc);
           uint32_t packed[kEpiCols / 2];
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
-            const uint32_t cw[4] = {creg[j][v].x, creg[j][v].y, creg[j][v].z, creg[j][v].w};
+            const uint4 c4 = load_c ? *reinterpret_cast<const uint4*>(stg + lane * 64 + ((v ^ ((lane >> 1) & 3)) * 16))
+                                    : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t cw[4] = {c4.x, c4.y, c4.z, c4.w};
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
               const int i = 4 * v + h;

@@ -141,14 +141,18 @@ long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
 // and 224 re-base their scale words on the MMA-issuing thread, which costs
 // more than they gain; they are available through dg_set_tile_config but
 // never chosen automatically.
+// FP4 B (per_kb_fp4) is staged from half the bytes, which helps wide tiles,
+// but every K-block needs its own scale-factor copy into TMEM ahead of its
+// MMAs (1x32 scales), which costs narrow tiles.
 struct WidthCost {
   int bn;
   double per_kb, per_tile, epilogue;
   bool automatic;
+  double per_kb_fp4;
 };
 constexpr WidthCost kWidthCosts[] = {
-    {128, 0.2305, 1.9, 2.94, true}, {160, 0.32, 2.4, 3.6, false}, {192, 0.368, 1.6, 3.97, true},
-    {224, 0.41, 3.0, 4.6, false},   {256, 0.4236, 4.34, 0.0, true},
+    {128, 0.2305, 1.9, 2.94, true, 0.264}, {160, 0.32, 2.4, 3.6, false, 0.33}, {192, 0.368, 1.6, 3.97, true, 0.345},
+    {224, 0.41, 3.0, 4.6, false, 0.36},    {256, 0.4236, 4.34, 0.0, true, 0.343},
 };
 
 // Tile-configuration override (dg_set_tile_config; initial values from the
@@ -206,7 +210,7 @@ int sk_max_segments(int sk_tiles, int kb, int G) {
 // among plans at the floor the one with the least estimated SM time wins.  Sharing is offered for the dense layout only
 // (allow_sk) and only within ws_cap bytes of workspace (0: no cap).  Ties
 // keep whole tiles.
-Plan plan_gemm(long long m_blocks, int n, int k, int sms, bool allow_sk, size_t ws_cap = 0) {
+Plan plan_gemm(long long m_blocks, int n, int k, int sms, bool allow_sk, size_t ws_cap = 0, bool fp4 = false) {
   Plan best;
   best.cost = 1e300;
   const int kb = k / 128;
@@ -215,7 +219,9 @@ Plan plan_gemm(long long m_blocks, int n, int k, int sms, bool allow_sk, size_t 
   const bool streams_b = m_blocks <= 2;
   const double hbm_floor = std::max((rows * k + (double)n * k + 4.0 * rows * n) / 5.5e6,
                                     streams_b ? (double)n * k / 4.0e6 : 0.0);
-  for (const WidthCost& wc : kWidthCosts) {
+  for (const WidthCost& base : kWidthCosts) {
+    WidthCost wc = base;
+    if (fp4) wc.per_kb = wc.per_kb_fp4;
     const int bn = wc.bn;
     if (forced_block_n() ? bn != forced_block_n() : !wc.automatic) continue;
     const long long tiles = m_blocks * ceil_div(n, bn);
@@ -377,7 +383,7 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
     plan = plan_gemm((long long)p.groups * ceil_div(em, dg::kBM), p.n, p.k, sms, false);
     plan.grid = (int)std::min<long long>((long long)p.groups * m_blocks * ceil_div(p.n, plan.bn), sms);
   } else {
-    plan = plan_gemm(m_blocks, p.n, p.k, sms, LAYOUT == dg::kDense, fixed_ws != nullptr ? fixed_ws_bytes : 0);
+    plan = plan_gemm(m_blocks, p.n, p.k, sms, LAYOUT == dg::kDense, fixed_ws != nullptr ? fixed_ws_bytes : 0, FP4);
   }
 
   dg::GemmArgs args{};
