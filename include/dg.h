@@ -214,8 +214,8 @@ dg_status dg_set_pdl(int enable);
 int dg_get_pdl(void);
 
 /* Restricts the tile heuristic (all later calls, all threads): block_n in
- * {128, 160, 192, 224, 256} (0 = the heuristic's choice among 128, 192, 256;
- * 160 and 224 are only used when forced) and schedule 0 (heuristic), 1
+ * {64, 128, 160, 192, 224, 256} (0 = the heuristic's choice among 128, 192,
+ * 256; the others are only used when forced) and schedule 0 (heuristic), 1
  * (whole tiles only), 2 (the last tiles cut into per-tile K-slices, one per
  * CTA) or 3 (stream-K: the last tiles' K-iterations shared evenly over the
  * grid); 2 and 3 apply to the dense calls whenever such a split exists.

@@ -151,7 +151,7 @@ struct WidthCost {
   double per_kb_fp4;
 };
 constexpr WidthCost kWidthCosts[] = {
-    {128, 0.2305, 1.9, 2.94, true, 0.264}, {160, 0.32, 2.4, 3.6, false, 0.33}, {192, 0.368, 1.6, 3.97, true, 0.345},
+    {64, 0.19, 1.5, 1.6, true, 0.21},      {128, 0.2305, 1.9, 2.94, true, 0.264}, {160, 0.32, 2.4, 3.6, false, 0.33}, {192, 0.368, 1.6, 3.97, true, 0.345},
     {224, 0.41, 3.0, 4.6, false, 0.36},    {256, 0.4236, 4.34, 0.0, true, 0.343},
 };
 
@@ -224,6 +224,9 @@ Plan plan_gemm(long long m_blocks, int n, int k, int sms, bool allow_sk, size_t 
     if (fp4) wc.per_kb = wc.per_kb_fp4;
     const int bn = wc.bn;
     if (forced_block_n() ? bn != forced_block_n() : !wc.automatic) continue;
+    // 64-wide tiles double the CTAs of a dense problem of at most two
+    // m-blocks; elsewhere (and for the grouped layouts) they only add A reads
+    if (bn == 64 && !forced_block_n() && !(streams_b && allow_sk)) continue;
     const long long tiles = m_blocks * ceil_div(n, bn);
     auto consider = [&](const Plan& p) {
       if (p.cost < best.cost * (1 - 1e-9)) best = p;
@@ -344,6 +347,7 @@ dg_status dispatch(int bn, int ctas, const CUtensorMap& ta, const CUtensorMap& t
   // with "illegal instruction" and the cause is not yet known.
   if (ctas != 1) return DG_ERR_UNSUPPORTED;
   switch (bn) {
+    case 64: return launch_gemm<64, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
     case 128: return launch_gemm<128, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
     case 160: return launch_gemm<160, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
     case 192: return launch_gemm<192, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);

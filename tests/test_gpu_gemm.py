@@ -104,7 +104,7 @@ def test_dense_matches_oracle(dg, M, N, K, with_c):
 
 @pytest.mark.parametrize("schedule", [2, 3])
 @pytest.mark.parametrize("sms", [0, 7])
-@pytest.mark.parametrize("bn", [128, 192, 256])
+@pytest.mark.parametrize("bn", [64, 128, 192, 256])
 @pytest.mark.parametrize("M,N,K,with_c,fp4", [
     (1100, 520, 512, True, False),     # ragged M and N tails, 4 K-blocks
     (300, 1000, 1536, True, False),    # pieces that start and end inside tiles
@@ -150,11 +150,12 @@ def test_dense_shared_tail_is_deterministic_and_agrees_with_whole_tiles(dg):
         check_close(outs[sched][0], p.ref(), f"schedule {sched} vs oracle")
 
 
-@pytest.mark.parametrize("bn", [160, 224])
+@pytest.mark.parametrize("bn", [64, 160, 224])
 @pytest.mark.parametrize("M,N,K,fp4", [(300, 1000, 1024, False), (1100, 2112, 512, False), (200, 904, 512, True)])
-def test_dense_rebased_scale_widths(dg, bn, M, N, K, fp4):
-    # widths that start tiles 32 or 96 rows into a 128-row scale chunk: the B
-    # scale words are re-based in shared memory before the TMEM copy
+def test_dense_forced_widths(dg, bn, M, N, K, fp4):
+    # widths the heuristic does not pick by default: 64 (narrow tiles for small
+    # M), and 160 / 224, which start tiles 32 or 96 rows into a 128-row scale
+    # chunk so the B scale words are re-based in shared memory first
     dg.dg_set_tile_config(bn, 1)
     try:
         assert dg.dg_query_dense_config(M, N, K)["block_n"] == bn
@@ -164,8 +165,8 @@ def test_dense_rebased_scale_widths(dg, bn, M, N, K, fp4):
         dg.dg_set_tile_config(0, 0)
 
 
-@pytest.mark.parametrize("bn", [160, 224])
-def test_grouped_rebased_scale_widths(dg, bn):
+@pytest.mark.parametrize("bn", [64, 160, 224])
+def test_grouped_forced_widths(dg, bn):
     dg.dg_set_tile_config(bn, 1)
     try:
         N, K = 1000, 512
