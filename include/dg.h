@@ -236,6 +236,11 @@ dg_status dg_get_last_error(void* stream);
  * DG_ERR_TIMEOUT.  Faults nothing and leaves the context usable. */
 dg_status dg_debug_starved_wait(unsigned int limit_us, void* stream);
 
+/* Test hook: n / d computed the way the kernels divide by per-launch
+ * constants (multiply-high, add, shift); d >= 1 and n < 2^31, else
+ * 0xFFFFFFFF. */
+uint32_t dg_debug_fastdiv(uint32_t d, uint32_t n);
+
 /* Human-readable name of a status code (static string). */
 const char* dg_status_string(int status);
 

@@ -22,7 +22,7 @@ __all__ = [
     "dg_m_grouped_fp8_gemm_nt_masked", "dg_fp8_gemm_nt_noalloc", "dg_noalloc_scratch_bytes", "dg_fp8_fp4_gemm_nt", "dg_m_grouped_fp8_fp4_gemm_nt_contiguous",
     "dg_quantize_fp8", "dg_quantize_fp4", "dg_pack_sf", "dg_packed_sf_words", "dg_get_num_sms",
     "dg_set_num_sms", "dg_set_pdl", "dg_get_pdl", "dg_set_tile_config", "dg_get_mk_alignment_for_contiguous_layout", "dg_get_last_error",
-    "dg_debug_starved_wait", "dg_launch_count", "dg_query_dense_config", "dg_num_tiles", "dg_shutdown",
+    "dg_debug_starved_wait", "dg_launch_count", "dg_query_dense_config", "dg_num_tiles", "dg_debug_fastdiv", "dg_shutdown",
     "SYMBOLS",
 ]
 
@@ -60,6 +60,7 @@ SYMBOLS = {
     "dg_launch_count": (ctypes.c_uint64, []),
     "dg_query_dense_config": (_INT, [_INT, _INT, _INT, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "dg_num_tiles": (_I64, [_INT, _INT, _INT, _INT]),
+    "dg_debug_fastdiv": (ctypes.c_uint32, [ctypes.c_uint32, ctypes.c_uint32]),
     "dg_shutdown": (None, []),
 }
 
@@ -249,6 +250,10 @@ def dg_query_dense_config(m: int, n: int, k: int, workspace_cap: int = 0) -> dic
 
 def dg_num_tiles(m: int, n: int, block_m: int, block_n: int) -> int:
     return int(lib().dg_num_tiles(m, n, block_m, block_n))
+
+
+def dg_debug_fastdiv(d: int, n: int) -> int:
+    return int(lib().dg_debug_fastdiv(d, n))
 
 
 def dg_shutdown() -> None:

@@ -45,6 +45,29 @@ constexpr int kMaxMaskedGroups = 1024;
 
 enum : int { kDense = 0, kContig = 1, kMasked = 2 };
 
+// Unsigned division by a run-time divisor d >= 1 fixed per launch, as one
+// multiply-high, an add and a shift (Granlund and Montgomery, "Division by
+// invariant integers using multiplication", 1994): with s = ceil(log2 d) and
+// m = floor(2^32 (2^s - d) / d) + 1, n / d = (mulhi(n, m) + n) >> s for every
+// n < 2^31.
+struct FastDiv {
+  uint32_t d, mul, shift;
+  __host__ __device__ void init(uint32_t dd) {
+    d = dd;
+    shift = 0;
+    while ((1ull << shift) < d) ++shift;
+    mul = (uint32_t)(((1ull << 32) * ((1ull << shift) - d)) / d + 1);
+  }
+  __host__ __device__ __forceinline__ uint32_t div(uint32_t n) const {
+#ifdef __CUDA_ARCH__
+    const uint32_t t = __umulhi(n, mul);
+#else
+    const uint32_t t = (uint32_t)(((uint64_t)n * mul) >> 32);
+#endif
+    return (t + n) >> shift;
+  }
+};
+
 struct GemmArgs {
   const int32_t* sfa;        // packed scale words of A
   const int32_t* sfb;        // packed scale words of B
@@ -74,6 +97,7 @@ struct GemmArgs {
   long long sfa_group_words, sfb_group_words;
   int sfa_q, sfb_q;                    // packed groups along K
   int raster;                          // m-blocks per raster band
+  FastDiv band_div;                    // division by raster * num_n_blocks (tiles per band)
   unsigned long long timeout_ns;
   long long sfa_words, sfb_words;      // total packed words (self-check bounds)
 };
@@ -153,6 +177,21 @@ __host__ __device__ __forceinline__ void raster_tile(int tl, int raster, int num
   nb = rem / band_rows;
 }
 
+// raster_tile with the band division precomputed (FastDiv) and the usual
+// band height of 8 m-blocks done with a shift and a mask.
+__device__ __forceinline__ void raster_tile_fast(int tl, const GemmArgs& a, int& mb, int& nb) {
+  const int band = (int)a.band_div.div((uint32_t)tl);
+  const int rem = tl - band * (int)a.band_div.d;
+  const int band_rows = min(a.raster, a.num_m_blocks - band * a.raster);
+  if (band_rows == 8) {
+    mb = band * 8 + (rem & 7);
+    nb = rem >> 3;
+  } else {
+    mb = band * a.raster + rem % band_rows;
+    nb = rem / band_rows;
+  }
+}
+
 // Work units of one CTA, in the order all three roles walk them.
 // Dense: the whole tiles t = cta, cta + G, ... below dp_tiles, then this
 // CTA's stream-K share cut at tile boundaries.  Contiguous: every tile of the
@@ -185,8 +224,15 @@ struct WorkIter {
     u.kb1 = a.kb_total;
     if (t < num_units) {
       if (LAYOUT == kMasked) {
-        int g = 0;
-        while (s_prefix[g + 1] <= t) ++g;
+        // the group whose tile range holds t: s_prefix[g] <= t < s_prefix[g + 1]
+        int g = 0, hi = a.num_groups;
+        while (hi - g > 1) {
+          const int mid = (g + hi) >> 1;
+          if (s_prefix[mid] <= t)
+            g = mid;
+          else
+            hi = mid;
+        }
         const int local = t - s_prefix[g];
         const int valid_rows = min(max(__ldg(a.masked_m + g), 0), a.rows);
         const int mcount = (valid_rows + kBM - 1) / kBM;
@@ -194,7 +240,7 @@ struct WorkIter {
         u.nb = local / mcount;
         u.mb = local % mcount;
       } else {
-        raster_tile(t, a.raster, a.num_m_blocks, a.num_n_blocks, u.mb, u.nb);
+        raster_tile_fast(t, a, u.mb, u.nb);
         if (LAYOUT == kContig) {
           const int g = __ldg(a.m_indices + (long long)u.mb * kBM);  // 1-CTA tiles only
           u.g = g;
@@ -213,7 +259,7 @@ struct WorkIter {
       u.slot = t;
       u.kb0 = (int)((long long)t * kbt / a.sk_split);
       u.kb1 = (int)((long long)(t + 1) * kbt / a.sk_split);
-      raster_tile(a.dp_tiles + j, a.raster, a.num_m_blocks, a.num_n_blocks, u.mb, u.nb);
+      raster_tile_fast(a.dp_tiles + j, a, u.mb, u.nb);
       x = x_end;
       return true;
     }
@@ -223,7 +269,7 @@ struct WorkIter {
     const long long left = x_end - x;
     u.kb1 = (left < (long long)(kbt - u.kb0)) ? u.kb0 + (int)left : kbt;
     u.slot = cta - sk_cta_of((long long)j * kbt, step, a.sk_iters);
-    raster_tile(a.dp_tiles + j, a.raster, a.num_m_blocks, a.num_n_blocks, u.mb, u.nb);
+    raster_tile_fast(a.dp_tiles + j, a, u.mb, u.nb);
     x += u.kb1 - u.kb0;
     return true;
   }
@@ -624,9 +670,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       else
         mbar_arrive(&tempty[b]);
     };
+    // the iterator runs one unit ahead, so each unit is decoded once and the
+    // next unit (un) is known for the C prefetch
     WorkIter<LAYOUT> it(a, cta_id, num_ctas);
-    Unit u;
-    while (it.next(a, s_prefix, num_units, u)) {
+    Unit u, un;
+    bool has_un = it.next(a, s_prefix, num_units, un);
+    while (has_un) {
+      u = un;
+      has_un = it.next(a, s_prefix, num_units, un);
       if (LAYOUT == kContig && !u.valid) continue;
       const int buf = local % C::kAccBufs;
       const uint32_t use = (uint32_t)(local / C::kAccBufs);
@@ -653,13 +704,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // issue the loads of the next unit's C now, so that they arrive while
         // this unit is drained and stored
         have_next_c = false;
-        if (a.c != nullptr) {
-          WorkIter<LAYOUT> peek = it;
-          Unit un;
-          if (peek.next(a, s_prefix, num_units, un) && un.valid && un.slot < 0) {
-            load_c_rows(cnext, un, true);
-            have_next_c = true;
-          }
+        if (a.c != nullptr && has_un && un.valid && un.slot < 0) {
+          load_c_rows(cnext, un, true);
+          have_next_c = true;
         }
       } else {
         load_c_rows(creg, u, load_c);

@@ -417,6 +417,7 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
   args.sfa_group_words = (long long)args.sfa_q * args.sfa_chunks * 128;
   args.sfb_group_words = (long long)args.sfb_q * args.sfb_chunks * 128;
   args.raster = 8;
+  args.band_div.init((uint32_t)(args.raster * args.num_n_blocks));
   args.timeout_ns = timeout_ns();
   args.sfa_words = args.sfa_group_words * ((LAYOUT == dg::kMasked) ? p.groups : 1);
   args.sfb_words = args.sfb_group_words * ((LAYOUT == dg::kDense) ? 1 : p.groups);
@@ -742,6 +743,13 @@ dg_status dg_query_dense_config(int m, int n, int k, int64_t workspace_cap, int*
   if (grid) *grid = p.grid;
   if (workspace_bytes) *workspace_bytes = (int64_t)p.ws_bytes();
   return DG_OK;
+}
+
+uint32_t dg_debug_fastdiv(uint32_t d, uint32_t n) {
+  if (d == 0 || n >= (1u << 31)) return 0xFFFFFFFFu;
+  dg::FastDiv f;
+  f.init(d);
+  return f.div(n);
 }
 
 int64_t dg_num_tiles(int m, int n, int block_m, int block_n) {

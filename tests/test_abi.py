@@ -219,3 +219,19 @@ def test_tile_config_override(dg):
     finally:
         dg.dg_set_tile_config(0, 0)
         dg.dg_set_num_sms(0)
+
+
+def test_fast_division_matches_integer_division(dg):
+    # the kernels divide tile indices by per-launch constants with a
+    # multiply-high and a shift; it must equal integer division exactly
+    import random
+    rnd = random.Random(7)
+    divisors = list(range(1, 300)) + [2 ** p for p in range(31)] + [2 ** p - 1 for p in range(2, 32)] + \
+        [rnd.randrange(1, 2 ** 31) for _ in range(300)]
+    for d in divisors:
+        ns = [0, 1, d - 1, d, d + 1, 2 ** 31 - 1, 2 ** 31 - 2] + [rnd.randrange(0, 2 ** 31) for _ in range(40)]
+        for n in ns:
+            if 0 <= n < 2 ** 31:
+                assert dg.lib().dg_debug_fastdiv(d, n) == n // d, (d, n)
+    assert dg.lib().dg_debug_fastdiv(0, 5) == 0xFFFFFFFF
+    assert dg.lib().dg_debug_fastdiv(3, 2 ** 31) == 0xFFFFFFFF
