@@ -60,6 +60,8 @@ def parse_args():
     ap.add_argument("--workload", default="dense", choices=["dense", "contiguous", "masked", "fp4"],
                     help="dense: the DeepSeek-V3 dense sweep (default); contiguous / masked / fp4: the "
                          "M-grouped prefill, masked decode and FP8 x FP4 cases, one JSON line each")
+    ap.add_argument("--graph", action="store_true",
+                    help="grouped workloads: capture each case's call in a CUDA graph and time its replay")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -303,6 +305,22 @@ def run_grouped(args, dg, torch, rank, world, use_dist, local_rank):
     gen = torch.Generator(device="cuda")
     gen.manual_seed(4321 + rank)
     cases = grouped_cases(dg, torch, args.workload, gen, 99 + rank)
+    graphs = []
+    if args.graph:
+        # one CUDA graph per case (the calls read their group metadata on the
+        # device, so a captured launch is replayable); first call eager
+        cap = torch.cuda.Stream()
+        for i, (name, call, f, by) in enumerate(cases):
+            with torch.cuda.stream(cap):
+                call()
+            cap.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                call()
+            # the graph holds raw pointers into the case's tensors: keep the
+            # original call (whose closure owns them) alive with the graph
+            graphs.append((g, call))
+            cases[i] = (name, g.replay, f, by)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     flush_rd = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
     stream = torch.cuda.current_stream()
@@ -320,7 +338,8 @@ def run_grouped(args, dg, torch, rank, world, use_dist, local_rank):
 
     for _ in range(max(args.warmup, 1)):
         step(None)
-    assert dg.dg_get_last_error() == 0, "device error during warm-up"
+    err = dg.dg_get_last_error()
+    assert err == 0, f"device error during warm-up: {dg.status_string(err)} ({err})"
     events = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in cases]
               for _ in range(args.steps)]
     sampler = ClockSampler(local_rank)
@@ -335,7 +354,8 @@ def run_grouped(args, dg, torch, rank, world, use_dist, local_rank):
     torch.cuda.synchronize()
     launches = dg.dg_launch_count() - launches0
     clocks = sampler.stop()
-    assert dg.dg_get_last_error() == 0, "device error during timing"
+    err = dg.dg_get_last_error()
+    assert err == 0, f"device error during timing: {dg.status_string(err)} ({err})"
     ms = [sum(events[s_][i][0].elapsed_time(events[s_][i][1]) for s_ in range(args.steps)) / args.steps
           for i in range(len(cases))]
     t = torch.tensor([sum(ms)], dtype=torch.float64, device="cuda")
@@ -363,7 +383,7 @@ def run_grouped(args, dg, torch, rank, world, use_dist, local_rank):
         line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": round(float(t.item()), 4), "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
-                "config": {"workload": args.workload, "cases": len(cases),
+                "config": {"workload": args.workload, "cases": len(cases), "cuda_graph": bool(args.graph),
                            "l2": "flushed before every timed call: 256 MB write then 256 MB read, not timed",
                            "parallelism": f"replicas x{world}"},
                 "roofline": roofline, "cpu_baseline": None, "e2e": None, "gpu_launches": int(launches),
@@ -510,7 +530,8 @@ def main():
 
     for _ in range(max(args.warmup, 1)):
         sweep(None)
-    assert dg.dg_get_last_error() == 0, "device error during warm-up"
+    err = dg.dg_get_last_error()
+    assert err == 0, f"device error during warm-up: {dg.status_string(err)} ({err})"
 
     events = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in shapes] for _ in range(args.steps)]
@@ -530,7 +551,8 @@ def main():
     if use_dist:
         dist.barrier()
     clocks = sampler.stop()
-    assert dg.dg_get_last_error() == 0, "device error during timing"
+    err = dg.dg_get_last_error()
+    assert err == 0, f"device error during timing: {dg.status_string(err)} ({err})"
 
     per_shape_ms = [sum(events[s][i][0].elapsed_time(events[s][i][1]) for s in range(args.steps)) / args.steps
                     for i in range(len(shapes))]

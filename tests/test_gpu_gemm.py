@@ -340,6 +340,41 @@ def test_masked_matches_oracle_and_leaves_rows(dg):
             check_close(dd[g, :v], ref[g, :v], f"masked group {g}")
 
 
+def test_masked_decode_replays_from_a_cuda_graph(dg):
+    # The masked call reads masked_m on the device and allocates nothing, so
+    # one captured launch serves every step of a decode loop: the counts are
+    # rewritten in place between replays.
+    G, max_m, N, K = 4, 128, 256, 512
+    qa, ea, sfa, qb, eb, sfb = _masked_case(5600, G, max_m, N, K, np.full(G, max_m, np.int32))
+    t_a, t_sfa, t_b, t_sfb = dev(qa), dev(sfa), dev(qb), dev(sfb)
+    t_mm = torch.zeros(G, dtype=torch.int32, device="cuda")
+    d = torch.full((G, max_m, N), SENTINEL, dtype=torch.int16, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):            # first call outside the capture (kernel attributes)
+        dg.dg_m_grouped_fp8_gemm_nt_masked(t_a, t_sfa, t_b, t_sfb, d, t_mm, expected_m=32)
+    s.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    launches = dg.dg_launch_count()
+    with torch.cuda.graph(graph, stream=s):
+        dg.dg_m_grouped_fp8_gemm_nt_masked(t_a, t_sfa, t_b, t_sfb, d, t_mm, expected_m=32)
+    assert dg.dg_launch_count() == launches + 1
+    for counts in ([0, 5, 128, 77], [128, 0, 1, 64], [33, 33, 33, 33]):
+        mm = np.array(counts, np.int32)
+        d.fill_(SENTINEL)
+        t_mm.copy_(torch.from_numpy(mm))
+        graph.replay()
+        torch.cuda.synchronize()
+        assert dg.dg_get_last_error() == 0
+        ref = oracle.gemm_masked(qa, ea, qb, eb, mm)
+        got = bf16_dev_to_f64(d)
+        raw = host(d).view(np.uint16)
+        for g in range(G):
+            if mm[g] > 0:
+                check_close(got[g, :mm[g]], ref[g, :mm[g]], f"graph replay {counts} g={g}")
+            assert np.all(raw[g, mm[g]:] == SENTINEL), f"graph replay {counts}: rows >= masked_m written"
+    del graph
+
+
 def test_masked_count_above_max_is_clamped_and_reported(dg):
     G, max_m, N, K = 2, 128, 128, 256
     mm = np.array([300, 5], np.int32)
