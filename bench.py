@@ -57,7 +57,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--shape", default=None, help="run one M,N,K shape instead of the sweep")
-    ap.add_argument("--workload", default="dense", choices=["dense", "contiguous", "masked", "fp4"],
+    ap.add_argument("--workload", default="dense", choices=["dense", "contiguous", "masked", "fp4", "moe_decode_fp4"],
                     help="dense: the DeepSeek-V3 dense sweep (default); contiguous / masked / fp4: the "
                          "M-grouped prefill, masked decode and FP8 x FP4 cases, one JSON line each")
     ap.add_argument("--graph", action="store_true",
@@ -282,6 +282,33 @@ def grouped_cases(dg, torch, workload, gen, seed):
                 cases.append((name, (lambda a=a, sfa=sfa, b=b, sfb=sfb, d=d, t_mm=t_mm, em=em:
                                      dg.dg_m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, t_mm, expected_m=em)),
                               2.0 * valid * n * k, by))
+    elif workload == "moe_decode_fp4":
+        # one MoE decode step per expected_m with FP4 expert weights:
+        # linear1 (N = 2 x 2048 gate/up rows interleaved by 64, K = 7168) with
+        # SwiGLU fused, then linear2 (N = 7168, K = 2048)
+        G, max_m = MASKED_GROUPS, MASKED_MAX_M
+        b1, sfb1 = quant_b_dev(dg, torch, G, 4096, 7168, gen, fp4=True)
+        b2, sfb2 = quant_b_dev(dg, torch, G, 7168, 2048, gen, fp4=True)
+        for em in MASKED_EXPECTED:
+            mm = np.minimum(rng.integers(0, 2 * em + 1, G), max_m).astype(np.int32)
+            t_mm = torch.from_numpy(mm).cuda()
+            valid = int(mm.sum())
+            a1, sfa1 = quant_a_dev(dg, torch, max_m, 7168, gen, groups=G)
+            a1 = a1.view(G, max_m, 7168)
+            act = torch.empty((G, max_m, 2048), dtype=torch.bfloat16, device="cuda")
+            a2, sfa2 = quant_a_dev(dg, torch, max_m, 2048, gen, groups=G)
+            a2 = a2.view(G, max_m, 2048)
+            out = torch.empty((G, max_m, 7168), dtype=torch.bfloat16, device="cuda")
+            by1 = valid * 7168 + G * 4096 * 7168 // 2 + 2 * valid * 2048 + sfb1.numel() * 4
+            by2 = valid * 2048 + G * 7168 * 2048 // 2 + 2 * valid * 7168 + sfb2.numel() * 4
+            cases.append((f"linear1+SwiGLU fp4 G={G} expected_m={em} ({valid} valid rows) N=4096 K=7168",
+                          (lambda a=a1, sfa=sfa1, d=act, t=t_mm, em=em:
+                           dg.dg_m_grouped_fp8_fp4_gemm_nt_masked_swiglu(a, sfa, b1, sfb1, d, t, expected_m=em)),
+                          2.0 * valid * 4096 * 7168, by1))
+            cases.append((f"linear2 fp4 G={G} expected_m={em} ({valid} valid rows) N=7168 K=2048",
+                          (lambda a=a2, sfa=sfa2, d=out, t=t_mm, em=em:
+                           dg.dg_m_grouped_fp8_fp4_gemm_nt_masked(a, sfa, b2, sfb2, d, t, expected_m=em)),
+                          2.0 * valid * 7168 * 2048, by2))
     elif workload == "fp4":
         for (n, k) in GROUPED_NK:
             m = 4096

@@ -125,6 +125,36 @@ dg_status dg_m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa, con
                                           int num_groups, int max_m, int n, int k, int expected_m,
                                           void* stream);
 
+/* M-grouped masked FP8 x FP4 GEMM: as dg_m_grouped_fp8_gemm_nt_masked with
+ * B in e2m1 like dg_fp8_fp4_gemm_nt:
+ *   b    e2m1 [num_groups][n][k/2] (two per byte, low nibble = even k)
+ *   sfb  num_groups blocks of sf words, R = n, G = k/32 (one UE8M0 per 1x32)
+ * Source: linlog.top, "FP4 精度支持" (FP8 x FP4 GEMM); masked layout as above. */
+dg_status dg_m_grouped_fp8_fp4_gemm_nt_masked(const void* a, const int32_t* sfa, const void* b,
+                                              const int32_t* sfb, void* d, const int32_t* masked_m,
+                                              int num_groups, int max_m, int n, int k, int expected_m,
+                                              void* stream);
+
+/* Masked GEMM with SwiGLU fused into the epilogue (the linear1 -> SwiGLU step
+ * of a MoE expert: the pages' "linear1 -> SwiGLU -> linear2", charles2530.github.io
+ * "DeepGEMM：FP8 GEMM 与 Mega-MoE" and the Mega MoE section of the linlog.top page).
+ * B holds the gate and up projections with their rows interleaved in blocks
+ * of 64: B rows [128j, 128j + 64) are gate rows 64j.., rows [128j + 64,
+ * 128j + 128) the matching up rows.  With G = A * B^T in FP32 (n columns),
+ *   d[g][m][64j + i] = bf16( silu(G[m][128j + i]) * G[m][128j + 64 + i] ),
+ *   silu(x) = x / (1 + exp(-x)),   i < 64,
+ * so d is bf16 [num_groups][max_m][n/2].  Requires n % 128 == 0; no C.  The
+ * _fp4_ form takes B as in dg_m_grouped_fp8_fp4_gemm_nt_masked.  Other
+ * arguments, metadata rules and errors as dg_m_grouped_fp8_gemm_nt_masked. */
+dg_status dg_m_grouped_fp8_gemm_nt_masked_swiglu(const void* a, const int32_t* sfa, const void* b,
+                                                 const int32_t* sfb, void* d, const int32_t* masked_m,
+                                                 int num_groups, int max_m, int n, int k, int expected_m,
+                                                 void* stream);
+dg_status dg_m_grouped_fp8_fp4_gemm_nt_masked_swiglu(const void* a, const int32_t* sfa, const void* b,
+                                                     const int32_t* sfb, void* d, const int32_t* masked_m,
+                                                     int num_groups, int max_m, int n, int k, int expected_m,
+                                                     void* stream);
+
 /* Dense NT FP8 GEMM that allocates no memory.  The pages have no counterpart
  * of this call; it exists for callers that cannot allocate device memory at
  * call time -- for example code running under another framework's memory

@@ -19,7 +19,8 @@ import torch
 
 __all__ = [
     "DGError", "lib", "dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
-    "dg_m_grouped_fp8_gemm_nt_masked", "dg_fp8_gemm_nt_noalloc", "dg_noalloc_scratch_bytes", "dg_fp8_fp4_gemm_nt", "dg_m_grouped_fp8_fp4_gemm_nt_contiguous",
+    "dg_m_grouped_fp8_gemm_nt_masked", "dg_m_grouped_fp8_fp4_gemm_nt_masked",
+    "dg_m_grouped_fp8_gemm_nt_masked_swiglu", "dg_m_grouped_fp8_fp4_gemm_nt_masked_swiglu", "dg_fp8_gemm_nt_noalloc", "dg_noalloc_scratch_bytes", "dg_fp8_fp4_gemm_nt", "dg_m_grouped_fp8_fp4_gemm_nt_contiguous",
     "dg_quantize_fp8", "dg_quantize_fp4", "dg_pack_sf", "dg_packed_sf_words", "dg_get_num_sms",
     "dg_set_num_sms", "dg_set_pdl", "dg_get_pdl", "dg_set_tile_config", "dg_get_mk_alignment_for_contiguous_layout", "dg_get_last_error",
     "dg_debug_starved_wait", "dg_launch_count", "dg_query_dense_config", "dg_num_tiles", "dg_debug_fastdiv", "dg_shutdown",
@@ -37,8 +38,11 @@ SYMBOLS = {
     "dg_fp8_gemm_nt": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _INT, _INT, _INT, _VP]),
     "dg_m_grouped_fp8_gemm_nt_contiguous": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _I32P, _INT, _INT, _INT,
                                                    _INT, _VP]),
-    "dg_m_grouped_fp8_gemm_nt_masked": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _I32P, _INT, _INT, _INT, _INT, _INT,
-                                               _VP]),
+    "dg_m_grouped_fp8_gemm_nt_masked": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _I32P, _INT, _INT, _INT, _INT, _INT, _VP]),
+    "dg_m_grouped_fp8_fp4_gemm_nt_masked": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _I32P, _INT, _INT, _INT, _INT, _INT, _VP]),
+    "dg_m_grouped_fp8_gemm_nt_masked_swiglu": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _I32P, _INT, _INT, _INT, _INT, _INT, _VP]),
+    "dg_m_grouped_fp8_fp4_gemm_nt_masked_swiglu": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _I32P, _INT, _INT, _INT, _INT,
+                                                          _INT, _VP]),
     "dg_fp8_gemm_nt_noalloc": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _INT, _INT, _INT, _VP]),
     "dg_noalloc_scratch_bytes": (ctypes.c_size_t, []),
     "dg_fp8_fp4_gemm_nt": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _INT, _INT, _INT, _VP]),
@@ -172,6 +176,29 @@ def dg_m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, masked_m, expected_m: int
     _check(lib().dg_m_grouped_fp8_gemm_nt_masked(_p(a), _p(sfa), _p(b), _p(sfb), _p(d), _p(masked_m), g, max_m,
                                                  n, k, int(expected_m), _stream(stream)),
            "dg_m_grouped_fp8_gemm_nt_masked")
+
+
+def _masked_call(name, a, sfa, b, sfb, d, masked_m, expected_m, stream):
+    g, max_m, k = a.shape
+    n = b.shape[1]
+    _check(getattr(lib(), name)(_p(a), _p(sfa), _p(b), _p(sfb), _p(d), _p(masked_m), g, max_m, n, k,
+                                int(expected_m), _stream(stream)), name)
+
+
+def dg_m_grouped_fp8_fp4_gemm_nt_masked(a, sfa, b, sfb, d, masked_m, expected_m: int = 0, stream=None) -> None:
+    """a: e4m3 [groups, max_m, k]; b: e2m1 [groups, n, k/2]; d: bf16 [groups, max_m, n]."""
+    _masked_call("dg_m_grouped_fp8_fp4_gemm_nt_masked", a, sfa, b, sfb, d, masked_m, expected_m, stream)
+
+
+def dg_m_grouped_fp8_gemm_nt_masked_swiglu(a, sfa, b, sfb, d, masked_m, expected_m: int = 0, stream=None) -> None:
+    """b: e4m3 [groups, n, k], gate/up rows interleaved in blocks of 64; d: bf16 [groups, max_m, n/2]."""
+    _masked_call("dg_m_grouped_fp8_gemm_nt_masked_swiglu", a, sfa, b, sfb, d, masked_m, expected_m, stream)
+
+
+def dg_m_grouped_fp8_fp4_gemm_nt_masked_swiglu(a, sfa, b, sfb, d, masked_m, expected_m: int = 0,
+                                               stream=None) -> None:
+    """b: e2m1 [groups, n, k/2], gate/up rows interleaved in blocks of 64; d: bf16 [groups, max_m, n/2]."""
+    _masked_call("dg_m_grouped_fp8_fp4_gemm_nt_masked_swiglu", a, sfa, b, sfb, d, masked_m, expected_m, stream)
 
 
 # ------------------------------------------------------- input preparation

@@ -45,6 +45,12 @@ constexpr int kMaxMaskedGroups = 1024;
 
 enum : int { kDense = 0, kContig = 1, kMasked = 2 };
 
+// Epilogues: D = bf16(acc + C), or SwiGLU on B rows interleaved in blocks of
+// kSwiGluBlock (gate rows, then the matching up rows): act = bf16(silu(gate)
+// * up), half as many columns as the GEMM.
+enum : int { kEpiPlain = 0, kEpiSwiGlu = 1 };
+constexpr int kSwiGluBlock = 64;
+
 // Unsigned division by a run-time divisor d >= 1 fixed per launch, as one
 // multiply-high, an add and a shift (Granlund and Montgomery, "Division by
 // invariant integers using multiplication", 1994): with s = ceil(log2 d) and
@@ -78,6 +84,7 @@ struct GemmArgs {
   const int32_t* masked_m;   // masked: valid rows per group
   int rows;                  // dense: M; contiguous: M_total; masked: max_m
   int n, k;
+  int d_cols;                // columns of D: n, or n / 2 for SwiGLU
   int num_groups;
   int num_m_blocks;          // per group for masked
   int num_n_blocks;
@@ -278,12 +285,13 @@ struct WorkIter {
 // CTAS = 2: a cluster of two CTAs computes 256 x BN tiles (dense layout only);
 // tm_sfa / tm_sfb view the packed scale words as rows of 512 bytes so that
 // the peer's scale loads can complete on the leader's barrier.
-template <int BN, bool FP4, int LAYOUT, int CTAS>
+template <int BN, bool FP4, int LAYOUT, int CTAS, int EPI = kEpiPlain>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_d, const __grid_constant__ CUtensorMap tm_sfa,
                 const __grid_constant__ CUtensorMap tm_sfb, const GemmArgs args) {
   static_assert(CTAS == 1 || (CTAS == 2 && LAYOUT == kDense), "CTA pairs serve the dense layout");
+  static_assert(EPI == kEpiPlain || (CTAS == 1 && BN % (2 * kSwiGluBlock) == 0), "SwiGLU tiles hold whole block pairs");
   using C = Cfg<BN, FP4, CTAS>;
   constexpr bool kPair = (CTAS == 2);
   constexpr int kTileM = kBM * CTAS;
@@ -744,13 +752,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_commit_group();
           }
         } else if ((int)lane < vr &&
-                   DG_CHECK((reinterpret_cast<uintptr_t>(a.d + grow * a.n + col0) & 15) == 0 && row < limit_rows,
+                   DG_CHECK((reinterpret_cast<uintptr_t>(a.d + grow * a.d_cols + col0) & 15) == 0 && row < limit_rows,
                             2)) {
           // partial box (M tail or masked group tail): predicated row stores
-          uint4* dst = reinterpret_cast<uint4*>(a.d + grow * a.n + col0);
+          uint4* dst = reinterpret_cast<uint4*>(a.d + grow * a.d_cols + col0);
 #pragma unroll
           for (int v = 0; v < kEpiCols / 8; ++v)
-            if (col0 + 8 * v < a.n)
+            if (col0 + 8 * v < a.d_cols)
               dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
         }
       };
@@ -788,35 +796,68 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
 
+      if constexpr (EPI == kEpiSwiGlu) {
+        // ---- SwiGLU: the tile's BN columns are BN / 128 pairs of 64 gate and
+        // 64 up columns; its BN / 2 output columns are cut into 32-column
+        // chunks, the first half of them for warp half 0.  Output chunk c
+        // reads gate chunk 4 (c / 2) + c % 2 and up chunk 4 (c / 2) + 2 + c % 2.
+        constexpr int kOutCh = BN / (2 * kEpiCols);
+        const uint32_t t_tile = tmem_base + ((uint32_t)(q * 32) << 16) + C::kColAcc + buf * C::kAccStride;
 #pragma unroll
-      for (int j = 0; j < kChunks; ++j) {
-        const int col0 = colw + j * kEpiCols;
-        if (j < nch_w && vr > 0 && col0 < a.n) {
-          uint32_t acc[kEpiCols];
-          DG_CHECK(((t_row & 0xFFFF) + j * kEpiCols + kEpiCols <= (uint32_t)kTmemCols) &&
-                       ((t_row >> 16) & 0xFFFF) == (uint32_t)(q * 32) + (tmem_base >> 16) && (warp & 3) == q,
-                   8);
-          tc_ld_32x32b_x32(t_row + j * kEpiCols, acc);
-          if (load_c) stage_c(creg[j]);
-          tc_wait_ld_regs(acc);
-          uint32_t packed[kEpiCols / 2];
+        for (int e = 0; e < kOutCh / 2; ++e) {
+          const int c = half * (kOutCh / 2) + e;
+          const int col0 = u.nb * (BN / 2) + c * kEpiCols;
+          if (vr > 0 && col0 < a.d_cols) {
+            const int gch = 4 * (c >> 1) + (c & 1);
+            uint32_t g[kEpiCols], up[kEpiCols];
+            DG_CHECK(((t_tile & 0xFFFF) + (gch + 2) * kEpiCols + kEpiCols <= (uint32_t)kTmemCols), 8);
+            tc_ld_32x32b_x32(t_tile + gch * kEpiCols, g);
+            tc_ld_32x32b_x32(t_tile + (gch + 2) * kEpiCols, up);
+            tc_wait_ld_regs(g);
+            tc_wait_ld_regs(up);
+            uint32_t packed[kEpiCols / 2];
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const uint4 c4 = load_c ? *reinterpret_cast<const uint4*>(stg + lane * 64 + ((v ^ ((lane >> 1) & 3)) * 16))
-                                    : make_uint4(0u, 0u, 0u, 0u);
-            const uint32_t cw[4] = {c4.x, c4.y, c4.z, c4.w};
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              const int i = 4 * v + h;
-              __nv_bfloat162 bv = __floats2bfloat162_rn(__uint_as_float(acc[2 * i]) + __uint_as_float(cw[h] << 16),
-                                                        __uint_as_float(acc[2 * i + 1]) +
-                                                            __uint_as_float(cw[h] & 0xFFFF0000u));
+            for (int i = 0; i < kEpiCols / 2; ++i) {
+              const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+              const float s0 = g0 / (1.0f + __expf(-g0)), s1 = g1 / (1.0f + __expf(-g1));
+              __nv_bfloat162 bv =
+                  __floats2bfloat162_rn(s0 * __uint_as_float(up[2 * i]), s1 * __uint_as_float(up[2 * i + 1]));
               packed[i] = *reinterpret_cast<uint32_t*>(&bv);
             }
+            store_chunk(col0, packed);
           }
-          store_chunk(col0, packed);
         }
-      }
+      } else {
+#pragma unroll
+        for (int j = 0; j < kChunks; ++j) {
+          const int col0 = colw + j * kEpiCols;
+          if (j < nch_w && vr > 0 && col0 < a.n) {
+            uint32_t acc[kEpiCols];
+            DG_CHECK(((t_row & 0xFFFF) + j * kEpiCols + kEpiCols <= (uint32_t)kTmemCols) &&
+                         ((t_row >> 16) & 0xFFFF) == (uint32_t)(q * 32) + (tmem_base >> 16) && (warp & 3) == q,
+                     8);
+            tc_ld_32x32b_x32(t_row + j * kEpiCols, acc);
+            if (load_c) stage_c(creg[j]);
+            tc_wait_ld_regs(acc);
+            uint32_t packed[kEpiCols / 2];
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const uint4 c4 = load_c ? *reinterpret_cast<const uint4*>(stg + lane * 64 + ((v ^ ((lane >> 1) & 3)) * 16))
+                                      : make_uint4(0u, 0u, 0u, 0u);
+              const uint32_t cw[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const int i = 4 * v + h;
+                __nv_bfloat162 bv = __floats2bfloat162_rn(__uint_as_float(acc[2 * i]) + __uint_as_float(cw[h] << 16),
+                                                          __uint_as_float(acc[2 * i + 1]) +
+                                                              __uint_as_float(cw[h] & 0xFFFF0000u));
+                packed[i] = *reinterpret_cast<uint32_t*>(&bv);
+              }
+            }
+            store_chunk(col0, packed);
+          }
+        }
+      }  // plain epilogue
       tc_fence_before();
       __syncwarp();
       if (lane == 0) release_acc(buf);

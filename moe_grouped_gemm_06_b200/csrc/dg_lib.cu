@@ -318,11 +318,11 @@ float* workspace(size_t bytes, cudaStream_t s) {
 
 // ------------------------------------------------------------ launches
 
-template <int BN, bool FP4, int LAYOUT, int CTAS>
+template <int BN, bool FP4, int LAYOUT, int CTAS, int EPI = dg::kEpiPlain>
 dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td, const CUtensorMap& tsfa,
                       const CUtensorMap& tsfb, const dg::GemmArgs& args, int grid, cudaStream_t s) {
   using C = dg::Cfg<BN, FP4, CTAS>;
-  auto kern = dg::gemm_kernel<BN, FP4, LAYOUT, CTAS>;
+  auto kern = dg::gemm_kernel<BN, FP4, LAYOUT, CTAS, EPI>;
   static std::atomic<uint64_t> attr_set_mask{0};  // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
@@ -339,13 +339,21 @@ dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
   return DG_OK;
 }
 
-template <bool FP4, int LAYOUT>
+template <bool FP4, int LAYOUT, int EPI = dg::kEpiPlain>
 dg_status dispatch(int bn, int ctas, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
                    const CUtensorMap& tsfa, const CUtensorMap& tsfb, const dg::GemmArgs& args, int grid,
                    cudaStream_t s) {
   // CTA-pair (cta_group::2) kernels are not launched: on B200 they stopped
   // with "illegal instruction" and the cause is not yet known.
   if (ctas != 1) return DG_ERR_UNSUPPORTED;
+  if constexpr (EPI == dg::kEpiSwiGlu) {
+    // SwiGLU tiles hold whole (64 gate, 64 up) row blocks: widths 128, 256
+    switch (bn) {
+      case 128: return launch_gemm<128, FP4, LAYOUT, 1, EPI>(ta, tb, td, tsfa, tsfb, args, grid, s);
+      case 256: return launch_gemm<256, FP4, LAYOUT, 1, EPI>(ta, tb, td, tsfa, tsfb, args, grid, s);
+      default: return DG_ERR_UNSUPPORTED;
+    }
+  }
   switch (bn) {
     case 64: return launch_gemm<64, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
     case 128: return launch_gemm<128, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
@@ -376,7 +384,7 @@ struct Problem {
 // caller-provided device buffer instead of the per-stream workspace, and the
 // planner only considers plans that fit in fixed_ws_bytes (whole tiles
 // always do).
-template <bool FP4, int LAYOUT>
+template <bool FP4, int LAYOUT, int EPI = dg::kEpiPlain>
 dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, size_t fixed_ws_bytes = 0) {
   const int sms = num_sms();
   if (sms <= 0) return DG_ERR_CUDA;
@@ -385,6 +393,8 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
   if (LAYOUT == dg::kMasked) {
     const int em = p.expected_m > 0 ? std::min(p.expected_m, p.rows) : p.rows;
     plan = plan_gemm((long long)p.groups * ceil_div(em, dg::kBM), p.n, p.k, sms, false);
+    if (EPI == dg::kEpiSwiGlu && plan.bn != 128 && plan.bn != 256 && !forced_block_n())
+      plan.bn = plan.bn > 192 ? 256 : 128;  // SwiGLU tiles hold whole gate/up block pairs
     plan.grid = (int)std::min<long long>((long long)p.groups * m_blocks * ceil_div(p.n, plan.bn), sms);
   } else {
     plan = plan_gemm(m_blocks, p.n, p.k, sms, LAYOUT == dg::kDense, fixed_ws != nullptr ? fixed_ws_bytes : 0, FP4);
@@ -400,6 +410,7 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
   args.masked_m = p.masked_m;
   args.rows = p.rows;
   args.n = p.n;
+  args.d_cols = (EPI == dg::kEpiSwiGlu) ? p.n / 2 : p.n;
   args.k = p.k;
   args.num_groups = p.groups;
   args.num_m_blocks = (int)(plan.ctas == 2 ? ceil_div(p.rows, 2 * dg::kBM) : m_blocks);
@@ -456,8 +467,8 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
     ok = ok && make_map(&tsfb, CU_TENSOR_MAP_DATA_TYPE_INT32, p.sfb, 128, rows_b, 1, 512, rows_b * 512, 128, 1,
                         CU_TENSOR_MAP_SWIZZLE_NONE);
   }
-  ok = ok && make_map(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.d, p.n, p.rows, ga, (uint64_t)p.n * 2,
-                      (uint64_t)p.rows * p.n * 2, dg::kEpiCols, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+  ok = ok && make_map(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.d, args.d_cols, p.rows, ga, (uint64_t)args.d_cols * 2,
+                      (uint64_t)p.rows * args.d_cols * 2, dg::kEpiCols, 32, CU_TENSOR_MAP_SWIZZLE_64B);
   if (!ok) return DG_ERR_CUDA;
 
   if (log_enabled())
@@ -467,7 +478,7 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
                  LAYOUT, (int)FP4, p.rows, p.n, p.k, p.groups, plan.bn, plan.dp_tiles, plan.sk_tiles, plan.sk_split,
                  plan.max_seg, plan.grid, plan.cost);
 
-  dg_status st = dispatch<FP4, LAYOUT>(plan.bn, plan.ctas, ta, tb, td, tsfa, tsfb, args, plan.grid, s);
+  dg_status st = dispatch<FP4, LAYOUT, EPI>(plan.bn, plan.ctas, ta, tb, td, tsfa, tsfb, args, plan.grid, s);
   if (st != DG_OK || plan.sk_tiles == 0) return st;
 
   dg::SkReduceArgs r{};
@@ -604,15 +615,44 @@ dg_status dg_m_grouped_fp8_fp4_gemm_nt_contiguous(const void* a, const int32_t* 
   return contiguous_impl(true, a, sfa, b, sfb, c, d, m_indices, m_total, n, k, num_groups, stream);
 }
 
-dg_status dg_m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
-                                          void* d, const int32_t* masked_m, int num_groups, int max_m, int n, int k,
-                                          int expected_m, void* stream) {
+static dg_status masked_impl(bool fp4, bool swiglu, const void* a, const int32_t* sfa, const void* b,
+                             const int32_t* sfb, void* d, const int32_t* masked_m, int num_groups, int max_m, int n,
+                             int k, int expected_m, void* stream) {
   if (num_groups <= 0 || num_groups > dg::kMaxMaskedGroups || max_m <= 0 || !masked_m || expected_m < 0)
     return DG_ERR_INVALID_ARG;
+  if (swiglu && n % (2 * dg::kSwiGluBlock) != 0) return DG_ERR_INVALID_ARG;
   dg_status st = check_common(a, sfa, b, sfb, nullptr, d, n, k);
   if (st != DG_OK) return st;
   Problem p{a, sfa, b, sfb, nullptr, d, nullptr, masked_m, max_m, n, k, num_groups, expected_m};
-  return run_gemm<false, dg::kMasked>(p, static_cast<cudaStream_t>(stream));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (swiglu)
+    return fp4 ? run_gemm<true, dg::kMasked, dg::kEpiSwiGlu>(p, s) : run_gemm<false, dg::kMasked, dg::kEpiSwiGlu>(p, s);
+  return fp4 ? run_gemm<true, dg::kMasked>(p, s) : run_gemm<false, dg::kMasked>(p, s);
+}
+
+dg_status dg_m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                                          void* d, const int32_t* masked_m, int num_groups, int max_m, int n, int k,
+                                          int expected_m, void* stream) {
+  return masked_impl(false, false, a, sfa, b, sfb, d, masked_m, num_groups, max_m, n, k, expected_m, stream);
+}
+
+dg_status dg_m_grouped_fp8_fp4_gemm_nt_masked(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                                              void* d, const int32_t* masked_m, int num_groups, int max_m, int n,
+                                              int k, int expected_m, void* stream) {
+  return masked_impl(true, false, a, sfa, b, sfb, d, masked_m, num_groups, max_m, n, k, expected_m, stream);
+}
+
+dg_status dg_m_grouped_fp8_gemm_nt_masked_swiglu(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                                                 void* d, const int32_t* masked_m, int num_groups, int max_m, int n,
+                                                 int k, int expected_m, void* stream) {
+  return masked_impl(false, true, a, sfa, b, sfb, d, masked_m, num_groups, max_m, n, k, expected_m, stream);
+}
+
+dg_status dg_m_grouped_fp8_fp4_gemm_nt_masked_swiglu(const void* a, const int32_t* sfa, const void* b,
+                                                     const int32_t* sfb, void* d, const int32_t* masked_m,
+                                                     int num_groups, int max_m, int n, int k, int expected_m,
+                                                     void* stream) {
+  return masked_impl(true, true, a, sfa, b, sfb, d, masked_m, num_groups, max_m, n, k, expected_m, stream);
 }
 
 dg_status dg_quantize_fp8(const float* x, int rows, int cols, int block_rows, uint8_t* q, uint8_t* sf,

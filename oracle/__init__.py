@@ -16,7 +16,9 @@ Sources (page title, section):
     section 五 "使用方法": D = C + A @ B, NT layout, SM100 packed UE8M0 scale
     factors, M-grouped contiguous and masked layouts.
   * "DeepSeek 发布 DeepGEMM 重大更新" (linlog.top), section "FP4 精度支持":
-    FP8 x FP4 GEMM, UE8M0 scales packed 4 per int32.
+    FP8 x FP4 GEMM, UE8M0 scales packed 4 per int32; its Mega MoE section and
+    "DeepGEMM：FP8 GEMM 与 Mega-MoE" (charles2530.github.io): each expert runs
+    linear1 -> SwiGLU -> linear2 (swiglu_interleaved below).
 
 Every function is pinned by a ``-m "not gpu"`` test in ``tests/test_oracle.py``
 against something other than itself (ml_dtypes code tables, numpy float64
@@ -208,3 +210,28 @@ def gemm_masked(a, sfa, b, sfb, masked_m, b_fp4=False, out=None) -> np.ndarray:
     _load().or_gemm_masked(_p(a), _p(sfa), _p(b), _p(sfb), ctypes.c_int(fp4), _p(mm),
                            I64(G), I64(max_m), I64(N), I64(K), _p(res))
     return res
+
+
+SWIGLU_BLOCK = 64
+
+
+def silu(x) -> np.ndarray:
+    """silu(x) = x / (1 + exp(-x)) = x * sigmoid(x), in float64."""
+    x = np.asarray(x, np.float64)
+    with np.errstate(over="ignore"):
+        return x / (1.0 + np.exp(-x))
+
+
+def swiglu_interleaved(g, block: int = SWIGLU_BLOCK) -> np.ndarray:
+    """SwiGLU of a linear1 output whose columns hold gate and up projections
+    interleaved in blocks: columns [2jb, 2jb + b) are gate columns jb.., the
+    next b the matching up columns.  out[..., jb + i] = silu(g[..., 2jb + i])
+    * g[..., 2jb + b + i]; the last axis halves.  float64 in, float64 out
+    (the library rounds this once to bf16)."""
+    g = np.asarray(g, np.float64)
+    n = g.shape[-1]
+    if n % (2 * block):
+        raise ValueError("columns must be a multiple of 2 * block")
+    blocks = g.reshape(g.shape[:-1] + (n // (2 * block), 2, block))
+    out = silu(blocks[..., 0, :]) * blocks[..., 1, :]
+    return out.reshape(g.shape[:-1] + (n // 2,))

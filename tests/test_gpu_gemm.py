@@ -340,6 +340,75 @@ def test_masked_matches_oracle_and_leaves_rows(dg):
             check_close(dd[g, :v], ref[g, :v], f"masked group {g}")
 
 
+def _masked_fp4_case(seed, G, max_m, N, K, masked_m):
+    qa, ea, sfa, _, _, _ = _masked_case(seed, G, max_m, N, K, masked_m)
+    qb, eb, sfb = quantize_groups_b(seed + 2000, G, N, K, fp4=True)
+    return qa, ea, sfa, qb, eb, sfb
+
+
+def test_masked_fp4_matches_oracle(dg):
+    G, max_m, N, K = 3, 256, 384, 512
+    mm = np.array([5, 256, 130], np.int32)
+    qa, ea, sfa, qb, eb, sfb = _masked_fp4_case(5700, G, max_m, N, K, mm)
+    d = torch.full((G, max_m, N), SENTINEL, dtype=torch.int16, device="cuda")
+    dg.dg_m_grouped_fp8_fp4_gemm_nt_masked(dev(qa), dev(sfa), dev(qb), dev(sfb), d, dev(mm), expected_m=128)
+    torch.cuda.synchronize()
+    ref = oracle.gemm_masked(qa, ea, qb, eb, mm, b_fp4=True)
+    got = bf16_dev_to_f64(d)
+    for g in range(G):
+        check_close(got[g, :mm[g]], ref[g, :mm[g]], f"masked fp4 g={g}")
+        assert np.all(host(d).view(np.uint16)[g, mm[g]:] == SENTINEL)
+
+
+@pytest.mark.parametrize("bn", [0, 128, 256])
+@pytest.mark.parametrize("fp4", [False, True])
+def test_masked_swiglu_matches_oracle(dg, fp4, bn):
+    # linear1 with SwiGLU in the epilogue: B rows are gate/up blocks of 64,
+    # D has half the GEMM's columns
+    G, max_m, N, K = 3, 256, 512, 512
+    mm = np.array([0, 200, 256], np.int32)
+    if fp4:
+        qa, ea, sfa, qb, eb, sfb = _masked_fp4_case(5800, G, max_m, N, K, mm)
+        fn = dg.dg_m_grouped_fp8_fp4_gemm_nt_masked_swiglu
+    else:
+        qa, ea, sfa, qb, eb, sfb = _masked_case(5800, G, max_m, N, K, mm)
+        fn = dg.dg_m_grouped_fp8_gemm_nt_masked_swiglu
+    d = torch.full((G, max_m, N // 2), SENTINEL, dtype=torch.int16, device="cuda")
+    dg.dg_set_tile_config(bn, 0)
+    try:
+        fn(dev(qa), dev(sfa), dev(qb), dev(sfb), d, dev(mm), expected_m=128)
+        torch.cuda.synchronize()
+    finally:
+        dg.dg_set_tile_config(0, 0)
+    ref = oracle.swiglu_interleaved(oracle.gemm_masked(qa, ea, qb, eb, mm, b_fp4=fp4))
+    got = bf16_dev_to_f64(d)
+    for g in range(G):
+        if mm[g]:
+            check_close(got[g, :mm[g]], ref[g, :mm[g]], f"swiglu fp4={fp4} bn={bn} g={g}")
+        assert np.all(host(d).view(np.uint16)[g, mm[g]:] == SENTINEL)
+
+
+def test_masked_swiglu_rejects_bad_widths(dg):
+    z = torch.zeros(16, dtype=torch.int32, device="cuda")
+    # n not a multiple of 128 (whole gate/up block pairs)
+    st = dg.lib().dg_m_grouped_fp8_gemm_nt_masked_swiglu(_p_(z), _p_(z), _p_(z), _p_(z), _p_(z), _p_(z), 1, 128,
+                                                         192, 128, 0, None)
+    assert st == -1
+    # a forced tile width that cannot hold whole block pairs
+    dg.dg_set_tile_config(192, 0)
+    try:
+        st = dg.lib().dg_m_grouped_fp8_gemm_nt_masked_swiglu(_p_(z), _p_(z), _p_(z), _p_(z), _p_(z), _p_(z), 1,
+                                                             128, 256, 128, 0, None)
+    finally:
+        dg.dg_set_tile_config(0, 0)
+    assert st == -2
+
+
+def _p_(t):
+    import ctypes
+    return ctypes.c_void_p(t.data_ptr())
+
+
 def test_masked_decode_replays_from_a_cuda_graph(dg):
     # The masked call reads masked_m on the device and allocates nothing, so
     # one captured launch serves every step of a decode loop: the counts are

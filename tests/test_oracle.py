@@ -364,3 +364,47 @@ def test_contiguous_fp4_equals_per_group_dense():
     for g in range(G):
         sel = np.nonzero(mi == g)[0]
         assert np.array_equal(d[sel], oracle.gemm(a[sel], sfa[sel], b[g], sfb[g], b_fp4=True))
+
+
+# ------------------------------------------------------------------ SwiGLU
+
+def test_silu_closed_forms():
+    # silu(x) = x * sigmoid(x): silu(0) = 0, silu(+-1) = +-1 / (1 + e^-+1),
+    # silu(x) -> x for large x and -> 0 from below for very negative x
+    e = 2.718281828459045
+    got = oracle.silu(np.array([0.0, 1.0, -1.0, 40.0, -40.0, -800.0]))
+    assert got[0] == 0.0
+    assert abs(got[1] - 1.0 / (1.0 + 1.0 / e)) < 1e-15
+    assert abs(got[2] + 1.0 / (1.0 + e)) < 1e-15
+    assert abs(got[3] - 40.0) < 1e-12
+    assert -1e-15 < got[4] < 0.0
+    assert got[5] == 0.0 or (got[5] < 0.0 and got[5] > -1e-300)
+
+
+def test_swiglu_interleaved_picks_gate_and_up_columns():
+    # columns 0..255 hold their own index: gate blocks are columns 0-63 and
+    # 128-191, up blocks 64-127 and 192-255, so output j < 64 is
+    # silu(j) * (j + 64) and output 64 + i is silu(128 + i) * (192 + i)
+    g = np.arange(256, dtype=np.float64)[None, :] / 64.0
+    out = oracle.swiglu_interleaved(g)
+    assert out.shape == (1, 128)
+    for j in (0, 5, 63):
+        x, u = j / 64.0, (j + 64) / 64.0
+        assert abs(out[0, j] - x / (1 + np.exp(-x)) * u) < 1e-15
+    for i in (0, 6, 63):
+        x, u = (128 + i) / 64.0, (192 + i) / 64.0
+        assert abs(out[0, 64 + i] - x / (1 + np.exp(-x)) * u) < 1e-15
+    with pytest.raises(ValueError):
+        oracle.swiglu_interleaved(np.zeros((2, 96)))
+
+
+def test_swiglu_of_a_gemm_equals_gemm_of_the_deinterleaved_halves():
+    # the interleaving is a row permutation of B: computing the gate and up
+    # products as two separate GEMMs and combining them gives the same result
+    rng = np.random.default_rng(3)
+    qa, ea = oracle.quantize_fp8(rng.standard_normal((5, 256)).astype(np.float32), 1)
+    qb, eb = oracle.quantize_fp8(rng.standard_normal((256, 256)).astype(np.float32), 128)
+    g = oracle.gemm(qa, ea, qb, eb)
+    gate = np.concatenate([g[:, 0:64], g[:, 128:192]], axis=1)
+    up = np.concatenate([g[:, 64:128], g[:, 192:256]], axis=1)
+    assert np.array_equal(oracle.swiglu_interleaved(g), gate / (1 + np.exp(-gate)) * up)
