@@ -57,7 +57,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--shape", default=None, help="run one M,N,K shape instead of the sweep")
-    ap.add_argument("--workload", default="dense", choices=["dense", "contiguous", "masked", "fp4", "moe_decode_fp4"],
+    ap.add_argument("--workload", default="dense",
+                    choices=["dense", "contiguous", "masked", "fp4", "moe_decode_fp4", "bf16"],
                     help="dense: the DeepSeek-V3 dense sweep (default); contiguous / masked / fp4: the "
                          "M-grouped prefill, masked decode and FP8 x FP4 cases, one JSON line each")
     ap.add_argument("--graph", action="store_true",
@@ -309,6 +310,18 @@ def grouped_cases(dg, torch, workload, gen, seed):
                           (lambda a=a2, sfa=sfa2, d=out, t=t_mm, em=em:
                            dg.dg_m_grouped_fp8_fp4_gemm_nt_masked(a, sfa, b2, sfb2, d, t, expected_m=em)),
                           2.0 * valid * 7168 * 2048, by2))
+    elif workload == "bf16":
+        # dense bf16 at the M = 4096 sweep shapes, with cuBLAS (torch.matmul)
+        # on the same operands as a library reference
+        for (n, k) in DENSE_NK:
+            m = 4096
+            a = torch.randn((m, k), generator=gen, device="cuda", dtype=torch.float32).to(torch.bfloat16)
+            b = torch.randn((n, k), generator=gen, device="cuda", dtype=torch.float32).to(torch.bfloat16)
+            d = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+            d_ref = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+            cases.append((f"bf16 M={m} N={n} K={k}", (lambda a=a, b=b, d=d: dg.dg_bf16_gemm_nt(a, b, None, d)),
+                          2.0 * m * n * k, 2 * (m * k + n * k + m * n),
+                          (lambda a=a, b=b, d_ref=d_ref: torch.matmul(a, b.t(), out=d_ref))))
     elif workload == "fp4":
         for (n, k) in GROUPED_NK:
             m = 4096
@@ -352,6 +365,9 @@ def run_grouped(args, dg, torch, rank, world, use_dist, local_rank):
     flush_rd = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
     stream = torch.cuda.current_stream()
 
+    refs = [c[4] if len(c) > 4 else None for c in cases]
+    cases = [c[:4] for c in cases]
+
     def step(events):
         torch.cuda._sleep(HOLD_CYCLES)
         for i, (_, call, _, _) in enumerate(cases):
@@ -385,23 +401,49 @@ def run_grouped(args, dg, torch, rank, world, use_dist, local_rank):
     assert err == 0, f"device error during timing: {dg.status_string(err)} ({err})"
     ms = [sum(events[s_][i][0].elapsed_time(events[s_][i][1]) for s_ in range(args.steps)) / args.steps
           for i in range(len(cases))]
+    # library references (cuBLAS for bf16), timed the same way, after ours
+    ref_ms = [None] * len(cases)
+    if any(r is not None for r in refs):
+        rev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in cases]
+               for _ in range(args.steps)]
+        for s_ in range(-max(args.warmup, 1), args.steps):
+            torch.cuda._sleep(HOLD_CYCLES)
+            for i, r in enumerate(refs):
+                if r is None:
+                    continue
+                flush.zero_()
+                flush_rd.max()
+                if s_ >= 0:
+                    rev[s_][i][0].record(stream)
+                r()
+                if s_ >= 0:
+                    rev[s_][i][1].record(stream)
+        torch.cuda.synchronize()
+        ref_ms = [sum(rev[s_][i][0].elapsed_time(rev[s_][i][1]) for s_ in range(args.steps)) / args.steps
+                  if refs[i] is not None else None for i in range(len(cases))]
     t = torch.tensor([sum(ms)], dtype=torch.float64, device="cuda")
     if use_dist:
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     peaks, peak_kind = load_peaks()
     fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
     hbm = peaks["hbm_gbs"]
-    ridge = fp8_peak * 1e12 / (hbm * 1e9)
+    tensor_peak = peaks["bf16_tflops"] if args.workload == "bf16" else fp8_peak
+    ridge = tensor_peak * 1e12 / (hbm * 1e9)
     per_case = []
     for (name, _, f, by), m_ in zip(cases, ms):
         tf, gbs = f / (m_ * 1e-3) / 1e12, by / (m_ * 1e-3) / 1e9
         bound = "tensor" if f / by >= ridge else "hbm"
-        per_case.append({"case": name, "us": round(m_ * 1e3, 2), "tflops": round(tf, 1), "gbs": round(gbs, 1),
-                         "bound": bound, "frac": round(tf / fp8_peak if bound == "tensor" else gbs / hbm, 4)})
+        entry = {"case": name, "us": round(m_ * 1e3, 2), "tflops": round(tf, 1), "gbs": round(gbs, 1),
+                 "bound": bound, "frac": round(tf / tensor_peak if bound == "tensor" else gbs / hbm, 4)}
+        r_ms = ref_ms[len(per_case)]
+        if r_ms is not None:
+            entry["cublas_us"] = round(r_ms * 1e3, 2)
+            entry["cublas_tflops"] = round(f / (r_ms * 1e-3) / 1e12, 1)
+        per_case.append(entry)
     dom = max(range(len(cases)), key=lambda i: ms[i])
     pc = per_case[dom]
     roofline = {"bound": pc["bound"], "achieved": pc["tflops"] if pc["bound"] == "tensor" else pc["gbs"],
-                "peak": round(fp8_peak, 1) if pc["bound"] == "tensor" else hbm,
+                "peak": round(tensor_peak, 1) if pc["bound"] == "tensor" else hbm,
                 "unit": "TFLOP/s" if pc["bound"] == "tensor" else "GB/s", "frac": pc["frac"], "traffic": None,
                 "kernel": f"gemm_kernel on {pc['case']}",
                 "peak_source": f"{peak_kind}: FP8 = bf16 burst {peaks['bf16_tflops']} x {FP8_PER_BF16}; HBM {hbm} GB/s"}

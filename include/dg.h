@@ -184,6 +184,16 @@ dg_status dg_fp8_gemm_nt_noalloc(const void* a, const int32_t* sfa, const void* 
 /* Size in bytes of the fixed scratch array used by dg_fp8_gemm_nt_noalloc. */
 size_t dg_noalloc_scratch_bytes(void);
 
+/* Dense NT BF16 GEMM on the same persistent kernel: D[M,N] = C + A * B^T
+ * with bf16 A [m][k], B [n][k] (row-major, K contiguous), FP32 accumulation
+ * in TMEM (tcgen05 kind::f16), bf16 D; c bf16 [m][n] or NULL, may equal d.
+ * No scale factors.  Requires m >= 0, n > 0 and n % 8 == 0, k > 0 and
+ * k % 64 == 0; 16-byte aligned pointers.  The pages list BF16 GEMM among
+ * the library's kernels ("DeepGEMM：统一高性能张量核心 GEMM 计算库编译与使用
+ * 指南" (zhouruolin.cn), introduction; "DeepGEMM：FP8 GEMM 与 Mega-MoE"
+ * (charles2530.github.io), section 一). */
+dg_status dg_bf16_gemm_nt(const void* a, const void* b, const void* c, void* d, int m, int n, int k, void* stream);
+
 /* FP8 x FP4 dense NT GEMM: as dg_fp8_gemm_nt but
  *   b    e2m1 [n][k/2] (two codes per byte, low nibble = even k)
  *   sfb  sf words of B: R = n, G = k/32 (one UE8M0 code per 1x32 group)

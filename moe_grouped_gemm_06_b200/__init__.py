@@ -20,7 +20,7 @@ import torch
 __all__ = [
     "DGError", "lib", "dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
     "dg_m_grouped_fp8_gemm_nt_masked", "dg_m_grouped_fp8_fp4_gemm_nt_masked",
-    "dg_m_grouped_fp8_gemm_nt_masked_swiglu", "dg_m_grouped_fp8_fp4_gemm_nt_masked_swiglu", "dg_fp8_gemm_nt_noalloc", "dg_noalloc_scratch_bytes", "dg_fp8_fp4_gemm_nt", "dg_m_grouped_fp8_fp4_gemm_nt_contiguous",
+    "dg_m_grouped_fp8_gemm_nt_masked_swiglu", "dg_m_grouped_fp8_fp4_gemm_nt_masked_swiglu", "dg_fp8_gemm_nt_noalloc", "dg_noalloc_scratch_bytes", "dg_fp8_fp4_gemm_nt", "dg_bf16_gemm_nt", "dg_m_grouped_fp8_fp4_gemm_nt_contiguous",
     "dg_quantize_fp8", "dg_quantize_fp4", "dg_pack_sf", "dg_packed_sf_words", "dg_get_num_sms",
     "dg_set_num_sms", "dg_set_pdl", "dg_get_pdl", "dg_set_tile_config", "dg_get_mk_alignment_for_contiguous_layout", "dg_get_last_error",
     "dg_debug_starved_wait", "dg_launch_count", "dg_query_dense_config", "dg_num_tiles", "dg_debug_fastdiv", "dg_shutdown",
@@ -46,6 +46,7 @@ SYMBOLS = {
     "dg_fp8_gemm_nt_noalloc": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _INT, _INT, _INT, _VP]),
     "dg_noalloc_scratch_bytes": (ctypes.c_size_t, []),
     "dg_fp8_fp4_gemm_nt": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _INT, _INT, _INT, _VP]),
+    "dg_bf16_gemm_nt": (_INT, [_VP, _VP, _VP, _VP, _INT, _INT, _INT, _VP]),
     "dg_m_grouped_fp8_fp4_gemm_nt_contiguous": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _I32P, _INT, _INT,
                                                        _INT, _INT, _VP]),
     "dg_quantize_fp8": (_INT, [_VP, _INT, _INT, _INT, _VP, _VP, _VP]),
@@ -148,6 +149,13 @@ def dg_fp8_fp4_gemm_nt(a, sfa, b, sfb, c, d, stream=None) -> None:
     n = b.shape[0]
     _check(lib().dg_fp8_fp4_gemm_nt(_p(a), _p(sfa), _p(b), _p(sfb), _p(c), _p(d), m, n, k, _stream(stream)),
            "dg_fp8_fp4_gemm_nt")
+
+
+def dg_bf16_gemm_nt(a, b, c, d, stream=None) -> None:
+    """a: bf16 [m, k]; b: bf16 [n, k]; c: bf16 [m, n] or None; d: bf16 [m, n]."""
+    m, k = a.shape
+    n = b.shape[0]
+    _check(lib().dg_bf16_gemm_nt(_p(a), _p(b), _p(c), _p(d), m, n, k, _stream(stream)), "dg_bf16_gemm_nt")
 
 
 def dg_m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, c, d, m_indices, stream=None) -> None:

@@ -109,8 +109,13 @@ struct GemmArgs {
   long long sfa_words, sfb_words;      // total packed words (self-check bounds)
 };
 
-template <int BN, bool FP4, int CTAS = 1>
+// BF16 = true: A and B bf16 (kind::f16, no scales); a stage then holds 64
+// K-elements, the same 128-byte rows as 128 e4m3 elements, so the staging,
+// descriptors and schedules are shared with the FP8 kernels.
+template <int BN, bool FP4, int CTAS = 1, bool BF16 = false>
 struct Cfg {
+  static_assert(!(BF16 && FP4), "bf16 A and B");
+  static constexpr int kKPerStage = BF16 ? 64 : kBK;  // K-elements per stage
   // The scale-factor operand of the MMA is addressed in TMEM columns of 32
   // rows (a 128-row chunk spans 4 columns), and that address must be even: a
   // tile starting 32 or 96 rows into a chunk (odd column) faults with a
@@ -122,7 +127,7 @@ struct Cfg {
   static constexpr int kSfbChunks = (kMaxOffRows + BN + 127) / 128;  // 128-row scale chunks a tile can touch
   static constexpr bool kRebase = (BN % 64 != 0);
   static constexpr int kSfrChunks = (BN + 127) / 128;                // re-based chunks (tile rows only)
-  static constexpr int kSfrBytes = kRebase ? kSfrChunks * 512 : 0;
+  static constexpr int kSfrBytes = (kRebase && !BF16) ? kSfrChunks * 512 : 0;
   // FP32 accumulator buffers in TMEM: three of 128 columns (BN = 128), two at
   // columns 0 and 256 (BN = 192), one (BN = 256); scale factors after them.
   static constexpr int kAccBufs = (BN <= 128) ? 3 : (BN <= 240 ? 2 : 1);
@@ -130,8 +135,8 @@ struct Cfg {
   static constexpr int kBRows = BN / CTAS;                   // B rows each CTA of a pair loads
   static constexpr int kBBytes = kBRows * kBK;               // smem bytes (FP4 lands padded to 1 B/elt)
   static constexpr int kBTxBytes = FP4 ? kBBytes / 2 : kBBytes;  // bytes the TMA copy reports (packed)
-  static constexpr int kSfaBytes = 512;
-  static constexpr int kSfbBytes = kSfbChunks * 512;
+  static constexpr int kSfaBytes = BF16 ? 0 : 512;
+  static constexpr int kSfbBytes = BF16 ? 0 : kSfbChunks * 512;
   static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes + kSfrBytes;
   static constexpr int kEpiBytes = kEpiWarps * 32 * 64;        // one 32 x 64 B staging box per epilogue warp
   static constexpr int kMaskBytes = ((kMaxMaskedGroups + 1) * 4 + 15) / 16 * 16;
@@ -149,8 +154,13 @@ struct Cfg {
   // Instruction descriptor of kind::mxf8f6f4 with block scaling: A = E4M3,
   // B = E4M3 (0) or E2M1 (5), both K-major, UE8M0 scales, M = 128 per CTA
   // (256 for a CTA pair), N = BN.
-  static constexpr uint32_t kIdesc = (0u << 7) | ((FP4 ? 5u : 0u) << 10) | ((uint32_t)(BN >> 3) << 17) |
-                                     (1u << 23) | ((uint32_t)((kBM * CTAS) >> 4) << 24);
+  static constexpr uint32_t kIdescScaled = (0u << 7) | ((FP4 ? 5u : 0u) << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                           (1u << 23) | ((uint32_t)((kBM * CTAS) >> 4) << 24);
+  // kind::f16: FP32 accumulator (bits 4-5 = 1), A and B bf16 (formats 1),
+  // both K-major, N >> 3, M >> 4
+  static constexpr uint32_t kIdescBf16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                         ((uint32_t)((kBM * CTAS) >> 4) << 24);
+  static constexpr uint32_t kIdesc = BF16 ? kIdescBf16 : kIdescScaled;
 };
 
 struct Unit {
@@ -285,14 +295,15 @@ struct WorkIter {
 // CTAS = 2: a cluster of two CTAs computes 256 x BN tiles (dense layout only);
 // tm_sfa / tm_sfb view the packed scale words as rows of 512 bytes so that
 // the peer's scale loads can complete on the leader's barrier.
-template <int BN, bool FP4, int LAYOUT, int CTAS, int EPI = kEpiPlain>
+template <int BN, bool FP4, int LAYOUT, int CTAS, int EPI = kEpiPlain, bool BF16 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_d, const __grid_constant__ CUtensorMap tm_sfa,
                 const __grid_constant__ CUtensorMap tm_sfb, const GemmArgs args) {
   static_assert(CTAS == 1 || (CTAS == 2 && LAYOUT == kDense), "CTA pairs serve the dense layout");
   static_assert(EPI == kEpiPlain || (CTAS == 1 && BN % (2 * kSwiGluBlock) == 0), "SwiGLU tiles hold whole block pairs");
-  using C = Cfg<BN, FP4, CTAS>;
+  using C = Cfg<BN, FP4, CTAS, BF16>;
+  static_assert(!BF16 || (CTAS == 1 && EPI == kEpiPlain), "bf16: single CTAs, plain epilogue");
   constexpr bool kPair = (CTAS == 2);
   constexpr int kTileM = kBM * CTAS;
   constexpr int S = C::kStages;
@@ -419,8 +430,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          const bool new_sfa = ((kb & 3) == 0) || kb == kb0;
-          const bool new_sfb = FP4 || new_sfa;
+          const bool new_sfa = !BF16 && (((kb & 3) == 0) || kb == kb0);
+          const bool new_sfb = !BF16 && (FP4 || new_sfa);
           uint32_t bytes = C::kABytes + C::kBTxBytes;
           if (new_sfa) bytes += C::kSfaBytes;
           if (new_sfb) bytes += 512u * nchunks;
@@ -451,8 +462,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             continue;
           }
           mbar_arrive_expect_tx(&full[stage], bytes);
-          tma_load_3d(s_a + stage * C::kABytes, &tm_a, &full[stage], kb * kBK, a_row, a_grp);
-          tma_load_3d(s_b + stage * C::kBBytes, &tm_b, &full[stage], kb * kBK, n0, b_grp);
+          tma_load_3d(s_a + stage * C::kABytes, &tm_a, &full[stage], kb * C::kKPerStage, a_row, a_grp);
+          tma_load_3d(s_b + stage * C::kBBytes, &tm_b, &full[stage], kb * C::kKPerStage, n0, b_grp);
           if (new_sfa) {
             const int32_t* src = sfa_g + ((long long)(kb >> 2) * a.sfa_chunks + u.mb) * 128;
             if (DG_CHECK(src >= a.sfa && src + 128 <= a.sfa + a.sfa_words &&
@@ -526,6 +537,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
+          if constexpr (BF16) {
+            // 4 x (M=128, N=BN, K=16) per stage, 32 bytes of each row apart
+            const uint64_t adesc = sdesc_k_sw128(s_a + stage * C::kABytes);
+            const uint64_t bdesc = sdesc_k_sw128(s_b + stage * C::kBBytes);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+              tc_mma_f16(d_t, adesc + (uint64_t)(ks * 2), bdesc + (uint64_t)(ks * 2), C::kIdesc,
+                         (kb > kb0 || ks > 0) ? 1u : 0u);
+            tc_commit(&empty[stage]);
+            if (++stage == S) {
+              stage = 0;
+              phase ^= 1;
+            }
+            continue;
+          }
           const bool new_sfa = ((kb & 3) == 0) || kb == kb0;
           const bool new_sfb = FP4 || new_sfa;
           const uint8_t* sfb_src = s_sfb + stage * C::kSfbBytes;

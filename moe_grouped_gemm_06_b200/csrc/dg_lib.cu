@@ -318,11 +318,11 @@ float* workspace(size_t bytes, cudaStream_t s) {
 
 // ------------------------------------------------------------ launches
 
-template <int BN, bool FP4, int LAYOUT, int CTAS, int EPI = dg::kEpiPlain>
+template <int BN, bool FP4, int LAYOUT, int CTAS, int EPI = dg::kEpiPlain, bool BF16 = false>
 dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td, const CUtensorMap& tsfa,
                       const CUtensorMap& tsfb, const dg::GemmArgs& args, int grid, cudaStream_t s) {
-  using C = dg::Cfg<BN, FP4, CTAS>;
-  auto kern = dg::gemm_kernel<BN, FP4, LAYOUT, CTAS, EPI>;
+  using C = dg::Cfg<BN, FP4, CTAS, BF16>;
+  auto kern = dg::gemm_kernel<BN, FP4, LAYOUT, CTAS, EPI, BF16>;
   static std::atomic<uint64_t> attr_set_mask{0};  // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
@@ -339,14 +339,23 @@ dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
   return DG_OK;
 }
 
-template <bool FP4, int LAYOUT, int EPI = dg::kEpiPlain>
+template <bool FP4, int LAYOUT, int EPI = dg::kEpiPlain, bool BF16 = false>
 dg_status dispatch(int bn, int ctas, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
                    const CUtensorMap& tsfa, const CUtensorMap& tsfb, const dg::GemmArgs& args, int grid,
                    cudaStream_t s) {
   // CTA-pair (cta_group::2) kernels are not launched: on B200 they stopped
   // with "illegal instruction" and the cause is not yet known.
   if (ctas != 1) return DG_ERR_UNSUPPORTED;
-  if constexpr (EPI == dg::kEpiSwiGlu) {
+  if constexpr (BF16) {
+    // bf16: dense tiles of the widths the heuristic picks
+    switch (bn) {
+      case 64: return launch_gemm<64, false, LAYOUT, 1, EPI, true>(ta, tb, td, tsfa, tsfb, args, grid, s);
+      case 128: return launch_gemm<128, false, LAYOUT, 1, EPI, true>(ta, tb, td, tsfa, tsfb, args, grid, s);
+      case 192: return launch_gemm<192, false, LAYOUT, 1, EPI, true>(ta, tb, td, tsfa, tsfb, args, grid, s);
+      case 256: return launch_gemm<256, false, LAYOUT, 1, EPI, true>(ta, tb, td, tsfa, tsfb, args, grid, s);
+      default: return DG_ERR_UNSUPPORTED;
+    }
+  } else if constexpr (EPI == dg::kEpiSwiGlu) {
     // SwiGLU tiles hold whole (64 gate, 64 up) row blocks: widths 128, 256
     switch (bn) {
       case 128: return launch_gemm<128, FP4, LAYOUT, 1, EPI>(ta, tb, td, tsfa, tsfb, args, grid, s);
@@ -384,8 +393,11 @@ struct Problem {
 // caller-provided device buffer instead of the per-stream workspace, and the
 // planner only considers plans that fit in fixed_ws_bytes (whole tiles
 // always do).
-template <bool FP4, int LAYOUT, int EPI = dg::kEpiPlain>
+template <bool FP4, int LAYOUT, int EPI = dg::kEpiPlain, bool BF16 = false>
 dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, size_t fixed_ws_bytes = 0) {
+  // a bf16 stage covers 64 K-elements in the time an e4m3 stage covers 128:
+  // the planner sees bf16 as an e4m3 problem of twice the K
+  const int k_plan = BF16 ? 2 * p.k : p.k;
   const int sms = num_sms();
   if (sms <= 0) return DG_ERR_CUDA;
   const long long m_blocks = ceil_div(p.rows, dg::kBM);
@@ -397,7 +409,7 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
       plan.bn = plan.bn > 192 ? 256 : 128;  // SwiGLU tiles hold whole gate/up block pairs
     plan.grid = (int)std::min<long long>((long long)p.groups * m_blocks * ceil_div(p.n, plan.bn), sms);
   } else {
-    plan = plan_gemm(m_blocks, p.n, p.k, sms, LAYOUT == dg::kDense, fixed_ws != nullptr ? fixed_ws_bytes : 0, FP4);
+    plan = plan_gemm(m_blocks, p.n, k_plan, sms, LAYOUT == dg::kDense, fixed_ws != nullptr ? fixed_ws_bytes : 0, FP4);
   }
 
   dg::GemmArgs args{};
@@ -415,7 +427,7 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
   args.num_groups = p.groups;
   args.num_m_blocks = (int)(plan.ctas == 2 ? ceil_div(p.rows, 2 * dg::kBM) : m_blocks);
   args.num_n_blocks = (int)ceil_div(p.n, plan.bn);
-  args.kb_total = p.k / 128;
+  args.kb_total = p.k / (BF16 ? 64 : 128);
   args.dp_tiles = (int)plan.dp_tiles;
   args.sk_tiles = plan.sk_tiles;
   args.max_seg = plan.max_seg;
@@ -447,9 +459,18 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
   const int ga = (LAYOUT == dg::kMasked) ? p.groups : 1;
   const int gb = (LAYOUT == dg::kDense) ? 1 : p.groups;
   CUtensorMap ta, tb, td;
-  bool ok = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.a, p.k, p.rows, ga, (uint64_t)p.k,
-                     (uint64_t)p.rows * p.k, 128, dg::kBM, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (FP4)
+  bool ok;
+  if (BF16) {
+    ok = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.a, p.k, p.rows, ga, (uint64_t)p.k * 2,
+                  (uint64_t)p.rows * p.k * 2, 64, dg::kBM, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.b, p.k, p.n, gb, (uint64_t)p.k * 2,
+                        (uint64_t)p.n * p.k * 2, 64, plan.bn, CU_TENSOR_MAP_SWIZZLE_128B);
+  } else {
+    ok = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.a, p.k, p.rows, ga, (uint64_t)p.k, (uint64_t)p.rows * p.k,
+                  128, dg::kBM, CU_TENSOR_MAP_SWIZZLE_128B);
+  }
+  if (BF16) {
+  } else if (FP4)
     ok = ok && make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, p.b, p.k, p.n, gb, (uint64_t)p.k / 2,
                         (uint64_t)p.n * p.k / 2, 128, plan.bn / plan.ctas, CU_TENSOR_MAP_SWIZZLE_128B);
   else
@@ -478,7 +499,7 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
                  LAYOUT, (int)FP4, p.rows, p.n, p.k, p.groups, plan.bn, plan.dp_tiles, plan.sk_tiles, plan.sk_split,
                  plan.max_seg, plan.grid, plan.cost);
 
-  dg_status st = dispatch<FP4, LAYOUT, EPI>(plan.bn, plan.ctas, ta, tb, td, tsfa, tsfb, args, plan.grid, s);
+  dg_status st = dispatch<FP4, LAYOUT, EPI, BF16>(plan.bn, plan.ctas, ta, tb, td, tsfa, tsfb, args, plan.grid, s);
   if (st != DG_OK || plan.sk_tiles == 0) return st;
 
   dg::SkReduceArgs r{};
@@ -578,6 +599,15 @@ dg_status dg_fp8_gemm_nt_noalloc(const void* a, const int32_t* sfa, const void* 
 }
 
 size_t dg_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+dg_status dg_bf16_gemm_nt(const void* a, const void* b, const void* c, void* d, int m, int n, int k, void* stream) {
+  if (m < 0 || !a || !b || !d || !aligned16(a) || !aligned16(b) || !aligned16(d) || (c && !aligned16(c)))
+    return DG_ERR_INVALID_ARG;
+  if (n <= 0 || n % 8 != 0 || k <= 0 || k % 64 != 0) return DG_ERR_INVALID_ARG;
+  if (m == 0) return DG_OK;
+  Problem p{a, nullptr, b, nullptr, c, d, nullptr, nullptr, m, n, k, 1, 0};
+  return run_gemm<false, dg::kDense, dg::kEpiPlain, true>(p, static_cast<cudaStream_t>(stream));
+}
 
 dg_status dg_fp8_fp4_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, const void* c,
                              void* d, int m, int n, int k, void* stream) {

@@ -235,3 +235,20 @@ def swiglu_interleaved(g, block: int = SWIGLU_BLOCK) -> np.ndarray:
     blocks = g.reshape(g.shape[:-1] + (n // (2 * block), 2, block))
     out = silu(blocks[..., 0, :]) * blocks[..., 1, :]
     return out.reshape(g.shape[:-1] + (n // 2,))
+
+
+
+def bf16_to_f64(bits) -> np.ndarray:
+    """bf16 bit patterns (uint16) -> float64: the upper half of an IEEE
+    binary32 (sign, 8 exponent bits, 7 mantissa bits)."""
+    bits = np.asarray(bits, np.uint16)
+    return (bits.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+def gemm_bf16(a_bits, b_bits, c_bits=None) -> np.ndarray:
+    """Plain bf16 GEMM reference D = C + A * B^T in float64 (no scales):
+    a_bits [M, K], b_bits [N, K], c_bits [M, N] or None, bf16 bit patterns."""
+    d = bf16_to_f64(a_bits) @ bf16_to_f64(b_bits).T
+    if c_bits is not None:
+        d = d + bf16_to_f64(c_bits)
+    return d

@@ -236,6 +236,52 @@ def test_dense_full_size_sampled(dg):
             torch.cuda.empty_cache()
 
 
+# ------------------------------------------------------------------ bf16
+
+def _bf16_case(seed, M, N, K, with_c):
+    import ml_dtypes
+    a = synth.normal_f32(seed, (M, K)).astype(ml_dtypes.bfloat16).view(np.uint16)
+    b = synth.normal_f32(seed + 1, (N, K)).astype(ml_dtypes.bfloat16).view(np.uint16)
+    c = synth.normal_bf16_bits(seed + 2, (M, N)) if with_c else None
+    return a, b, c
+
+
+def _run_bf16(dg, a, b, c):
+    M, N = a.shape[0], b.shape[0]
+    d = torch.full((M, N), SENTINEL, dtype=torch.int16, device="cuda")
+    dg.dg_bf16_gemm_nt(dev(a.view(np.int16)), dev(b.view(np.int16)),
+                       dev(c.view(np.int16)) if c is not None else None, d)
+    torch.cuda.synchronize()
+    return bf16_dev_to_f64(d)
+
+
+@pytest.mark.parametrize("M,N,K,with_c", [
+    (128, 512, 1024, False), (200, 328, 192, True), (1100, 520, 512, True), (64, 2112, 7168, True),
+    (3, 64, 64, True)])
+def test_bf16_dense_matches_oracle(dg, M, N, K, with_c):
+    a, b, c = _bf16_case(6000 + M + N, M, N, K, with_c)
+    check_close(_run_bf16(dg, a, b, c), oracle.gemm_bf16(a, b, c), f"bf16 {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("bn,schedule", [(64, 1), (128, 1), (192, 1), (256, 1), (128, 2), (256, 3)])
+def test_bf16_widths_and_shared_tails(dg, bn, schedule):
+    M, N, K = 1100, 1000, 1024
+    a, b, c = _bf16_case(6100 + bn + schedule, M, N, K, True)
+    dg.dg_set_num_sms(7 if schedule > 1 else 0)
+    dg.dg_set_tile_config(bn, schedule)
+    try:
+        got = _run_bf16(dg, a, b, c)
+    finally:
+        dg.dg_set_tile_config(0, 0)
+        dg.dg_set_num_sms(0)
+    check_close(got, oracle.gemm_bf16(a, b, c), f"bf16 bn={bn} schedule={schedule}")
+
+
+def test_bf16_rejects_k_not_multiple_of_64(dg):
+    z = torch.zeros(1024, dtype=torch.int16, device="cuda")
+    assert dg.lib().dg_bf16_gemm_nt(_p_(z), _p_(z), None, _p_(z), 8, 8, 96, None) == -1
+
+
 # ------------------------------------------------------------------ contiguous
 
 def _contiguous_case(seed, G, lo, hi, N, K, fp4=False, with_c=True):

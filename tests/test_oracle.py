@@ -408,3 +408,31 @@ def test_swiglu_of_a_gemm_equals_gemm_of_the_deinterleaved_halves():
     gate = np.concatenate([g[:, 0:64], g[:, 128:192]], axis=1)
     up = np.concatenate([g[:, 64:128], g[:, 192:256]], axis=1)
     assert np.array_equal(oracle.swiglu_interleaved(g), gate / (1 + np.exp(-gate)) * up)
+
+
+# ------------------------------------------------------------------ BF16
+
+def test_bf16_decode_matches_ml_dtypes_on_every_code():
+    codes = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = oracle.bf16_to_f64(codes)
+    want = codes.view(ml_dtypes.bfloat16).astype(np.float64)
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], want[~nan])
+
+
+def test_bf16_gemm_brute_force():
+    rng = np.random.default_rng(11)
+    a = rng.standard_normal((3, 70)).astype(ml_dtypes.bfloat16).view(np.uint16)
+    b = rng.standard_normal((4, 70)).astype(ml_dtypes.bfloat16).view(np.uint16)
+    c = rng.standard_normal((3, 4)).astype(ml_dtypes.bfloat16).view(np.uint16)
+    got = oracle.gemm_bf16(a, b, c)
+    av = a.view(ml_dtypes.bfloat16).astype(float)
+    bv = b.view(ml_dtypes.bfloat16).astype(float)
+    cv = c.view(ml_dtypes.bfloat16).astype(float)
+    for i in range(3):
+        for j in range(4):
+            s = float(cv[i, j])
+            for kk in range(70):
+                s += float(av[i, kk]) * float(bv[j, kk])
+            assert abs(got[i, j] - s) <= 1e-12 * (1 + abs(s))
