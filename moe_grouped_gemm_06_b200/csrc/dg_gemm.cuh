@@ -925,12 +925,11 @@ __global__ void __launch_bounds__(256) sk_reduce_kernel(const SkReduceArgs r) {
   pdl_wait();
   const int q4 = r.bn / 4;
   const int per_tile = kBM * q4;
-  const long long items = (long long)r.sk_tiles * per_tile;
+  const int items = r.sk_tiles * per_tile;  // < 2^31: at most 4 x 148 tiles of 128 x 256
   const long long slot4 = (long long)kBM * r.bn / 4;  // float4s between slots
-  for (long long it = blockIdx.x * (long long)blockDim.x + threadIdx.x; it < items;
-       it += (long long)gridDim.x * blockDim.x) {
-    const int j = (int)(it / per_tile);
-    const int rem = (int)(it - (long long)j * per_tile);
+  for (int it = blockIdx.x * blockDim.x + threadIdx.x; it < items; it += gridDim.x * blockDim.x) {
+    const int j = it / per_tile;
+    const int rem = it - j * per_tile;
     const int lr = rem / q4;
     const int lc = (rem - lr * q4) * 4;
     int mb, nb;
@@ -938,6 +937,9 @@ __global__ void __launch_bounds__(256) sk_reduce_kernel(const SkReduceArgs r) {
     const int row = mb * kBM + lr;
     const int col = nb * r.bn + lc;
     if (row >= r.rows || col >= r.n) continue;
+    // C first, so its load overlaps the slots'
+    uint2 cw = make_uint2(0u, 0u);
+    if (r.c != nullptr) cw = __ldg(reinterpret_cast<const uint2*>(r.c + (long long)row * r.n + col));
     int nseg = r.sk_split;
     if (nseg == 0) {
       const long long x0 = (long long)j * r.kb_total;
@@ -958,13 +960,10 @@ __global__ void __launch_bounds__(256) sk_reduce_kernel(const SkReduceArgs r) {
         acc3 += part[s].w;
       }
     }
-    if (r.c != nullptr) {
-      const uint2 w = __ldg(reinterpret_cast<const uint2*>(r.c + (long long)row * r.n + col));
-      acc0 += __uint_as_float(w.x << 16);
-      acc1 += __uint_as_float(w.x & 0xFFFF0000u);
-      acc2 += __uint_as_float(w.y << 16);
-      acc3 += __uint_as_float(w.y & 0xFFFF0000u);
-    }
+    acc0 += __uint_as_float(cw.x << 16);
+    acc1 += __uint_as_float(cw.x & 0xFFFF0000u);
+    acc2 += __uint_as_float(cw.y << 16);
+    acc3 += __uint_as_float(cw.y & 0xFFFF0000u);
     __nv_bfloat162 lo = __floats2bfloat162_rn(acc0, acc1), hi = __floats2bfloat162_rn(acc2, acc3);
     *reinterpret_cast<uint2*>(r.d + (long long)row * r.n + col) =
         make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));

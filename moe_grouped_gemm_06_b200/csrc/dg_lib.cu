@@ -246,7 +246,8 @@ Plan plan_gemm(long long m_blocks, int n, int k, int sms, bool allow_sk, size_t 
     const long long full_waves = tiles / sms;
     for (long long q = full_waves; q >= std::max(0LL, full_waves - 1); --q) {
       const long long sk = tiles - q * sms;
-      if (sk <= 0 || sk > 4 * (long long)sms) continue;
+      // (the fix-up kernel indexes a shared tile's elements with 32-bit ints)
+      if (sk <= 0 || sk > 4 * (long long)sms || sk * dg::kBM * (bn / 4) >= (1LL << 31)) continue;
       const double shared_reads = q > 0 ? (double)sk * (dg::kBM + bn) * k / 6e6 : 0.0;
       Plan p;
       p.bn = bn;
