@@ -37,8 +37,9 @@ namespace dg {
 
 constexpr int kBM = 128;           // rows of A per tile (= TMEM lanes)
 constexpr int kBK = 128;           // K per pipeline stage (= one scale block)
-constexpr int kThreads = 320;       // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 8;        // 4 TMEM sub-partitions x kEpiParts column parts
+constexpr int kEpiParts = kEpiWarps / 4;
+constexpr int kThreads = 64 + 32 * kEpiWarps;  // warp 0 TMA, warp 1 MMA, the rest epilogue
 constexpr int kEpiCols = 32;       // columns per epilogue store box
 constexpr int kTmemCols = 512;
 constexpr int kMaxMaskedGroups = 1024;
@@ -641,11 +642,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // column half (w-2)/4 of the tile.  All C loads of a tile are issued into
     // registers before waiting for its accumulator, so they overlap the MMAs.
     const int q = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int half = (warp - 2) >> 2;             // column part of this warp (0 .. kEpiParts - 1)
     constexpr int kNch = BN / kEpiCols;           // 32-column chunks of the tile
-    constexpr int kChunks = (kNch + 1) / 2;       // chunks of the first half; the second has kNch - kChunks
-    constexpr int kCols = kChunks * kEpiCols;     // column offset of the second half
-    const int nch_w = half ? (kNch - kChunks) : kChunks;  // chunks of this warp
+    constexpr int kChunks = (kNch + kEpiParts - 1) / kEpiParts;  // chunks per part (the last may have fewer)
+    constexpr int kCols = kChunks * kEpiCols;     // columns between parts
+    const int nch_w = max(0, min(kChunks, kNch - half * kChunks));  // chunks of this warp
     uint8_t* stg = s_epi + (warp - 2) * (32 * 64);
     int local = 0;
     // where this warp releases an accumulator buffer: the leader's barrier
@@ -828,12 +829,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         // chunks, the first half of them for warp half 0.  Output chunk c
         // reads gate chunk 4 (c / 2) + c % 2 and up chunk 4 (c / 2) + 2 + c % 2.
         constexpr int kOutCh = BN / (2 * kEpiCols);
+        constexpr int kOutPer = (kOutCh + kEpiParts - 1) / kEpiParts;
         const uint32_t t_tile = tmem_base + ((uint32_t)(q * 32) << 16) + C::kColAcc + buf * C::kAccStride;
 #pragma unroll
-        for (int e = 0; e < kOutCh / 2; ++e) {
-          const int c = half * (kOutCh / 2) + e;
+        for (int e = 0; e < kOutPer; ++e) {
+          const int c = half * kOutPer + e;
           const int col0 = u.nb * (BN / 2) + c * kEpiCols;
-          if (vr > 0 && col0 < a.d_cols) {
+          if (c < kOutCh && vr > 0 && col0 < a.d_cols) {
             const int gch = 4 * (c >> 1) + (c & 1);
             uint32_t g[kEpiCols], up[kEpiCols];
             DG_CHECK(((t_tile & 0xFFFF) + (gch + 2) * kEpiCols + kEpiCols <= (uint32_t)kTmemCols), 8);
