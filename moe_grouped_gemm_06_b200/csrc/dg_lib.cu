@@ -144,15 +144,18 @@ long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
 // FP4 B (per_kb_fp4) is staged from half the bytes, which helps wide tiles,
 // but every K-block needs its own scale-factor copy into TMEM ahead of its
 // MMAs (1x32 scales), which costs narrow tiles.
+// BF16 (per_kb_bf16, per 64-element K-block) runs a 192-wide MMA at the
+// rate of its width, where e4m3 pays nearly the 256-wide cost for it.
 struct WidthCost {
   int bn;
   double per_kb, per_tile, epilogue;
   bool automatic;
-  double per_kb_fp4;
+  double per_kb_fp4, per_kb_bf16;
 };
 constexpr WidthCost kWidthCosts[] = {
-    {64, 0.19, 1.5, 1.6, true, 0.21},      {128, 0.2305, 1.9, 2.94, true, 0.264}, {160, 0.32, 2.4, 3.6, false, 0.33}, {192, 0.368, 1.6, 3.97, true, 0.345},
-    {224, 0.41, 3.0, 4.6, false, 0.36},    {256, 0.4236, 4.34, 0.0, true, 0.343},
+    {64, 0.19, 1.5, 1.6, true, 0.21, 0.13},      {128, 0.2305, 1.9, 2.94, true, 0.264, 0.213},
+    {160, 0.32, 2.4, 3.6, false, 0.33, 0.26},    {192, 0.368, 1.6, 3.97, true, 0.345, 0.284},
+    {224, 0.41, 3.0, 4.6, false, 0.36, 0.33},    {256, 0.4236, 4.34, 0.0, true, 0.343, 0.357},
 };
 
 // Tile-configuration override (dg_set_tile_config; initial values from the
@@ -210,7 +213,8 @@ int sk_max_segments(int sk_tiles, int kb, int G) {
 // among plans at the floor the one with the least estimated SM time wins.  Sharing is offered for the dense layout only
 // (allow_sk) and only within ws_cap bytes of workspace (0: no cap).  Ties
 // keep whole tiles.
-Plan plan_gemm(long long m_blocks, int n, int k, int sms, bool allow_sk, size_t ws_cap = 0, bool fp4 = false) {
+Plan plan_gemm(long long m_blocks, int n, int k, int sms, bool allow_sk, size_t ws_cap = 0, bool fp4 = false,
+               bool bf16 = false) {
   Plan best;
   best.cost = 1e300;
   const int kb = k / 128;
@@ -222,6 +226,7 @@ Plan plan_gemm(long long m_blocks, int n, int k, int sms, bool allow_sk, size_t 
   for (const WidthCost& base : kWidthCosts) {
     WidthCost wc = base;
     if (fp4) wc.per_kb = wc.per_kb_fp4;
+    if (bf16) wc.per_kb = wc.per_kb_bf16;
     const int bn = wc.bn;
     if (forced_block_n() ? bn != forced_block_n() : !wc.automatic) continue;
     // 64-wide tiles double the CTAs of a dense problem of at most two
@@ -410,7 +415,8 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
       plan.bn = plan.bn > 192 ? 256 : 128;  // SwiGLU tiles hold whole gate/up block pairs
     plan.grid = (int)std::min<long long>((long long)p.groups * m_blocks * ceil_div(p.n, plan.bn), sms);
   } else {
-    plan = plan_gemm(m_blocks, p.n, k_plan, sms, LAYOUT == dg::kDense, fixed_ws != nullptr ? fixed_ws_bytes : 0, FP4);
+    plan = plan_gemm(m_blocks, p.n, k_plan, sms, LAYOUT == dg::kDense, fixed_ws != nullptr ? fixed_ws_bytes : 0, FP4,
+                     BF16);
   }
 
   dg::GemmArgs args{};
