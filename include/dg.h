@@ -109,6 +109,49 @@ dg_status dg_m_grouped_fp8_gemm_nt_contiguous(const void* a, const int32_t* sfa,
                                               const int32_t* m_indices, int m_total, int n, int k,
                                               int num_groups, void* stream);
 
+/* M-grouped contiguous FP8 GEMM with B not transposed (NN): as
+ * dg_m_grouped_fp8_gemm_nt_contiguous, D = C + A * B[g] per row, but
+ *   b    e4m3 [num_groups][k][n] row-major (n contiguous: "MN-major")
+ *   sfb  num_groups blocks of sf words, R = n, G = k/128: the 128x128 block
+ *        codes of B[g] (block (k/128, n/128)) expanded per column n, exactly
+ *        as for the NT call's B
+ * Requires n % 16 == 0 as well (the rows of B are n bytes).  Other
+ * arguments, rules and errors as dg_m_grouped_fp8_gemm_nt_contiguous.
+ * Source: zhouruolin.cn guide, section 五 (SM100 takes all of the NT, TN, NN
+ * and TT layouts; m_grouped_fp8_gemm_{nt, nn}_contiguous for the training
+ * forward / prefill). */
+dg_status dg_m_grouped_fp8_gemm_nn_contiguous(const void* a, const int32_t* sfa, const void* b,
+                                              const int32_t* sfb, const void* c, void* d,
+                                              const int32_t* m_indices, int m_total, int n, int k,
+                                              int num_groups, void* stream);
+
+/* K-grouped FP8 GEMM, TN layout (MoE weight gradient): the K axis (tokens)
+ * is cut into num_groups consecutive ranges, group g owning the ks[g] rows
+ * starting at k_g = ks[0] + ... + ks[g-1], and for every group
+ *   D[g] = C[g] + A_g^T * B_g,   A_g = a[k_g .. k_g + ks[g]),  B_g likewise,
+ * i.e. d[g][i][j] = c[g][i][j] + sum_k a[k][i] * b[k][j] with the scales below.
+ *   a    e4m3 [k_total][m] row-major (m contiguous)
+ *   sfa  sf words, R = m, G = k_total/128: one UE8M0 code per (column i of a,
+ *        128-row block of K) -- A quantised 1x128 along K
+ *   b    e4m3 [k_total][n] row-major (n contiguous)
+ *   sfb  sf words, R = n, G = k_total/128: one code per (column j, 128-row
+ *        block of K) -- B quantised 1x128 along K as well (no 128x128 blocks)
+ *   c    bf16 [num_groups][m][n] or NULL (C = 0); may equal d
+ *   d    bf16 [num_groups][m][n]; a group with ks[g] == 0 gets D[g] = C[g] (0)
+ *   ks   int32 [num_groups] on the device: rows of K per group, each a
+ *        multiple of 128 (so no 128-row scale block spans two groups), read
+ *        inside the kernel (graph-capturable); their sum may not exceed k_total
+ * Requires 1 <= num_groups <= 1024, m > 0 and m % 16 == 0, n > 0 and
+ * n % 16 == 0, k_total >= 0 and k_total % 128 == 0.  A ks value that is
+ * negative or not a multiple of 128 counts as 0 and a sum beyond k_total is
+ * cut at k_total, both reported as DG_ERR_BAD_METADATA by dg_get_last_error.
+ * Source: zhouruolin.cn guide, section 五 (k_grouped_fp8_gemm_tn_contiguous,
+ * weight backward grouped along K; SM100 takes the TN layout). */
+dg_status dg_k_grouped_fp8_gemm_tn_contiguous(const void* a, const int32_t* sfa, const void* b,
+                                              const int32_t* sfb, const void* c, void* d,
+                                              const int32_t* ks, int num_groups, int m, int n, int k_total,
+                                              void* stream);
+
 /* M-grouped masked FP8 GEMM (MoE decode): group g uses rows [0, masked_m[g])
  * of its [max_m][k] slab of A.
  *   a         e4m3 [num_groups][max_m][k]  sfa  num_groups blocks of sf words, R = max_m

@@ -21,6 +21,7 @@ __all__ = [
     "DGError", "lib", "dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
     "dg_m_grouped_fp8_gemm_nt_masked", "dg_m_grouped_fp8_fp4_gemm_nt_masked",
     "dg_m_grouped_fp8_gemm_nt_masked_swiglu", "dg_m_grouped_fp8_fp4_gemm_nt_masked_swiglu", "dg_fp8_gemm_nt_noalloc", "dg_noalloc_scratch_bytes", "dg_fp8_fp4_gemm_nt", "dg_bf16_gemm_nt", "dg_m_grouped_fp8_fp4_gemm_nt_contiguous",
+    "dg_m_grouped_fp8_gemm_nn_contiguous", "dg_k_grouped_fp8_gemm_tn_contiguous",
     "dg_quantize_fp8", "dg_quantize_fp4", "dg_pack_sf", "dg_packed_sf_words", "dg_get_num_sms",
     "dg_set_num_sms", "dg_set_pdl", "dg_get_pdl", "dg_set_tile_config", "dg_get_mk_alignment_for_contiguous_layout", "dg_get_last_error",
     "dg_debug_starved_wait", "dg_launch_count", "dg_query_dense_config", "dg_num_tiles", "dg_debug_fastdiv", "dg_shutdown",
@@ -49,6 +50,10 @@ SYMBOLS = {
     "dg_bf16_gemm_nt": (_INT, [_VP, _VP, _VP, _VP, _INT, _INT, _INT, _VP]),
     "dg_m_grouped_fp8_fp4_gemm_nt_contiguous": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _I32P, _INT, _INT,
                                                        _INT, _INT, _VP]),
+    "dg_m_grouped_fp8_gemm_nn_contiguous": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _I32P, _INT, _INT, _INT,
+                                                   _INT, _VP]),
+    "dg_k_grouped_fp8_gemm_tn_contiguous": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _I32P, _INT, _INT, _INT,
+                                                   _INT, _VP]),
     "dg_quantize_fp8": (_INT, [_VP, _INT, _INT, _INT, _VP, _VP, _VP]),
     "dg_quantize_fp4": (_INT, [_VP, _INT, _INT, _VP, _VP, _VP]),
     "dg_pack_sf": (_INT, [_VP, _INT, _INT, _INT, _VP, _VP]),
@@ -174,6 +179,28 @@ def dg_m_grouped_fp8_fp4_gemm_nt_contiguous(a, sfa, b, sfb, c, d, m_indices, str
     _check(lib().dg_m_grouped_fp8_fp4_gemm_nt_contiguous(_p(a), _p(sfa), _p(b), _p(sfb), _p(c), _p(d),
                                                          _p(m_indices), m_total, n, k, g, _stream(stream)),
            "dg_m_grouped_fp8_fp4_gemm_nt_contiguous")
+
+
+def dg_m_grouped_fp8_gemm_nn_contiguous(a, sfa, b, sfb, c, d, m_indices, stream=None) -> None:
+    """a: e4m3 [m_total, k]; b: e4m3 [groups, k, n] (not transposed);
+    m_indices: int32 [m_total]."""
+    m_total, k = a.shape
+    g, n = b.shape[0], b.shape[2]
+    _check(lib().dg_m_grouped_fp8_gemm_nn_contiguous(_p(a), _p(sfa), _p(b), _p(sfb), _p(c), _p(d), _p(m_indices),
+                                                     m_total, n, k, g, _stream(stream)),
+           "dg_m_grouped_fp8_gemm_nn_contiguous")
+
+
+def dg_k_grouped_fp8_gemm_tn_contiguous(a, sfa, b, sfb, c, d, ks, stream=None) -> None:
+    """a: e4m3 [k_total, m]; b: e4m3 [k_total, n]; ks: int32 [groups] on the
+    device (K rows per group); c: bf16 [groups, m, n] or None; d: bf16
+    [groups, m, n]."""
+    k_total, m = a.shape
+    n = b.shape[1]
+    g = ks.shape[0]
+    _check(lib().dg_k_grouped_fp8_gemm_tn_contiguous(_p(a), _p(sfa), _p(b), _p(sfb), _p(c), _p(d), _p(ks), g, m, n,
+                                                     k_total, _stream(stream)),
+           "dg_k_grouped_fp8_gemm_tn_contiguous")
 
 
 def dg_m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, masked_m, expected_m: int = 0, stream=None) -> None:

@@ -44,7 +44,13 @@ constexpr int kEpiCols = 32;       // columns per epilogue store box
 constexpr int kTmemCols = 512;
 constexpr int kMaxMaskedGroups = 1024;
 
-enum : int { kDense = 0, kContig = 1, kMasked = 2 };
+// kKGrouped: the weight-gradient layout, grouped along K -- group g owns the
+// K rows [K_0 + ... + K_(g-1), ... + K_g) of A and B and its own D[g].
+enum : int { kDense = 0, kContig = 1, kMasked = 2, kKGrouped = 3 };
+
+// Operand majorness (template parameter MAJ): which of A and B are stored
+// MN-major (M or N contiguous, K rows) instead of K-major.
+enum : int { kMajorK = 0, kAMajorMN = 1, kBMajorMN = 2 };
 
 // Epilogues: D = bf16(acc + C), or SwiGLU on B rows interleaved in blocks of
 // kSwiGluBlock (gate rows, then the matching up rows): act = bf16(silu(gate)
@@ -83,6 +89,7 @@ struct GemmArgs {
   float* ws;                 // stream-K partials [sk_tiles][max_seg][kBM][BN] (FP32)
   const int32_t* m_indices;  // contiguous: group of each row (-1 = padding)
   const int32_t* masked_m;   // masked: valid rows per group
+  const int32_t* ks;         // k-grouped: K of each group (multiples of 128)
   int rows;                  // dense: M; contiguous: M_total; masked: max_m
   int n, k;
   int d_cols;                // columns of D: n, or n / 2 for SwiGLU
@@ -106,6 +113,7 @@ struct GemmArgs {
   int sfa_q, sfb_q;                    // packed groups along K
   int raster;                          // m-blocks per raster band
   FastDiv band_div;                    // division by raster * num_n_blocks (tiles per band)
+  FastDiv group_div;                   // k-grouped: division by num_m_blocks * num_n_blocks
   unsigned long long timeout_ns;
   long long sfa_words, sfb_words;      // total packed words (self-check bounds)
 };
@@ -215,7 +223,8 @@ __device__ __forceinline__ void raster_tile_fast(int tl, const GemmArgs& a, int&
 // CTA's stream-K share cut at tile boundaries.  Contiguous: every tile of the
 // raster order round robin (a tile's group from its first row).  Masked:
 // group by group, n-blocks, m-blocks fastest (m-blocks of a group share its B
-// tiles).
+// tiles).  K-grouped: group by group, raster order inside a group; a unit's
+// K-blocks are its group's (global K-block indices, from s_prefix).
 template <int LAYOUT>
 struct WorkIter {
   int t, step, cta;
@@ -257,6 +266,12 @@ struct WorkIter {
         u.g = g;
         u.nb = local / mcount;
         u.mb = local % mcount;
+      } else if (LAYOUT == kKGrouped) {
+        const int g = (int)a.group_div.div((uint32_t)t);
+        raster_tile_fast(t - g * (int)a.group_div.d, a, u.mb, u.nb);
+        u.g = g;
+        u.kb0 = s_prefix[g];
+        u.kb1 = s_prefix[g + 1];
       } else {
         raster_tile_fast(t, a, u.mb, u.nb);
         if (LAYOUT == kContig) {
@@ -296,7 +311,12 @@ struct WorkIter {
 // CTAS = 2: a cluster of two CTAs computes 256 x BN tiles (dense layout only);
 // tm_sfa / tm_sfb view the packed scale words as rows of 512 bytes so that
 // the peer's scale loads can complete on the leader's barrier.
-template <int BN, bool FP4, int LAYOUT, int CTAS, int EPI = kEpiPlain, bool BF16 = false>
+//
+// MAJ != kMajorK: A and/or B staged MN-major (TN / NN layouts): each 128-wide
+// M or N block of a stage is one TMA box of 128 elements x 128 K rows, and
+// the MMA reads it through an MN-major descriptor (plain FP8 tiles of width
+// 128 or 256 only).
+template <int BN, bool FP4, int LAYOUT, int CTAS, int EPI = kEpiPlain, bool BF16 = false, int MAJ = kMajorK>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_d, const __grid_constant__ CUtensorMap tm_sfa,
@@ -305,6 +325,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   static_assert(EPI == kEpiPlain || (CTAS == 1 && BN % (2 * kSwiGluBlock) == 0), "SwiGLU tiles hold whole block pairs");
   using C = Cfg<BN, FP4, CTAS, BF16>;
   static_assert(!BF16 || (CTAS == 1 && EPI == kEpiPlain), "bf16: single CTAs, plain epilogue");
+  constexpr bool kAMn = (MAJ & kAMajorMN) != 0;
+  constexpr bool kBMn = (MAJ & kBMajorMN) != 0;
+  static_assert(MAJ == kMajorK || (!FP4 && !BF16 && CTAS == 1 && EPI == kEpiPlain && BN % 128 == 0),
+                "MN-major operands: FP8, single CTAs, plain epilogue, 128-wide column blocks");
+  static_assert(LAYOUT != kKGrouped || MAJ == (kAMajorMN | kBMajorMN), "k-grouped: A and B MN-major");
+  // D and C of the masked and k-grouped layouts are [groups][rows][n]
+  constexpr bool kGroupRows = (LAYOUT == kMasked || LAYOUT == kKGrouped);
   constexpr bool kPair = (CTAS == 2);
   constexpr int kTileM = kBM * CTAS;
   constexpr int S = C::kStages;
@@ -384,6 +411,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int g = 0; g < a.num_groups; ++g) s_prefix[g + 1] += s_prefix[g];
     }
   }
+  if (LAYOUT == kKGrouped) {
+    // K-blocks per group, read from device memory, then an exclusive prefix
+    // (the first K-block of each group); K of a group must be a non-negative
+    // multiple of 128 and the groups must fit in the K rows of A and B
+    for (int g = threadIdx.x; g < a.num_groups; g += kThreads) {
+      int kk = __ldg(a.ks + g);
+      if (kk < 0 || kk % kBK != 0) {
+        record_error(-5 /* DG_ERR_BAD_METADATA */);
+        kk = 0;
+      }
+      s_prefix[g + 1] = kk / kBK;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      s_prefix[0] = 0;
+      for (int g = 0; g < a.num_groups; ++g) {
+        int next = s_prefix[g] + s_prefix[g + 1];
+        if (next > a.kb_total) {
+          record_error(-5 /* DG_ERR_BAD_METADATA */);
+          next = a.kb_total;
+        }
+        s_prefix[g + 1] = next;
+      }
+    }
+  }
   tc_fence_before();
   if constexpr (kPair)
     cluster_sync_all();  // both CTAs' barriers initialised before any cross-CTA arrival
@@ -395,6 +447,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     num_units = s_prefix[a.num_groups];
   else if (LAYOUT == kDense)
     num_units = a.dp_tiles;
+  else if (LAYOUT == kKGrouped)
+    num_units = a.num_groups * a.num_m_blocks * a.num_n_blocks;
   else
     num_units = a.num_m_blocks * a.num_n_blocks;
 
@@ -423,7 +477,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nchunks = c1 - c0 + 1;
         const int a_row = u.mb * kTileM + (int)rank * kBM;
         const int a_grp = (LAYOUT == kMasked) ? u.g : 0;
-        const int b_grp = (LAYOUT == kDense) ? 0 : u.g;
+        const int b_grp = (LAYOUT == kDense || LAYOUT == kKGrouped) ? 0 : u.g;
+        // MN-major B: the 128-wide column blocks of the tile that hold
+        // columns below n (a block wholly past n is not loaded; the MMA
+        // columns it feeds are never stored)
+        const int b_blocks = kBMn ? min(BN / 128, (a.n - n0 + 127) / 128) : 1;
         const int32_t* sfa_g = a.sfa + (LAYOUT == kMasked ? (long long)u.g * a.sfa_group_words : 0);
         const int32_t* sfb_g = a.sfb + (long long)b_grp * a.sfb_group_words;
         for (int kb = kb0; kb < kb1; ++kb) {
@@ -433,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const bool new_sfa = !BF16 && (((kb & 3) == 0) || kb == kb0);
           const bool new_sfb = !BF16 && (FP4 || new_sfa);
-          uint32_t bytes = C::kABytes + C::kBTxBytes;
+          uint32_t bytes = C::kABytes + (kBMn ? (uint32_t)b_blocks * (kBK * 128) : (uint32_t)C::kBTxBytes);
           if (new_sfa) bytes += C::kSfaBytes;
           if (new_sfb) bytes += 512u * nchunks;
           DG_CHECK(((smem_u32(s_a + stage * C::kABytes) | smem_u32(s_b + stage * C::kBBytes)) & 1023) == 0 &&
@@ -463,8 +521,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             continue;
           }
           mbar_arrive_expect_tx(&full[stage], bytes);
-          tma_load_3d(s_a + stage * C::kABytes, &tm_a, &full[stage], kb * C::kKPerStage, a_row, a_grp);
-          tma_load_3d(s_b + stage * C::kBBytes, &tm_b, &full[stage], kb * C::kKPerStage, n0, b_grp);
+          if constexpr (kAMn)
+            tma_load_3d(s_a + stage * C::kABytes, &tm_a, &full[stage], a_row, kb * kBK, a_grp);
+          else
+            tma_load_3d(s_a + stage * C::kABytes, &tm_a, &full[stage], kb * C::kKPerStage, a_row, a_grp);
+          if constexpr (kBMn) {
+            for (int cb = 0; cb < b_blocks; ++cb)
+              tma_load_3d(s_b + stage * C::kBBytes + cb * (kBK * 128), &tm_b, &full[stage], n0 + 128 * cb, kb * kBK,
+                          b_grp);
+          } else {
+            tma_load_3d(s_b + stage * C::kBBytes, &tm_b, &full[stage], kb * C::kKPerStage, n0, b_grp);
+          }
           if (new_sfa) {
             const int32_t* src = sfa_g + ((long long)(kb >> 2) * a.sfa_chunks + u.mb) * 128;
             if (DG_CHECK(src >= a.sfa && src + 128 <= a.sfa + a.sfa_words &&
@@ -517,6 +584,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       Unit u;
       while (ok && it.next(a, s_prefix, num_units, u)) {
         if (LAYOUT == kContig && !u.valid) continue;
+        // a k-grouped tile of an empty group takes no accumulator: its
+        // epilogue writes C (or zeros) alone
+        if (LAYOUT == kKGrouped && u.kb0 == u.kb1) continue;
         const int kb0 = u.kb0;
         const int kb1 = u.kb1;
         const int n0 = u.nb * BN;
@@ -597,19 +667,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_cp_32x128b_x4(tmem_base + C::kColSfb + 4 * ch, sd);
             }
           }
-          const uint64_t adesc = sdesc_k_sw128(s_a + stage * C::kABytes);
-          const uint64_t bdesc = sdesc_k_sw128(s_b + stage * C::kBBytes);
+          // K-major: a K-step of 32 e4m3 is 32 bytes along the swizzled rows
+          // (+2 in the 16-byte address field); MN-major: 32 rows of 128 bytes
+          // (+256).  Bits 15 / 16 of the instruction descriptor mark A / B
+          // as MN-major.
+          const uint64_t adesc = kAMn ? sdesc_mn_sw128(s_a + stage * C::kABytes, 0)
+                                      : sdesc_k_sw128(s_a + stage * C::kABytes);
+          const uint64_t bdesc = kBMn ? sdesc_mn_sw128(s_b + stage * C::kBBytes, kBK * 128)
+                                      : sdesc_k_sw128(s_b + stage * C::kBBytes);
+          constexpr uint64_t kAStep = kAMn ? 256 : 2, kBStep = kBMn ? 256 : 2;
+          constexpr uint32_t kMajBits = (kAMn ? 1u << 15 : 0u) | (kBMn ? 1u << 16 : 0u);
           const uint32_t ida = (uint32_t)(kb & 3);
 #pragma unroll
           for (int ks = 0; ks < kBK / 32; ++ks) {
             const uint32_t idb = FP4 ? (uint32_t)ks : ida;
-            const uint32_t idesc = C::kIdesc | (ida << 29) | (idb << 4);
+            const uint32_t idesc = C::kIdesc | kMajBits | (ida << 29) | (idb << 4);
             if constexpr (kPair)
               tc_mma_mxf8f6f4_pair(d_t, adesc + (uint64_t)(ks * 2), bdesc + (uint64_t)(ks * 2), idesc,
                                    sfa_t | (ida << 30), sfb_t | (idb << 30), (kb > kb0 || ks > 0) ? 1u : 0u);
             else
-              tc_mma_mxf8f6f4(d_t, adesc + (uint64_t)(ks * 2), bdesc + (uint64_t)(ks * 2), idesc,
-                              sfa_t | (ida << 30), sfb_t | (idb << 30), (kb > kb0 || ks > 0) ? 1u : 0u);
+              tc_mma_mxf8f6f4(d_t, adesc + kAStep * ks, bdesc + kBStep * ks, idesc, sfa_t | (ida << 30),
+                              sfb_t | (idb << 30), (kb > kb0 || ks > 0) ? 1u : 0u);
           }
           if constexpr (kPair)
             tc_commit_pair_mc(&empty[stage], 0x3);  // frees the stage in both CTAs
@@ -670,7 +748,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int rrow = rr0 + 8 * i + (int)(lane >> 2);
-        const long long rg = (LAYOUT == kMasked) ? (long long)uu.g * a.rows + rrow : rrow;
+        const long long rg = kGroupRows ? (long long)uu.g * a.rows + rrow : rrow;
         if (rrow < lim &&
             DG_CHECK(((reinterpret_cast<uintptr_t>(a.c + rg * a.n + cw) & 15) == 0) && rrow < a.rows && rg >= 0, 1)) {
           const uint4* src = reinterpret_cast<const uint4*>(a.c + rg * a.n + cw) + seg;
@@ -721,7 +799,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (LAYOUT == kMasked) limit_rows = min(max(__ldg(a.masked_m + u.g), 0), a.rows);
       const int vr = min(32, limit_rows - r0);
       const int row = r0 + (int)lane;
-      const long long grow = (LAYOUT == kMasked) ? (long long)u.g * a.rows + row : row;
+      const long long grow = kGroupRows ? (long long)u.g * a.rows + row : row;
+      // k-grouped tile of an empty group: no accumulator, D = C (or 0)
+      const bool empty_k = (LAYOUT == kKGrouped) && u.kb0 == u.kb1;
       const int colw = u.nb * BN + half * kCols;  // first column of this warp
 
       uint4 creg[kChunks][4];
@@ -748,7 +828,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 
       int ok = 1;
-      if (lane == 0) ok = dg_wait(&tfull[buf], use & 1, s_abort, limit) ? 1 : 0;
+      if (lane == 0 && !empty_k) ok = dg_wait(&tfull[buf], use & 1, s_abort, limit) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
@@ -775,7 +855,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_3d(&tm_d, stg, col0, r0, (LAYOUT == kMasked) ? u.g : 0);
+            tma_store_3d(&tm_d, stg, col0, r0, kGroupRows ? u.g : 0);
             bulk_commit_group();
           }
         } else if ((int)lane < vr &&
@@ -864,9 +944,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             DG_CHECK(((t_row & 0xFFFF) + j * kEpiCols + kEpiCols <= (uint32_t)kTmemCols) &&
                          ((t_row >> 16) & 0xFFFF) == (uint32_t)(q * 32) + (tmem_base >> 16) && (warp & 3) == q,
                      8);
-            tc_ld_32x32b_x32(t_row + j * kEpiCols, acc);
+            if (!empty_k) {
+              tc_ld_32x32b_x32(t_row + j * kEpiCols, acc);
+            } else {
+#pragma unroll
+              for (int i = 0; i < kEpiCols; ++i) acc[i] = 0u;
+            }
             if (load_c) stage_c(creg[j]);
-            tc_wait_ld_regs(acc);
+            if (!empty_k) tc_wait_ld_regs(acc);
             uint32_t packed[kEpiCols / 2];
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
@@ -886,6 +971,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }  // plain epilogue
+      if (empty_k) continue;  // (no accumulator taken)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) release_acc(buf);

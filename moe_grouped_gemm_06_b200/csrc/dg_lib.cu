@@ -213,8 +213,9 @@ int sk_max_segments(int sk_tiles, int kb, int G) {
 // among plans at the floor the one with the least estimated SM time wins.  Sharing is offered for the dense layout only
 // (allow_sk) and only within ws_cap bytes of workspace (0: no cap).  Ties
 // keep whole tiles.
+// MN-major B (mn_b) is staged in 128-wide column blocks: widths 128 and 256.
 Plan plan_gemm(long long m_blocks, int n, int k, int sms, bool allow_sk, size_t ws_cap = 0, bool fp4 = false,
-               bool bf16 = false) {
+               bool bf16 = false, bool mn_b = false) {
   Plan best;
   best.cost = 1e300;
   const int kb = k / 128;
@@ -229,6 +230,7 @@ Plan plan_gemm(long long m_blocks, int n, int k, int sms, bool allow_sk, size_t 
     if (bf16) wc.per_kb = wc.per_kb_bf16;
     const int bn = wc.bn;
     if (forced_block_n() ? bn != forced_block_n() : !wc.automatic) continue;
+    if (mn_b && bn % 128 != 0) continue;
     // 64-wide tiles double the CTAs of a dense problem of at most two
     // m-blocks; elsewhere (and for the grouped layouts) they only add A reads
     if (bn == 64 && !forced_block_n() && !(streams_b && allow_sk)) continue;
@@ -324,11 +326,11 @@ float* workspace(size_t bytes, cudaStream_t s) {
 
 // ------------------------------------------------------------ launches
 
-template <int BN, bool FP4, int LAYOUT, int CTAS, int EPI = dg::kEpiPlain, bool BF16 = false>
+template <int BN, bool FP4, int LAYOUT, int CTAS, int EPI = dg::kEpiPlain, bool BF16 = false, int MAJ = dg::kMajorK>
 dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td, const CUtensorMap& tsfa,
                       const CUtensorMap& tsfb, const dg::GemmArgs& args, int grid, cudaStream_t s) {
   using C = dg::Cfg<BN, FP4, CTAS, BF16>;
-  auto kern = dg::gemm_kernel<BN, FP4, LAYOUT, CTAS, EPI, BF16>;
+  auto kern = dg::gemm_kernel<BN, FP4, LAYOUT, CTAS, EPI, BF16, MAJ>;
   static std::atomic<uint64_t> attr_set_mask{0};  // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
@@ -345,14 +347,24 @@ dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
   return DG_OK;
 }
 
-template <bool FP4, int LAYOUT, int EPI = dg::kEpiPlain, bool BF16 = false>
+template <bool FP4, int LAYOUT, int EPI = dg::kEpiPlain, bool BF16 = false, int MAJ = dg::kMajorK>
 dg_status dispatch(int bn, int ctas, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
                    const CUtensorMap& tsfa, const CUtensorMap& tsfb, const dg::GemmArgs& args, int grid,
                    cudaStream_t s) {
   // CTA-pair (cta_group::2) kernels are not launched: on B200 they stopped
   // with "illegal instruction" and the cause is not yet known.
   if (ctas != 1) return DG_ERR_UNSUPPORTED;
-  if constexpr (BF16) {
+  if constexpr (MAJ != dg::kMajorK) {
+    // MN-major operands: FP8, plain epilogue, 128-wide column blocks
+    static_assert(!FP4 && !BF16 && EPI == dg::kEpiPlain, "MN-major: FP8, plain epilogue");
+    switch (bn) {
+      case 128: return launch_gemm<128, false, LAYOUT, 1, EPI, false, MAJ>(ta, tb, td, tsfa, tsfb, args, grid, s);
+      case 256: return launch_gemm<256, false, LAYOUT, 1, EPI, false, MAJ>(ta, tb, td, tsfa, tsfb, args, grid, s);
+      default: return DG_ERR_UNSUPPORTED;
+    }
+  } else if constexpr (LAYOUT == dg::kKGrouped) {
+    return DG_ERR_UNSUPPORTED;  // (k-grouped is MN-major only)
+  } else if constexpr (BF16) {
     // bf16: dense tiles of the widths the heuristic picks
     switch (bn) {
       case 64: return launch_gemm<64, false, LAYOUT, 1, EPI, true>(ta, tb, td, tsfa, tsfb, args, grid, s);
@@ -368,15 +380,16 @@ dg_status dispatch(int bn, int ctas, const CUtensorMap& ta, const CUtensorMap& t
       case 256: return launch_gemm<256, FP4, LAYOUT, 1, EPI>(ta, tb, td, tsfa, tsfb, args, grid, s);
       default: return DG_ERR_UNSUPPORTED;
     }
-  }
-  switch (bn) {
-    case 64: return launch_gemm<64, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
-    case 128: return launch_gemm<128, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
-    case 160: return launch_gemm<160, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
-    case 192: return launch_gemm<192, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
-    case 224: return launch_gemm<224, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
-    case 256: return launch_gemm<256, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
-    default: return DG_ERR_UNSUPPORTED;
+  } else {
+    switch (bn) {
+      case 64: return launch_gemm<64, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
+      case 128: return launch_gemm<128, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
+      case 160: return launch_gemm<160, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
+      case 192: return launch_gemm<192, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
+      case 224: return launch_gemm<224, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
+      case 256: return launch_gemm<256, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
+      default: return DG_ERR_UNSUPPORTED;
+    }
   }
 }
 
@@ -393,14 +406,17 @@ struct Problem {
   int n, k;
   int groups;      // 1 for dense
   int expected_m;  // masked hint
+  const int32_t* ks = nullptr;  // k-grouped: K of each group (device)
 };
 
 // fixed_ws / fixed_ws_bytes: when given, stream-K partials go to this
 // caller-provided device buffer instead of the per-stream workspace, and the
 // planner only considers plans that fit in fixed_ws_bytes (whole tiles
 // always do).
-template <bool FP4, int LAYOUT, int EPI = dg::kEpiPlain, bool BF16 = false>
+template <bool FP4, int LAYOUT, int EPI = dg::kEpiPlain, bool BF16 = false, int MAJ = dg::kMajorK>
 dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, size_t fixed_ws_bytes = 0) {
+  constexpr bool kAMn = (MAJ & dg::kAMajorMN) != 0;
+  constexpr bool kBMn = (MAJ & dg::kBMajorMN) != 0;
   // a bf16 stage covers 64 K-elements in the time an e4m3 stage covers 128:
   // the planner sees bf16 as an e4m3 problem of twice the K
   const int k_plan = BF16 ? 2 * p.k : p.k;
@@ -414,10 +430,15 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
     if (EPI == dg::kEpiSwiGlu && plan.bn != 128 && plan.bn != 256 && !forced_block_n())
       plan.bn = plan.bn > 192 ? 256 : 128;  // SwiGLU tiles hold whole gate/up block pairs
     plan.grid = (int)std::min<long long>((long long)p.groups * m_blocks * ceil_div(p.n, plan.bn), sms);
+  } else if (LAYOUT == dg::kKGrouped) {
+    // every group has the same tiles; planned at the mean K of a group
+    const int k_mean = std::max(128, (int)(p.k / p.groups) / 128 * 128);
+    plan = plan_gemm((long long)p.groups * m_blocks, p.n, k_mean, sms, false, 0, false, false, kBMn);
   } else {
     plan = plan_gemm(m_blocks, p.n, k_plan, sms, LAYOUT == dg::kDense, fixed_ws != nullptr ? fixed_ws_bytes : 0, FP4,
-                     BF16);
+                     BF16, kBMn);
   }
+  if (plan.grid <= 0) return DG_ERR_UNSUPPORTED;  // (a forced width this layout cannot use)
 
   dg::GemmArgs args{};
   args.sfa = p.sfa;
@@ -427,6 +448,7 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
   args.ws = nullptr;
   args.m_indices = p.m_indices;
   args.masked_m = p.masked_m;
+  args.ks = p.ks;
   args.rows = p.rows;
   args.n = p.n;
   args.d_cols = (EPI == dg::kEpiSwiGlu) ? p.n / 2 : p.n;
@@ -448,9 +470,10 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
   args.sfb_group_words = (long long)args.sfb_q * args.sfb_chunks * 128;
   args.raster = 8;
   args.band_div.init((uint32_t)(args.raster * args.num_n_blocks));
+  args.group_div.init((uint32_t)(args.num_m_blocks * args.num_n_blocks));
   args.timeout_ns = timeout_ns();
   args.sfa_words = args.sfa_group_words * ((LAYOUT == dg::kMasked) ? p.groups : 1);
-  args.sfb_words = args.sfb_group_words * ((LAYOUT == dg::kDense) ? 1 : p.groups);
+  args.sfb_words = args.sfb_group_words * ((LAYOUT == dg::kDense || LAYOUT == dg::kKGrouped) ? 1 : p.groups);
 
   if (plan.sk_tiles > 0) {
     const size_t need = plan.ws_bytes();
@@ -464,7 +487,9 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
   }
 
   const int ga = (LAYOUT == dg::kMasked) ? p.groups : 1;
-  const int gb = (LAYOUT == dg::kDense) ? 1 : p.groups;
+  const int gb = (LAYOUT == dg::kDense || LAYOUT == dg::kKGrouped) ? 1 : p.groups;
+  const int gd = (LAYOUT == dg::kMasked || LAYOUT == dg::kKGrouped) ? p.groups : 1;
+  const uint64_t k_ext = (uint64_t)std::max(p.k, 128);  // K rows of MN-major maps
   CUtensorMap ta, tb, td;
   bool ok;
   if (BF16) {
@@ -472,12 +497,21 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
                   (uint64_t)p.rows * p.k * 2, 64, dg::kBM, CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.b, p.k, p.n, gb, (uint64_t)p.k * 2,
                         (uint64_t)p.n * p.k * 2, 64, plan.bn, CU_TENSOR_MAP_SWIZZLE_128B);
+  } else if (kAMn) {
+    // A stored [K][rows]: boxes of 128 rows of A (contiguous) x 128 K rows
+    // (K = 0, all groups empty: a map of one box that no load reads)
+    ok = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.a, p.rows, k_ext, ga, (uint64_t)p.rows,
+                  (uint64_t)p.rows * k_ext, dg::kBM, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   } else {
     ok = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.a, p.k, p.rows, ga, (uint64_t)p.k, (uint64_t)p.rows * p.k,
                   128, dg::kBM, CU_TENSOR_MAP_SWIZZLE_128B);
   }
   if (BF16) {
-  } else if (FP4)
+  } else if (kBMn)
+    // B stored [K][n]: boxes of 128 columns x 128 K rows
+    ok = ok && make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.b, p.n, k_ext, gb, (uint64_t)p.n, (uint64_t)p.n * k_ext,
+                        128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  else if (FP4)
     ok = ok && make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, p.b, p.k, p.n, gb, (uint64_t)p.k / 2,
                         (uint64_t)p.n * p.k / 2, 128, plan.bn / plan.ctas, CU_TENSOR_MAP_SWIZZLE_128B);
   else
@@ -495,7 +529,7 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
     ok = ok && make_map(&tsfb, CU_TENSOR_MAP_DATA_TYPE_INT32, p.sfb, 128, rows_b, 1, 512, rows_b * 512, 128, 1,
                         CU_TENSOR_MAP_SWIZZLE_NONE);
   }
-  ok = ok && make_map(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.d, args.d_cols, p.rows, ga, (uint64_t)args.d_cols * 2,
+  ok = ok && make_map(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.d, args.d_cols, p.rows, gd, (uint64_t)args.d_cols * 2,
                       (uint64_t)p.rows * args.d_cols * 2, dg::kEpiCols, 32, CU_TENSOR_MAP_SWIZZLE_64B);
   if (!ok) return DG_ERR_CUDA;
 
@@ -506,7 +540,7 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
                  LAYOUT, (int)FP4, p.rows, p.n, p.k, p.groups, plan.bn, plan.dp_tiles, plan.sk_tiles, plan.sk_split,
                  plan.max_seg, plan.grid, plan.cost);
 
-  dg_status st = dispatch<FP4, LAYOUT, EPI, BF16>(plan.bn, plan.ctas, ta, tb, td, tsfa, tsfb, args, plan.grid, s);
+  dg_status st = dispatch<FP4, LAYOUT, EPI, BF16, MAJ>(plan.bn, plan.ctas, ta, tb, td, tsfa, tsfb, args, plan.grid, s);
   if (st != DG_OK || plan.sk_tiles == 0) return st;
 
   dg::SkReduceArgs r{};
@@ -650,6 +684,35 @@ dg_status dg_m_grouped_fp8_fp4_gemm_nt_contiguous(const void* a, const int32_t* 
                                                   const int32_t* m_indices, int m_total, int n, int k,
                                                   int num_groups, void* stream) {
   return contiguous_impl(true, a, sfa, b, sfb, c, d, m_indices, m_total, n, k, num_groups, stream);
+}
+
+dg_status dg_m_grouped_fp8_gemm_nn_contiguous(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                                              const void* c, void* d, const int32_t* m_indices, int m_total, int n,
+                                              int k, int num_groups, void* stream) {
+  if (m_total < 0 || m_total % 128 != 0 || num_groups <= 0 || !m_indices) return DG_ERR_INVALID_ARG;
+  dg_status st = check_common(a, sfa, b, sfb, c, d, n, k);
+  if (st != DG_OK) return st;
+  if (n % 16 != 0) return DG_ERR_INVALID_ARG;  // B's K rows are n bytes: 16-byte TMA row stride
+  if (c == d && c != nullptr) return DG_ERR_INVALID_ARG;
+  if (m_total == 0) return DG_OK;
+  Problem p{a, sfa, b, sfb, c, d, m_indices, nullptr, m_total, n, k, num_groups, 0};
+  return run_gemm<false, dg::kContig, dg::kEpiPlain, false, dg::kBMajorMN>(p, static_cast<cudaStream_t>(stream));
+}
+
+dg_status dg_k_grouped_fp8_gemm_tn_contiguous(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                                              const void* c, void* d, const int32_t* ks, int num_groups, int m,
+                                              int n, int k_total, void* stream) {
+  if (!a || !sfa || !b || !sfb || !d || !ks) return DG_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(sfa) || !aligned16(b) || !aligned16(sfb) || !aligned16(d) || !aligned16(ks))
+    return DG_ERR_INVALID_ARG;
+  if (c && !aligned16(c)) return DG_ERR_INVALID_ARG;
+  if (num_groups <= 0 || num_groups > dg::kMaxMaskedGroups) return DG_ERR_INVALID_ARG;
+  // A's and B's K rows are m and n bytes (16-byte TMA row stride)
+  if (m <= 0 || m % 16 != 0 || n <= 0 || n % 16 != 0) return DG_ERR_INVALID_ARG;
+  if (k_total < 0 || k_total % 128 != 0) return DG_ERR_INVALID_ARG;
+  Problem p{a, sfa, b, sfb, c, d, nullptr, nullptr, m, n, k_total, num_groups, 0, ks};
+  return run_gemm<false, dg::kKGrouped, dg::kEpiPlain, false, dg::kAMajorMN | dg::kBMajorMN>(
+      p, static_cast<cudaStream_t>(stream));
 }
 
 static dg_status masked_impl(bool fp4, bool swiglu, const void* a, const int32_t* sfa, const void* b,

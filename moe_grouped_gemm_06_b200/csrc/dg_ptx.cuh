@@ -376,6 +376,23 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(const void* tile) {
   return d;
 }
 
+// MN-major operand tile, 128-byte swizzle, as a tiled TMA copy with a box of
+// 128 bytes along M or N by K rows lays it out: K row r at r * 128 bytes
+// (so 8-row groups are 1024 bytes apart: the stride byte offset), and each
+// further 128-element column block of a wider tile `lbo` bytes after the
+// previous one (the leading byte offset).  A K-step of 32 rows starts 4096
+// bytes further on.
+__device__ __forceinline__ uint64_t sdesc_mn_sw128(const void* tile, uint32_t lbo) {
+  uint64_t addr = smem_u32(tile);
+  uint64_t d = 0;
+  d |= (addr >> 4) & 0x3FFFull;               // start address
+  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16; // leading byte offset: next 128-wide M/N block
+  d |= (uint64_t)(1024 >> 4) << 32;           // stride byte offset: next 8-row K group
+  d |= 1ull << 46;                            // descriptor version (sm_100)
+  d |= 2ull << 61;                            // 128-byte swizzle
+  return d;
+}
+
 // 32 rows x 16 bytes, no swizzle, rows contiguous (core matrices of 8 rows
 // are 128 bytes apart): the source of a 32x128b scale-factor copy.
 __device__ __forceinline__ uint64_t sdesc_sf_32x16(const void* p) {

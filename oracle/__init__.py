@@ -212,6 +212,52 @@ def gemm_masked(a, sfa, b, sfb, masked_m, b_fp4=False, out=None) -> np.ndarray:
     return res
 
 
+def gemm_nn_contiguous(a, sfa, b, sfb, m_indices, c=None, out=None) -> np.ndarray:
+    """M-grouped contiguous reference with B not transposed (NN).
+    b: e4m3 [G, K, N]; sfb: UE8M0 [G, ceil(N/128), K/128] (block (n/128,
+    k/128), the NT indexing).  Rows with m_indices < 0 keep ``out`` (NaN)."""
+    a, sfa, b, sfb, _, c = _gemm_args(a, sfa, b, sfb, False, c)
+    M, K = a.shape
+    G, N = b.shape[0], b.shape[2]
+    assert b.shape[1] == K
+    mi = _c(m_indices, np.int32)
+    res = np.full((M, N), np.nan) if out is None else _c(out, np.float64).copy()
+    _load().or_gemm_nn_contiguous(_p(a), _p(sfa), _p(b), _p(sfb), _p(c), _p(mi),
+                                  I64(M), I64(N), I64(K), I64(G), _p(res))
+    return res
+
+
+def gemm_k_grouped_tn(a, sfa, b, sfb, ks, c=None) -> np.ndarray:
+    """K-grouped TN reference (weight gradient), float64 [G, M, N].
+    a: e4m3 [Kt, M]; sfa: UE8M0 [M, Kt/128]; b: e4m3 [Kt, N]; sfb: UE8M0
+    [N, Kt/128]; ks: K rows per group (multiples of 128, sum <= Kt);
+    c: bf16 bits [G, M, N] or None.  D[g] = C[g] + A_g^T B_g."""
+    a, sfa, b, sfb, _, c = _gemm_args(a, sfa, b, sfb, False, c)
+    Kt, M = a.shape
+    N = b.shape[1]
+    ks = _c(ks, np.int32)
+    G = ks.size
+    assert b.shape[0] == Kt and int(ks.sum()) <= Kt and np.all(ks % 128 == 0) and np.all(ks >= 0)
+    out = np.zeros((G, M, N), np.float64)
+    _load().or_gemm_k_grouped_tn(_p(a), _p(sfa), _p(b), _p(sfb), _p(c), _p(ks),
+                                 I64(G), I64(M), I64(N), I64(Kt), _p(out))
+    return out
+
+
+def gemm_k_grouped_tn_points(a, sfa, b, sfb, ks, pg, pi, pj, c=None) -> np.ndarray:
+    """The K-grouped TN reference at the points (pg[t], pi[t], pj[t]) only."""
+    a, sfa, b, sfb, _, c = _gemm_args(a, sfa, b, sfb, False, c)
+    Kt, M = a.shape
+    N = b.shape[1]
+    ks = _c(ks, np.int32)
+    assert b.shape[0] == Kt and int(ks.sum()) <= Kt and np.all(ks % 128 == 0) and np.all(ks >= 0)
+    pg, pi, pj = _c(pg, np.int64), _c(pi, np.int64), _c(pj, np.int64)
+    out = np.zeros(pg.size, np.float64)
+    _load().or_gemm_k_grouped_tn_points(_p(a), _p(sfa), _p(b), _p(sfb), _p(c), _p(ks), I64(ks.size), I64(M),
+                                        I64(N), I64(Kt), _p(pg), _p(pi), _p(pj), I64(pg.size), _p(out))
+    return out
+
+
 SWIGLU_BLOCK = 64
 
 

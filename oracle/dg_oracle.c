@@ -25,6 +25,9 @@
  *        prefill, masked layout for decoding.
  *   [P1] "DeepSeek 发布 DeepGEMM 重大更新" (linlog.top), section "FP4 精度支持":
  *        FP8 x FP4 GEMM, FP4 weights with UE8M0 scale factors, 4 per int32.
+ *   [P5] also: SM100 takes every one of the NT, TN, NN and TT layouts; the
+ *        contiguous grouped GEMM comes as nt and nn; the weight backward is
+ *        k_grouped_fp8_gemm_tn_contiguous, grouped along K.
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *   - FP8 means OCP E4M3FN: bias 7, no infinities, S.1111.111 is NaN, max 448.
@@ -34,6 +37,12 @@
  *     clamped to [-127, 127]; amax == 0 gives i = 0 (code 127).
  *   - FP4 codes are packed two per byte along K, low nibble = even k.
  *   - packed scale layout: see or_pack_sf below.
+ *   - NN: B is stored [K][N] (B[k][n] is the element the NT layout stores at
+ *     [n][k]); its 128x128 block scales keep the NT indexing (n/128, k/128).
+ *   - K-grouped TN: group g owns the K rows [k_g, k_g + ks[g]) of A [K][M] and
+ *     B [K][N] and writes D[g] = C[g] + A_g^T B_g ([M][N]); both operands
+ *     carry one scale per (column, 128-row block of K), the ks[g] being
+ *     multiples of 128; an empty group gives D[g] = C[g].
  */
 #include <math.h>
 #include <stdint.h>
@@ -245,47 +254,65 @@ void or_pack_sf(const uint8_t* e, int64_t rows, int64_t ng, int row_div, int32_t
 /* The contraction.                                                          */
 /* ------------------------------------------------------------------------ */
 
-/* One operand of the product: codes plus the scale lookup. */
+/* One operand of the product: codes plus the scale lookup.  Element (r, k)
+ * of an fp8 operand is codes[r * row_stride + k * k_stride] (K-major storage
+ * [rows][K]: row_stride = K, k_stride = 1; MN-major storage [K][rows]:
+ * row_stride = 1, k_stride = rows).  An fp4 operand is always K-major with
+ * two codes per byte. */
 typedef struct {
-    const uint8_t* codes;   /* row-major [rows][K] bytes (fp8) or [rows][K/2] (fp4) */
-    const uint8_t* sf;      /* UE8M0 codes, [ceil(rows/sf_rows)][K/sf_k] */
+    const uint8_t* codes;
+    int64_t row_stride, k_stride;
+    const uint8_t* sf;      /* UE8M0 codes, [ceil(rows/sf_rows)][sf_cols] */
+    int64_t sf_cols;        /* scale columns per scale row (K / sf_k) */
     int fp4;                /* 1: E2M1 packed two per byte, low nibble = even k */
     int sf_rows;            /* rows sharing one scale (1 or 128) */
     int sf_k;               /* K elements sharing one scale (128 or 32) */
 } operand_t;
 
-static double elem(const operand_t* o, int64_t K, int64_t r, int64_t k) {
+static double elem(const operand_t* o, int64_t r, int64_t k) {
     if (o->fp4) {
-        uint8_t byte = o->codes[r * (K / 2) + k / 2];
+        uint8_t byte = o->codes[r * o->row_stride + k / 2];
         return E2M1[(k & 1) ? (byte >> 4) : (byte & 15)];
     }
-    return E4M3[o->codes[r * K + k]];
+    return E4M3[o->codes[r * o->row_stride + k * o->k_stride]];
 }
 
-static double scale(const operand_t* o, int64_t K, int64_t r, int64_t k) {
-    return UE8M0[o->sf[(r / o->sf_rows) * (K / o->sf_k) + k / o->sf_k]];
+static double scale(const operand_t* o, int64_t r, int64_t k) {
+    return UE8M0[o->sf[(r / o->sf_rows) * o->sf_cols + k / o->sf_k]];
 }
 
-/* sum over k of s_a(m,k) s_b(n,k) a(m,k) b(n,k), evaluated block by block:
- * the K axis is cut at every scale boundary of either operand, each piece is
- * summed unscaled and then multiplied by the two scales of that piece. */
-static double dot(const operand_t* A, int64_t m, const operand_t* B, int64_t n, int64_t K) {
+/* sum over k in [k_begin, k_end) of s_a(m,k) s_b(n,k) a(m,k) b(n,k),
+ * evaluated block by block: the K axis is cut at every scale boundary of
+ * either operand (k_begin is one), each piece is summed unscaled and then
+ * multiplied by the two scales of that piece. */
+static double dot_range(const operand_t* A, int64_t m, const operand_t* B, int64_t n, int64_t k_begin,
+                        int64_t k_end) {
     int64_t step = A->sf_k < B->sf_k ? A->sf_k : B->sf_k;
     double acc = 0;
-    for (int64_t k0 = 0; k0 < K; k0 += step) {
+    for (int64_t k0 = k_begin; k0 < k_end; k0 += step) {
         double part = 0;
-        for (int64_t k = k0; k < k0 + step; ++k) part += elem(A, K, m, k) * elem(B, K, n, k);
-        acc += scale(A, K, m, k0) * scale(B, K, n, k0) * part;
+        for (int64_t k = k0; k < k0 + step; ++k) part += elem(A, m, k) * elem(B, n, k);
+        acc += scale(A, m, k0) * scale(B, n, k0) * part;
     }
     return acc;
 }
 
+static double dot(const operand_t* A, int64_t m, const operand_t* B, int64_t n, int64_t K) {
+    return dot_range(A, m, B, n, 0, K);
+}
+
+/* The NT operands: A [M][K] with 1x128 scales, B [N][K] with 128x128 block
+ * scales (fp8) or [N][K/2] with 1x32 scales (fp4). */
 static void make_ops(operand_t* A, operand_t* B, const uint8_t* a, const uint8_t* sfa,
-                     const uint8_t* b, const uint8_t* sfb, int b_fp4) {
-    A->codes = a; A->sf = sfa; A->fp4 = 0; A->sf_rows = 1; A->sf_k = 128;
-    B->codes = b; B->sf = sfb; B->fp4 = b_fp4;
+                     const uint8_t* b, const uint8_t* sfb, int b_fp4, int64_t K) {
+    A->codes = a; A->row_stride = K; A->k_stride = 1;
+    A->sf = sfa; A->sf_cols = K / 128; A->fp4 = 0; A->sf_rows = 1; A->sf_k = 128;
+    B->codes = b; B->fp4 = b_fp4;
+    B->row_stride = b_fp4 ? K / 2 : K; B->k_stride = 1;
+    B->sf = sfb;
     B->sf_rows = b_fp4 ? 1 : 128;
     B->sf_k = b_fp4 ? 32 : 128;
+    B->sf_cols = K / B->sf_k;
 }
 
 /* Dense NT: out[m][n] = C[m][n] + sum_k ...  for all m < M, n < N.
@@ -297,7 +324,7 @@ void or_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8
              int b_fp4, const uint16_t* c, int64_t M, int64_t N, int64_t K, double* out) {
     build_tables();
     operand_t A, B;
-    make_ops(&A, &B, a, sfa, b, sfb, b_fp4);
+    make_ops(&A, &B, a, sfa, b, sfb, b_fp4, K);
 #pragma omp parallel for schedule(dynamic)
     for (int64_t m = 0; m < M; ++m)
         for (int64_t n = 0; n < N; ++n) {
@@ -313,7 +340,7 @@ void or_gemm_points(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, cons
     build_tables();
     (void)M;
     operand_t A, B;
-    make_ops(&A, &B, a, sfa, b, sfb, b_fp4);
+    make_ops(&A, &B, a, sfa, b, sfb, b_fp4, K);
 #pragma omp parallel for schedule(dynamic)
     for (int64_t t = 0; t < npts; ++t) {
         int64_t m = pm[t], n = pn[t];
@@ -344,7 +371,7 @@ void or_gemm_contiguous(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
         int64_t g = m_indices[m];
         if (g < 0 || g >= num_groups) continue;
         operand_t A, B;
-        make_ops(&A, &B, a, sfa, b + g * bc, sfb + g * bs, b_fp4);
+        make_ops(&A, &B, a, sfa, b + g * bc, sfb + g * bs, b_fp4, K);
         for (int64_t n = 0; n < N; ++n) {
             double base = c ? bf16_bits_to_double(c[m * N + n]) : 0.0;
             out[m * N + n] = base + dot(&A, m, &B, n, K);
@@ -368,8 +395,82 @@ void or_gemm_masked(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
             if (m >= valid) continue;
             operand_t A, B;
             make_ops(&A, &B, a + g * max_m * K, sfa + g * max_m * (K / 128),
-                     b + g * bc, sfb + g * bs, b_fp4);
+                     b + g * bc, sfb + g * bs, b_fp4, K);
             for (int64_t n = 0; n < N; ++n)
                 out[(g * max_m + m) * N + n] = dot(&A, m, &B, n, K);
         }
+}
+
+/* M-grouped contiguous with B not transposed (NN): as or_gemm_contiguous,
+ * but group g's weights are stored [K][N] (b + g*K*N, element (n, k) at
+ * [k][n]); the 128x128 block scales sfb + g*ceil(N/128)*(K/128) keep the
+ * [n/128][k/128] indexing of the NT call. */
+void or_gemm_nn_contiguous(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                           const uint8_t* sfb, const uint16_t* c, const int32_t* m_indices,
+                           int64_t M, int64_t N, int64_t K, int64_t num_groups, double* out) {
+    build_tables();
+    const int64_t bs = ((N + 127) / 128) * (K / 128);
+#pragma omp parallel for schedule(dynamic)
+    for (int64_t m = 0; m < M; ++m) {
+        int64_t g = m_indices[m];
+        if (g < 0 || g >= num_groups) continue;
+        operand_t A, B;
+        make_ops(&A, &B, a, sfa, b + g * K * N, sfb + g * bs, 0, K);
+        B.row_stride = 1;          /* (n, k) at [k][n] */
+        B.k_stride = N;
+        for (int64_t n = 0; n < N; ++n) {
+            double base = c ? bf16_bits_to_double(c[m * N + n]) : 0.0;
+            out[m * N + n] = base + dot(&A, m, &B, n, K);
+        }
+    }
+}
+
+/* K-grouped TN: a is [Kt][M], b is [Kt][N] (Kt = sum of ks); sfa is
+ * [M][Kt/128] and sfb [N][Kt/128] (one code per column and 128-row block of
+ * K).  out[g][i][j] = C[g][i][j] + sum over group g's K rows of
+ * a[k][i] b[k][j] scaled per block; ks[g] are multiples of 128. */
+void or_gemm_k_grouped_tn(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                          const uint8_t* sfb, const uint16_t* c, const int32_t* ks,
+                          int64_t G, int64_t M, int64_t N, int64_t Kt, double* out) {
+    build_tables();
+    operand_t A, B;
+    A.codes = a; A.row_stride = 1; A.k_stride = M;
+    A.sf = sfa; A.sf_cols = Kt / 128; A.fp4 = 0; A.sf_rows = 1; A.sf_k = 128;
+    B.codes = b; B.row_stride = 1; B.k_stride = N;
+    B.sf = sfb; B.sf_cols = Kt / 128; B.fp4 = 0; B.sf_rows = 1; B.sf_k = 128;
+    int64_t k0 = 0;
+    for (int64_t g = 0; g < G; ++g) {
+        const int64_t k1 = k0 + ks[g];
+#pragma omp parallel for schedule(dynamic)
+        for (int64_t i = 0; i < M; ++i)
+            for (int64_t j = 0; j < N; ++j) {
+                const int64_t o = (g * M + i) * N + j;
+                double base = c ? bf16_bits_to_double(c[o]) : 0.0;
+                out[o] = base + dot_range(&A, i, &B, j, k0, k1);
+            }
+        k0 = k1;
+    }
+}
+
+/* or_gemm_k_grouped_tn at the points (pg[t], pi[t], pj[t]) only. */
+void or_gemm_k_grouped_tn_points(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                                 const uint8_t* sfb, const uint16_t* c, const int32_t* ks,
+                                 int64_t G, int64_t M, int64_t N, int64_t Kt,
+                                 const int64_t* pg, const int64_t* pi, const int64_t* pj,
+                                 int64_t npts, double* out) {
+    build_tables();
+    operand_t A, B;
+    A.codes = a; A.row_stride = 1; A.k_stride = M;
+    A.sf = sfa; A.sf_cols = Kt / 128; A.fp4 = 0; A.sf_rows = 1; A.sf_k = 128;
+    B.codes = b; B.row_stride = 1; B.k_stride = N;
+    B.sf = sfb; B.sf_cols = Kt / 128; B.fp4 = 0; B.sf_rows = 1; B.sf_k = 128;
+#pragma omp parallel for schedule(dynamic)
+    for (int64_t t = 0; t < npts; ++t) {
+        const int64_t g = pg[t], i = pi[t], j = pj[t];
+        int64_t k0 = 0;
+        for (int64_t h = 0; h < g; ++h) k0 += ks[h];
+        const int64_t o = (g * M + i) * N + j;
+        double base = c ? bf16_bits_to_double(c[o]) : 0.0;
+        out[t] = base + dot_range(&A, i, &B, j, k0, k0 + ks[g]);
+    }
 }

@@ -54,6 +54,13 @@ def contiguous_layout(seed: int, num_groups: int, lo: int, hi: int, align: int =
     return r.astype(np.int64), m_indices
 
 
+def k_grouped_sizes(seed: int, num_groups: int, lo: int, hi: int, align: int = MK_ALIGNMENT) -> np.ndarray:
+    """K rows per group of a K-grouped (weight-gradient) call: U[lo, hi]
+    (inclusive integers) rounded up to a multiple of ``align``."""
+    r = rng(seed).integers(lo, hi, size=num_groups, endpoint=True)
+    return ((r + align - 1) // align * align).astype(np.int32)
+
+
 def masked_counts(seed: int, num_groups: int, expected_m: int, max_m: int) -> np.ndarray:
     """masked_m[g] = min(max_m, U{0 .. 2*expected_m})."""
     r = rng(seed).integers(0, 2 * expected_m, size=num_groups, endpoint=True)

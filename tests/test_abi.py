@@ -79,6 +79,20 @@ def test_invalid_arguments_rejected_on_host(dg):
                                                128, 128, 0, None) == -1
     assert lib.dg_m_grouped_fp8_gemm_nt_masked(p(fake), p(fake), p(fake), p(fake), p(fake), p(fake), 4, 0,
                                                128, 128, 0, None) == -1
+    # NN contiguous: B rows of n bytes need n % 16 == 0; no in-place C
+    assert lib.dg_m_grouped_fp8_gemm_nn_contiguous(p(fake), p(fake), p(fake), p(fake), None, p(fake), p(fake),
+                                                   128, 136, 128, 2, None) == -1
+    assert lib.dg_m_grouped_fp8_gemm_nn_contiguous(p(fake), p(fake), p(fake), p(fake), p(fake), p(fake), p(fake),
+                                                   128, 128, 128, 2, None) == -1
+    # K-grouped TN: ks given, 1..1024 groups, m and n multiples of 16, k_total % 128 == 0
+    tn = lib.dg_k_grouped_fp8_gemm_tn_contiguous
+    assert tn(p(fake), p(fake), p(fake), p(fake), None, p(fake), None, 2, 128, 128, 256, None) == -1
+    assert tn(p(fake), p(fake), p(fake), p(fake), None, p(fake), p(fake), 0, 128, 128, 256, None) == -1
+    assert tn(p(fake), p(fake), p(fake), p(fake), None, p(fake), p(fake), 1025, 128, 128, 256, None) == -1
+    assert tn(p(fake), p(fake), p(fake), p(fake), None, p(fake), p(fake), 2, 120, 128, 256, None) == -1
+    assert tn(p(fake), p(fake), p(fake), p(fake), None, p(fake), p(fake), 2, 128, 100, 256, None) == -1
+    assert tn(p(fake), p(fake), p(fake), p(fake), None, p(fake), p(fake), 2, 128, 128, 200, None) == -1
+    assert tn(p(fake + 8), p(fake), p(fake), p(fake), None, p(fake), p(fake), 2, 128, 128, 256, None) == -1
     # quantiser: cols % 128, block_rows in {1, 128}
     assert lib.dg_quantize_fp8(p(fake), 4, 100, 1, p(fake), p(fake), None) == -1
     assert lib.dg_quantize_fp8(p(fake), 4, 128, 64, p(fake), p(fake), None) == -1

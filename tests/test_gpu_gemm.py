@@ -564,3 +564,163 @@ def test_contiguous_group_index_out_of_range_is_reported(dg):
     cs["mi"] = mi
     _run_contiguous(dg, cs, N)
     assert dg.dg_get_last_error() == -5
+
+
+# ------------------------------------------------- NN contiguous (B [G, K, N])
+
+def _nn_case(seed, G, lo, hi, N, K):
+    cs = _contiguous_case(seed, G, lo, hi, N, K)
+    cs["qb_kn"] = np.ascontiguousarray(cs["qb"].transpose(0, 2, 1))   # the same weights, stored [K][N]
+    return cs
+
+
+def _run_nn(dg, cs, N, c_given=True):
+    d = torch.empty((cs["M"], N), dtype=torch.int16, device="cuda")
+    c = dev(cs["c"].view(np.int16)) if (c_given and cs["c"] is not None) else None
+    dg.dg_m_grouped_fp8_gemm_nn_contiguous(dev(cs["qa"]), dev(cs["sfa"]), dev(cs["qb_kn"]), dev(cs["sfb"]), c, d,
+                                           dev(cs["mi"]))
+    torch.cuda.synchronize()
+    return bf16_dev_to_f64(d)
+
+
+@pytest.mark.parametrize("bn", [0, 128, 256])
+@pytest.mark.parametrize("N", [384, 208, 112])
+def test_nn_contiguous_matches_oracle(dg, bn, N):
+    # N = 208: the second 128-column block of a 256-wide tile is partly past
+    # N; N = 112: wholly past it (not loaded)
+    K = 512
+    cs = _nn_case(8000 + N, 3, 50, 300, N, K)
+    dg.dg_set_tile_config(bn, 0)
+    try:
+        d = _run_nn(dg, cs, N)
+    finally:
+        dg.dg_set_tile_config(0, 0)
+    ref = oracle.gemm_nn_contiguous(cs["qa"], cs["ea"], cs["qb_kn"], cs["eb"], cs["mi"], c=cs["c"])
+    valid = cs["mi"] >= 0
+    check_close(d[valid], ref[valid], f"nn contiguous N={N} bn={bn}")
+
+
+def test_nn_contiguous_equals_nt_contiguous_on_the_same_weights(dg):
+    N, K = 256, 768
+    cs = _nn_case(8100, 2, 100, 260, N, K)
+    nn = _run_nn(dg, cs, N)
+    nt = _run_contiguous(dg, cs, N)
+    valid = cs["mi"] >= 0
+    check_close(nn[valid], nt[valid], "nn vs nt")
+
+
+@pytest.mark.parametrize("N,K", synth.GROUPED_NK)
+def test_nn_contiguous_full_size_sampled(dg, N, K):
+    cs = _nn_case(8200 + N, 8, 6000, 10000, N, K)
+    d = _run_nn(dg, cs, N)
+    valid_rows = np.nonzero(cs["mi"] >= 0)[0]
+    pm, pn = synth.sample_points(8300 + N, valid_rows, N, 4096)
+    ref = np.empty(pm.size)
+    for g in range(8):
+        sel = cs["mi"][pm] == g
+        # the oracle's NN call equals its NT call on the transposed weights
+        ref[sel] = oracle.gemm_points(cs["qa"], cs["ea"], cs["qb"][g], cs["eb"][g], pm[sel], pn[sel], c=cs["c"])
+    check_close(d[pm, pn], ref, f"nn contiguous {N}x{K}")
+
+
+# --------------------------------------- K-grouped TN (weight gradient)
+
+def _tn_case(seed, M, N, ks, with_c=True, tail=0):
+    """A [Kt, M], B [Kt, N] e4m3, each quantised 1x128 along K (per column),
+    Kt = sum(ks) + tail."""
+    ks = np.asarray(ks, np.int32)
+    Kt = int(ks.sum()) + tail
+    qaT, ea = oracle.quantize_fp8(synth.normal_f32(seed, (M, Kt)), 1) if Kt else (np.zeros((M, 0), np.uint8),
+                                                                                  np.zeros((M, 0), np.uint8))
+    qbT, eb = oracle.quantize_fp8(synth.normal_f32(seed + 1, (N, Kt)), 1) if Kt else (np.zeros((N, 0), np.uint8),
+                                                                                      np.zeros((N, 0), np.uint8))
+    G = ks.size
+    return dict(ks=ks, Kt=Kt, M=M, N=N, G=G, qa=np.ascontiguousarray(qaT.T), ea=ea,
+                qb=np.ascontiguousarray(qbT.T), eb=eb,
+                sfa=oracle.pack_sf(ea, M) if Kt else np.zeros(128, np.int32),
+                sfb=oracle.pack_sf(eb, N) if Kt else np.zeros(128, np.int32),
+                c=synth.normal_bf16_bits(seed + 2, (G, M, N)) if with_c else None)
+
+
+def _run_tn(dg, cs, in_place=False):
+    G, M, N = cs["G"], cs["M"], cs["N"]
+    a = dev(cs["qa"]) if cs["Kt"] else torch.zeros((1, M), dtype=torch.uint8, device="cuda")
+    b = dev(cs["qb"]) if cs["Kt"] else torch.zeros((1, N), dtype=torch.uint8, device="cuda")
+    if in_place:
+        d = dev(cs["c"].view(np.int16))
+        c = d
+    else:
+        d = torch.full((G, M, N), 0x7FC1, dtype=torch.int16, device="cuda")
+        c = dev(cs["c"].view(np.int16)) if cs["c"] is not None else None
+    fn = dg.dg_k_grouped_fp8_gemm_tn_contiguous
+    if cs["Kt"]:
+        fn(a, dev(cs["sfa"]), b, dev(cs["sfb"]), c, d, dev(cs["ks"]))
+    else:  # k_total = 0: the binding reads it from a's rows, so call the C ABI directly
+        import ctypes
+        st = dg.lib().dg_k_grouped_fp8_gemm_tn_contiguous(
+            ctypes.c_void_p(a.data_ptr()), ctypes.c_void_p(dev(cs["sfa"]).data_ptr()), ctypes.c_void_p(b.data_ptr()),
+            ctypes.c_void_p(dev(cs["sfb"]).data_ptr()), ctypes.c_void_p(c.data_ptr()) if c is not None else None,
+            ctypes.c_void_p(d.data_ptr()), ctypes.c_void_p(dev(cs["ks"]).data_ptr()), G, M, N, 0, None)
+        assert st == 0
+    torch.cuda.synchronize()
+    return bf16_dev_to_f64(d)
+
+
+def _tn_ref(cs):
+    return oracle.gemm_k_grouped_tn(cs["qa"], cs["ea"], cs["qb"], cs["eb"], cs["ks"], c=cs["c"])
+
+
+@pytest.mark.parametrize("bn", [0, 128, 256])
+@pytest.mark.parametrize("M,N", [(256, 384), (144, 208), (128, 112)])
+def test_k_grouped_tn_matches_oracle(dg, bn, M, N):
+    cs = _tn_case(9000 + M + N, M, N, [256, 0, 384, 128, 640], tail=128)
+    dg.dg_set_tile_config(bn, 0)
+    try:
+        d = _run_tn(dg, cs)
+    finally:
+        dg.dg_set_tile_config(0, 0)
+    check_close(d, _tn_ref(cs), f"k-grouped tn {M}x{N} bn={bn}")
+
+
+def test_k_grouped_tn_without_c_and_in_place(dg):
+    cs = _tn_case(9100, 160, 256, [128, 512, 0])
+    ref = _tn_ref(cs)
+    check_close(_run_tn(dg, cs, in_place=True), ref, "tn in place")
+    cs0 = dict(cs, c=None)
+    d = _run_tn(dg, cs0)
+    check_close(d, _tn_ref(cs0), "tn C = 0")
+    assert np.all(d[2] == 0.0)                       # empty group, no C: zeros
+
+
+def test_k_grouped_tn_all_groups_empty(dg):
+    cs = _tn_case(9200, 128, 128, [0, 0])
+    d = _run_tn(dg, cs)
+    assert np.array_equal(d, cs["c"].view(ml_dtypes_bf16()).astype(np.float64))
+
+
+def ml_dtypes_bf16():
+    import ml_dtypes
+    return ml_dtypes.bfloat16
+
+
+def test_k_grouped_tn_bad_sizes_are_reported(dg):
+    cs = _tn_case(9300, 128, 128, [256, 128])
+    bad = dict(cs, ks=np.array([256, 64], np.int32))     # 64 is not a multiple of 128
+    _run_tn(dg, bad)
+    assert dg.dg_get_last_error() == -5
+    over = dict(cs, ks=np.array([256, 256], np.int32))   # sum beyond k_total
+    _run_tn(dg, over)
+    assert dg.dg_get_last_error() == -5
+
+
+def test_k_grouped_tn_full_size_sampled(dg):
+    # weight gradient of the (N, K) = (4096, 7168) projection over 8 experts
+    # of ~6000-10000 tokens each: D[g] [4096, 7168]
+    M, N = 4096, 7168
+    ks = synth.k_grouped_sizes(9400, 8, 6000, 10000)
+    cs = _tn_case(9401, M, N, ks)
+    d = _run_tn(dg, cs)
+    r = synth.rng(9402)
+    pg, pi, pj = r.integers(0, 8, 2048), r.integers(0, M, 2048), r.integers(0, N, 2048)
+    ref = oracle.gemm_k_grouped_tn_points(cs["qa"], cs["ea"], cs["qb"], cs["eb"], cs["ks"], pg, pi, pj, c=cs["c"])
+    check_close(d[pg, pi, pj], ref, "k-grouped tn full size")

@@ -436,3 +436,148 @@ def test_bf16_gemm_brute_force():
             for kk in range(70):
                 s += float(av[i, kk]) * float(bv[j, kk])
             assert abs(got[i, j] - s) <= 1e-12 * (1 + abs(s))
+
+
+# ---- NN contiguous and K-grouped TN (the layouts whose B, or A and B, are
+# stored with K as the row index)
+
+def _deq_b_nn(bkn, sfb):
+    """B stored [K][N] with 128x128 block codes sfb [ceil(N/128)][K/128],
+    dequantised as a [K][N] array (independent of the oracle)."""
+    K, N = bkn.shape
+    v = bkn.view(E4M3_DT).astype(np.float64)
+    s = sfb.view(E8M0_DT).astype(np.float64)          # [n-block][k-block]
+    return v * np.repeat(np.repeat(s.T, 128, axis=0), 128, axis=1)[:K, :N]
+
+
+def test_nn_contiguous_vs_numpy_and_skips_padding():
+    G, N, K = 3, 200, 384                              # N is not a multiple of 128
+    rows, mi = synth.contiguous_layout(70, G, 20, 150)
+    M = mi.size
+    a = _finite_codes(71, (M, K))
+    a[mi < 0] = 0x7F
+    sfa = _scales(72, (M, 3))
+    b = np.stack([_finite_codes(73 + g, (K, N)) for g in range(G)])
+    sfb = np.stack([_scales(80 + g, (2, 3)) for g in range(G)])
+    c = synth.normal_bf16_bits(90, (M, N))
+    prior = np.full((M, N), -7.0)
+    d = oracle.gemm_nn_contiguous(a, sfa, b, sfb, mi, c=c, out=prior)
+    assert np.all(d[mi < 0] == -7.0)
+    cd = c.view(ml_dtypes.bfloat16).astype(np.float64)
+    for g in range(G):
+        sel = np.nonzero(mi == g)[0]
+        assert sel.size == rows[g]
+        want = cd[sel] + _deq_a(a[sel], sfa[sel]) @ _deq_b_nn(b[g], sfb[g])
+        np.testing.assert_allclose(d[sel], want, rtol=1e-12, atol=1e-300)
+
+
+def test_nn_contiguous_equals_nt_on_the_transposed_weights():
+    # the same products in the same order: bit-identical
+    G, N, K = 2, 136, 256
+    rows, mi = synth.contiguous_layout(91, G, 10, 140)
+    M = mi.size
+    a, sfa = _finite_codes(92, (M, K)), _scales(93, (M, 2))
+    b_nk = np.stack([_finite_codes(94 + g, (N, K)) for g in range(G)])
+    sfb = np.stack([_scales(96 + g, (2, 2)) for g in range(G)])
+    nt = oracle.gemm_contiguous(a, sfa, b_nk, sfb, mi)
+    nn = oracle.gemm_nn_contiguous(a, sfa, np.ascontiguousarray(b_nk.transpose(0, 2, 1)), sfb, mi)
+    assert np.array_equal(np.isnan(nt), np.isnan(nn))
+    assert np.array_equal(nt[mi >= 0], nn[mi >= 0])
+
+
+def test_nn_single_nonzero_lands_at_its_index():
+    M, N, K = 128, 260, 512
+    mi = np.zeros(M, np.int32)
+    a = np.zeros((M, K), np.uint8)
+    b = np.zeros((1, K, N), np.uint8)
+    a[2, 300] = 0x40      # 2.0
+    b[0, 300, 257] = 0xC4  # -3.0 at k = 300, n = 257
+    sfa = np.full((M, 4), 127, np.uint8)
+    sfb = np.full((1, 3, 4), 127, np.uint8)
+    sfa[2, 2] = 130       # 2^3 on K-block 2
+    sfb[0, 2, 2] = 125    # 2^-2 on B's block (n-block 2, K-block 2)
+    d = oracle.gemm_nn_contiguous(a, sfa, b, sfb, mi)
+    want = np.zeros((M, N))
+    want[2, 257] = 2.0 * -3.0 * 8.0 * 0.25
+    assert np.array_equal(d, want)
+
+
+def _deq_kmajor_cols(x, sf):
+    """x [Kt][R] codes with one code per (column r, 128-row block of K):
+    sf [R][Kt/128]; dequantised [Kt][R]."""
+    v = x.view(E4M3_DT).astype(np.float64)
+    s = sf.view(E8M0_DT).astype(np.float64)
+    return v * np.repeat(s.T, 128, axis=0)
+
+
+def test_k_grouped_tn_vs_numpy_with_an_empty_group():
+    M, N = 136, 200
+    ks = np.array([256, 0, 128, 384], np.int32)
+    Kt = int(ks.sum()) + 128                            # unused tail rows
+    a, b = _finite_codes(100, (Kt, M)), _finite_codes(101, (Kt, N))
+    sfa, sfb = _scales(102, (M, Kt // 128)), _scales(103, (N, Kt // 128))
+    c = synth.normal_bf16_bits(104, (ks.size, M, N))
+    d = oracle.gemm_k_grouped_tn(a, sfa, b, sfb, ks, c=c)
+    cd = c.view(ml_dtypes.bfloat16).astype(np.float64)
+    da, db = _deq_kmajor_cols(a, sfa), _deq_kmajor_cols(b, sfb)
+    k0 = 0
+    for g, kk in enumerate(ks):
+        want = cd[g] + da[k0:k0 + kk].T @ db[k0:k0 + kk]
+        np.testing.assert_allclose(d[g], want, rtol=1e-12, atol=1e-300)
+        k0 += kk
+    assert np.array_equal(d[1], cd[1])                 # empty group: C exactly
+    assert np.array_equal(oracle.gemm_k_grouped_tn(a, sfa, b, sfb, ks)[1], np.zeros((M, N)))
+
+
+def test_k_grouped_tn_single_nonzero_lands_in_its_group():
+    M, N = 40, 150
+    ks = np.array([256, 384], np.int32)                 # k = 300 is group 1, its K-block 2
+    Kt = 640
+    a = np.zeros((Kt, M), np.uint8)
+    b = np.zeros((Kt, N), np.uint8)
+    a[300, 5] = 0x40       # 2.0
+    b[300, 130] = 0xC4     # -3.0
+    sfa = np.full((M, 5), 127, np.uint8)
+    sfb = np.full((N, 5), 127, np.uint8)
+    sfa[5, 2] = 131        # 2^4
+    sfb[130, 2] = 124      # 2^-3
+    sfb[131, 2] = 140      # a neighbour's scale must not leak
+    d = oracle.gemm_k_grouped_tn(a, sfa, b, sfb, ks)
+    want = np.zeros((2, M, N))
+    want[1, 5, 130] = 2.0 * -3.0 * 16.0 * 0.125
+    assert np.array_equal(d, want)
+
+
+def test_k_grouped_tn_scale_bump_adds_exactly_one_block():
+    M, N = 6, 130
+    ks = np.array([128, 384], np.int32)
+    Kt = 512
+    a = np.where(synth.junk_bytes(110, (Kt, M)) < 128, 0x38, 0xB0).astype(np.uint8)   # +-1, -0.5
+    b = np.where(synth.junk_bytes(111, (Kt, N)) < 128, 0x40, 0xA8).astype(np.uint8)   # 2, -0.25
+    sfa, sfb = _scales(112, (M, 4)), _scales(113, (N, 4))
+    base = oracle.gemm_k_grouped_tn(a, sfa, b, sfb, ks)
+    for kb in range(4):
+        g = 0 if kb == 0 else 1
+        only = np.zeros_like(a)
+        only[kb * 128:(kb + 1) * 128] = a[kb * 128:(kb + 1) * 128]
+        block = oracle.gemm_k_grouped_tn(only, sfa, b, sfb, ks)
+        bumped = sfa.copy()
+        bumped[3, kb] += 1
+        d = oracle.gemm_k_grouped_tn(a, bumped, b, sfb, ks)
+        assert np.array_equal(d[g, 3], base[g, 3] + block[g, 3])
+        assert np.array_equal(d[1 - g], base[1 - g])
+        assert np.array_equal(np.delete(d[g], 3, axis=0), np.delete(base[g], 3, axis=0))
+
+
+def test_k_grouped_tn_points_match_the_full_reference():
+    M, N = 48, 160
+    ks = np.array([128, 256, 0, 128], np.int32)
+    Kt = 512
+    a, b = _finite_codes(120, (Kt, M)), _finite_codes(121, (Kt, N))
+    sfa, sfb = _scales(122, (M, 4)), _scales(123, (N, 4))
+    c = synth.normal_bf16_bits(124, (4, M, N))
+    full = oracle.gemm_k_grouped_tn(a, sfa, b, sfb, ks, c=c)
+    r = synth.rng(125)
+    pg, pi, pj = r.integers(0, 4, 300), r.integers(0, M, 300), r.integers(0, N, 300)
+    pts = oracle.gemm_k_grouped_tn_points(a, sfa, b, sfb, ks, pg, pi, pj, c=c)
+    assert np.array_equal(pts, full[pg, pi, pj])
