@@ -58,7 +58,8 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--shape", default=None, help="run one M,N,K shape instead of the sweep")
     ap.add_argument("--workload", default="dense",
-                    choices=["dense", "contiguous", "masked", "fp4", "moe_decode_fp4", "bf16"],
+                    choices=["dense", "contiguous", "masked", "fp4", "moe_decode_fp4", "bf16", "nn_contiguous",
+                             "kgrouped_tn"],
                     help="dense: the DeepSeek-V3 dense sweep (default); contiguous / masked / fp4: the "
                          "M-grouped prefill, masked decode and FP8 x FP4 cases, one JSON line each")
     ap.add_argument("--graph", action="store_true",
@@ -249,7 +250,7 @@ def grouped_cases(dg, torch, workload, gen, seed):
     rng = np.random.default_rng(seed)
     cases = []
 
-    def contiguous(n, k, fp4):
+    def contiguous(n, k, fp4, nn=False):
         rows = rng.integers(CONTIG_ROWS[0], CONTIG_ROWS[1] + 1, CONTIG_GROUPS)
         mi = np.concatenate([np.concatenate([np.full(r, g, np.int32), np.full(-r % 128, -1, np.int32)])
                              for g, r in enumerate(rows)])
@@ -259,14 +260,52 @@ def grouped_cases(dg, torch, workload, gen, seed):
         d = torch.empty((m_total, n), dtype=torch.bfloat16, device="cuda")
         t_mi = torch.from_numpy(mi).cuda()
         fn = dg.dg_m_grouped_fp8_fp4_gemm_nt_contiguous if fp4 else dg.dg_m_grouped_fp8_gemm_nt_contiguous
+        if nn:
+            # the same weights stored [G][K][N] (not transposed)
+            b = b.transpose(1, 2).contiguous()
+            fn = dg.dg_m_grouped_fp8_gemm_nn_contiguous
         bb = CONTIG_GROUPS * n * k // (2 if fp4 else 1)
         by = valid * k + bb + 2 * valid * n + (sfa.numel() + sfb.numel()) * 4 + 4 * m_total
-        name = f"contiguous{'-fp4' if fp4 else ''} G={CONTIG_GROUPS} M={m_total} ({valid} valid) N={n} K={k}"
+        kind = "nn-contiguous" if nn else "contiguous"
+        name = f"{kind}{'-fp4' if fp4 else ''} G={CONTIG_GROUPS} M={m_total} ({valid} valid) N={n} K={k}"
         cases.append((name, lambda: fn(a, sfa, b, sfb, None, d, t_mi), 2.0 * valid * n * k, by))
 
     if workload == "contiguous":
         for (n, k) in GROUPED_NK:
             contiguous(n, k, False)
+    elif workload == "nn_contiguous":
+        for (n, k) in GROUPED_NK:
+            contiguous(n, k, False, nn=True)
+    elif workload == "kgrouped_tn":
+        # weight gradient of the contiguous configuration's projections:
+        # forward D[tokens, n] = X[tokens, k] W[n, k]^T per expert, so
+        # dW[g] [n, k] = dY_g^T X_g, K-grouped over the 8 experts' tokens
+        # (U[6000, 10000] per expert, padded to 128); dY and X quantised 1x128
+        # along the token axis (one scale per column and 128 tokens)
+        for (n, k) in GROUPED_NK:
+            toks = rng.integers(CONTIG_ROWS[0], CONTIG_ROWS[1] + 1, CONTIG_GROUPS)
+            ks = ((toks + 127) // 128 * 128).astype(np.int32)
+            kt = int(ks.sum())
+
+            def col_quant(cols):
+                x = torch.randn((cols, kt), generator=gen, device="cuda", dtype=torch.float32)
+                q = torch.empty((cols, kt), dtype=torch.uint8, device="cuda")
+                e = torch.empty((cols, kt // 128), dtype=torch.uint8, device="cuda")
+                dg.dg_quantize_fp8(x, q, e, 1)
+                del x
+                sf = torch.empty(dg.dg_packed_sf_words(cols, kt // 128), dtype=torch.int32, device="cuda")
+                dg.dg_pack_sf(e, cols, sf, row_div=1)
+                return q.t().contiguous(), sf
+
+            a, sfa = col_quant(n)
+            b, sfb = col_quant(k)
+            d = torch.empty((CONTIG_GROUPS, n, k), dtype=torch.bfloat16, device="cuda")
+            t_ks = torch.from_numpy(ks).cuda()
+            by = kt * n + kt * k + 2 * CONTIG_GROUPS * n * k + (sfa.numel() + sfb.numel()) * 4
+            name = f"k-grouped-tn G={CONTIG_GROUPS} K={kt} M={n} N={k}"
+            cases.append((name, (lambda a=a, sfa=sfa, b=b, sfb=sfb, d=d, t_ks=t_ks:
+                                 dg.dg_k_grouped_fp8_gemm_tn_contiguous(a, sfa, b, sfb, None, d, t_ks)),
+                          2.0 * kt * n * k, by))
     elif workload == "masked":
         G, max_m = MASKED_GROUPS, MASKED_MAX_M
         for (n, k) in GROUPED_NK:
