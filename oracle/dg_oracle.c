@@ -289,6 +289,17 @@ static double dot_range(const operand_t* A, int64_t m, const operand_t* B, int64
                         int64_t k_end) {
     int64_t step = A->sf_k < B->sf_k ? A->sf_k : B->sf_k;
     double acc = 0;
+    if (!A->fp4 && !B->fp4 && A->k_stride == 1 && B->k_stride == 1) {
+        /* both rows contiguous along K: the same sums, read as two byte rows */
+        const uint8_t* ra = A->codes + m * A->row_stride;
+        const uint8_t* rb = B->codes + n * B->row_stride;
+        for (int64_t k0 = k_begin; k0 < k_end; k0 += step) {
+            double part = 0;
+            for (int64_t k = k0; k < k0 + step; ++k) part += E4M3[ra[k]] * E4M3[rb[k]];
+            acc += scale(A, m, k0) * scale(B, n, k0) * part;
+        }
+        return acc;
+    }
     for (int64_t k0 = k_begin; k0 < k_end; k0 += step) {
         double part = 0;
         for (int64_t k = k0; k < k0 + step; ++k) part += elem(A, m, k) * elem(B, n, k);
