@@ -50,7 +50,7 @@
  *
  * Scratch memory.  When the host heuristic shares the K-iterations of some
  * tiles out over several CTAs (stream-K: small M, or the last partial wave of
- * tiles), dg_fp8_gemm_nt keeps their FP32 partial sums in a workspace per
+ * tiles), the dense calls keep their FP32 partial sums in a workspace per
  * (device, stream), allocated stream-ordered on first use and grown on
  * demand; dg_shutdown() releases it.  No other call allocates device memory.
  */
@@ -90,6 +90,26 @@ typedef enum {
  * Requires m >= 0, n > 0 and n % 8 == 0, k > 0 and k % 128 == 0.  m == 0 is a
  * no-op.  Source: zhouruolin.cn guide, section 五, "非分组 FP8 GEMM". */
 dg_status dg_fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                         const void* c, void* d, int m, int n, int k, void* stream);
+
+/* Dense FP8 GEMM in the other three storage layouts (the guide, section 五:
+ * SM100 takes all of NT, TN, NN and TT).  The first letter names A's storage,
+ * the second B's, relative to D = A * B with A [m][k] and B [k][n]:
+ *   dg_fp8_gemm_nn   a e4m3 [m][k] (k contiguous), b e4m3 [k][n] (n contiguous)
+ *   dg_fp8_gemm_tn   a e4m3 [k][m] (m contiguous), b e4m3 [k][n]
+ *   dg_fp8_gemm_tt   a e4m3 [k][m],                b e4m3 [n][k] (as the NT call)
+ * The scales do not depend on the storage: sfa as for dg_fp8_gemm_nt (R = m,
+ * one code per row of D and 128-block of K), sfb as for dg_fp8_gemm_nt (the
+ * 128x128 block codes of B, block (n/128, k/128), expanded per n).  c, d, the
+ * result, the requirements and the errors are those of dg_fp8_gemm_nt, plus
+ * m % 16 == 0 when A is stored [k][m] and n % 16 == 0 when B is stored [k][n]
+ * (those rows are m or n bytes).  Operands stored with k as the row index are
+ * staged MN-major and the tiles are 128 or 256 columns wide. */
+dg_status dg_fp8_gemm_nn(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                         const void* c, void* d, int m, int n, int k, void* stream);
+dg_status dg_fp8_gemm_tn(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                         const void* c, void* d, int m, int n, int k, void* stream);
+dg_status dg_fp8_gemm_tt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
                          const void* c, void* d, int m, int n, int k, void* stream);
 
 /* M-grouped contiguous FP8 GEMM (MoE prefill / training forward): the rows of

@@ -21,7 +21,8 @@ __all__ = [
     "DGError", "lib", "dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
     "dg_m_grouped_fp8_gemm_nt_masked", "dg_m_grouped_fp8_fp4_gemm_nt_masked",
     "dg_m_grouped_fp8_gemm_nt_masked_swiglu", "dg_m_grouped_fp8_fp4_gemm_nt_masked_swiglu", "dg_fp8_gemm_nt_noalloc", "dg_noalloc_scratch_bytes", "dg_fp8_fp4_gemm_nt", "dg_bf16_gemm_nt", "dg_m_grouped_fp8_fp4_gemm_nt_contiguous",
-    "dg_m_grouped_fp8_gemm_nn_contiguous", "dg_k_grouped_fp8_gemm_tn_contiguous",
+    "dg_m_grouped_fp8_gemm_nn_contiguous", "dg_k_grouped_fp8_gemm_tn_contiguous", "dg_fp8_gemm_nn",
+    "dg_fp8_gemm_tn", "dg_fp8_gemm_tt",
     "dg_quantize_fp8", "dg_quantize_fp4", "dg_pack_sf", "dg_packed_sf_words", "dg_get_num_sms",
     "dg_set_num_sms", "dg_set_pdl", "dg_get_pdl", "dg_set_tile_config", "dg_get_mk_alignment_for_contiguous_layout", "dg_get_last_error",
     "dg_debug_starved_wait", "dg_launch_count", "dg_query_dense_config", "dg_num_tiles", "dg_debug_fastdiv", "dg_shutdown",
@@ -45,6 +46,9 @@ SYMBOLS = {
     "dg_m_grouped_fp8_fp4_gemm_nt_masked_swiglu": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _I32P, _INT, _INT, _INT, _INT,
                                                           _INT, _VP]),
     "dg_fp8_gemm_nt_noalloc": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _INT, _INT, _INT, _VP]),
+    "dg_fp8_gemm_nn": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _INT, _INT, _INT, _VP]),
+    "dg_fp8_gemm_tn": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _INT, _INT, _INT, _VP]),
+    "dg_fp8_gemm_tt": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _INT, _INT, _INT, _VP]),
     "dg_noalloc_scratch_bytes": (ctypes.c_size_t, []),
     "dg_fp8_fp4_gemm_nt": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _INT, _INT, _INT, _VP]),
     "dg_bf16_gemm_nt": (_INT, [_VP, _VP, _VP, _VP, _INT, _INT, _INT, _VP]),
@@ -146,6 +150,27 @@ def dg_fp8_gemm_nt_noalloc(a, sfa, b, sfb, c, d, stream=None) -> None:
 
 def dg_noalloc_scratch_bytes() -> int:
     return int(lib().dg_noalloc_scratch_bytes())
+
+
+def _dense_layout_call(name, a_mn, b_mn, a, sfa, b, sfb, c, d, stream):
+    k, m = a.shape if a_mn else (a.shape[1], a.shape[0])
+    n = b.shape[1] if b_mn else b.shape[0]
+    _check(getattr(lib(), name)(_p(a), _p(sfa), _p(b), _p(sfb), _p(c), _p(d), m, n, k, _stream(stream)), name)
+
+
+def dg_fp8_gemm_nn(a, sfa, b, sfb, c, d, stream=None) -> None:
+    """a: e4m3 [m, k]; b: e4m3 [k, n] (not transposed); sfa / sfb as for dg_fp8_gemm_nt."""
+    _dense_layout_call("dg_fp8_gemm_nn", False, True, a, sfa, b, sfb, c, d, stream)
+
+
+def dg_fp8_gemm_tn(a, sfa, b, sfb, c, d, stream=None) -> None:
+    """a: e4m3 [k, m] (A stored transposed); b: e4m3 [k, n]."""
+    _dense_layout_call("dg_fp8_gemm_tn", True, True, a, sfa, b, sfb, c, d, stream)
+
+
+def dg_fp8_gemm_tt(a, sfa, b, sfb, c, d, stream=None) -> None:
+    """a: e4m3 [k, m]; b: e4m3 [n, k] (as for dg_fp8_gemm_nt)."""
+    _dense_layout_call("dg_fp8_gemm_tt", True, False, a, sfa, b, sfb, c, d, stream)
 
 
 def dg_fp8_fp4_gemm_nt(a, sfa, b, sfb, c, d, stream=None) -> None:

@@ -413,6 +413,9 @@ struct Problem {
 // caller-provided device buffer instead of the per-stream workspace, and the
 // planner only considers plans that fit in fixed_ws_bytes (whole tiles
 // always do).
+// mean K of a k-grouped call's groups (the planner's K), at least one block
+int k_plan_mn(const Problem& p) { return std::max(128, (int)(p.k / p.groups) / 128 * 128); }
+
 template <bool FP4, int LAYOUT, int EPI = dg::kEpiPlain, bool BF16 = false, int MAJ = dg::kMajorK>
 dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, size_t fixed_ws_bytes = 0) {
   constexpr bool kAMn = (MAJ & dg::kAMajorMN) != 0;
@@ -432,11 +435,11 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
     plan.grid = (int)std::min<long long>((long long)p.groups * m_blocks * ceil_div(p.n, plan.bn), sms);
   } else if (LAYOUT == dg::kKGrouped) {
     // every group has the same tiles; planned at the mean K of a group
-    const int k_mean = std::max(128, (int)(p.k / p.groups) / 128 * 128);
-    plan = plan_gemm((long long)p.groups * m_blocks, p.n, k_mean, sms, false, 0, false, false, kBMn);
+    plan = plan_gemm((long long)p.groups * m_blocks, p.n, k_plan_mn(p), sms, false, 0, false, false, true);
   } else {
+    // MN-major operands run in 128- and 256-wide tiles only
     plan = plan_gemm(m_blocks, p.n, k_plan, sms, LAYOUT == dg::kDense, fixed_ws != nullptr ? fixed_ws_bytes : 0, FP4,
-                     BF16, kBMn);
+                     BF16, MAJ != dg::kMajorK);
   }
   if (plan.grid <= 0) return DG_ERR_UNSUPPORTED;  // (a forced width this layout cannot use)
 
@@ -648,6 +651,37 @@ dg_status dg_bf16_gemm_nt(const void* a, const void* b, const void* c, void* d, 
   if (m == 0) return DG_OK;
   Problem p{a, nullptr, b, nullptr, c, d, nullptr, nullptr, m, n, k, 1, 0};
   return run_gemm<false, dg::kDense, dg::kEpiPlain, true>(p, static_cast<cudaStream_t>(stream));
+}
+
+// Dense FP8 GEMM with A and / or B stored with K as the row index.
+static dg_status dense_layout_impl(bool a_mn, bool b_mn, const void* a, const int32_t* sfa, const void* b,
+                                   const int32_t* sfb, const void* c, void* d, int m, int n, int k, void* stream) {
+  if (m < 0) return DG_ERR_INVALID_ARG;
+  dg_status st = check_common(a, sfa, b, sfb, c, d, n, k);
+  if (st != DG_OK) return st;
+  // the rows of an MN-major operand are m or n bytes: 16-byte TMA row stride
+  if ((a_mn && m % 16 != 0) || (b_mn && n % 16 != 0)) return DG_ERR_INVALID_ARG;
+  if (m == 0) return DG_OK;
+  Problem p{a, sfa, b, sfb, c, d, nullptr, nullptr, m, n, k, 1, 0};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (a_mn && b_mn) return run_gemm<false, dg::kDense, dg::kEpiPlain, false, dg::kAMajorMN | dg::kBMajorMN>(p, s);
+  if (a_mn) return run_gemm<false, dg::kDense, dg::kEpiPlain, false, dg::kAMajorMN>(p, s);
+  return run_gemm<false, dg::kDense, dg::kEpiPlain, false, dg::kBMajorMN>(p, s);
+}
+
+dg_status dg_fp8_gemm_nn(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, const void* c, void* d,
+                         int m, int n, int k, void* stream) {
+  return dense_layout_impl(false, true, a, sfa, b, sfb, c, d, m, n, k, stream);
+}
+
+dg_status dg_fp8_gemm_tn(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, const void* c, void* d,
+                         int m, int n, int k, void* stream) {
+  return dense_layout_impl(true, true, a, sfa, b, sfb, c, d, m, n, k, stream);
+}
+
+dg_status dg_fp8_gemm_tt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, const void* c, void* d,
+                         int m, int n, int k, void* stream) {
+  return dense_layout_impl(true, false, a, sfa, b, sfb, c, d, m, n, k, stream);
 }
 
 dg_status dg_fp8_fp4_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, const void* c,

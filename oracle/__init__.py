@@ -212,6 +212,23 @@ def gemm_masked(a, sfa, b, sfb, masked_m, b_fp4=False, out=None) -> np.ndarray:
     return res
 
 
+def gemm_layout(a, sfa, b, sfb, layout: str, c=None) -> np.ndarray:
+    """Dense FP8 reference in one of the layouts "nt", "nn", "tn", "tt": the
+    first letter is A ("n": [M, K], "t": stored [K, M]), the second B ("t":
+    [N, K], "n": stored [K, N]).  sfa [M, K/128], sfb [ceil(N/128), K/128]
+    whatever the storage.  Float64 [M, N]."""
+    assert layout in ("nt", "nn", "tn", "tt")
+    a_mn, b_mn = layout[0] == "t", layout[1] == "n"
+    a, sfa, b, sfb, _, c = _gemm_args(a, sfa, b, sfb, False, c)
+    K, M = a.shape if a_mn else a.shape[::-1]
+    N = b.shape[1] if b_mn else b.shape[0]
+    assert (b.shape[0] if b_mn else b.shape[1]) == K
+    out = np.zeros((M, N), np.float64)
+    _load().or_gemm_layout(_p(a), _p(sfa), _p(b), _p(sfb), _p(c), ctypes.c_int(int(a_mn)), ctypes.c_int(int(b_mn)),
+                           I64(M), I64(N), I64(K), _p(out))
+    return out
+
+
 def gemm_nn_contiguous(a, sfa, b, sfb, m_indices, c=None, out=None) -> np.ndarray:
     """M-grouped contiguous reference with B not transposed (NN).
     b: e4m3 [G, K, N]; sfb: UE8M0 [G, ceil(N/128), K/128] (block (n/128,

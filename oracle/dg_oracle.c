@@ -485,3 +485,23 @@ void or_gemm_k_grouped_tn_points(const uint8_t* a, const uint8_t* sfa, const uin
         out[t] = base + dot_range(&A, i, &B, j, k0, k0 + ks[g]);
     }
 }
+
+/* Dense FP8 GEMM in any of the four storage layouts of A and B (NT, NN, TN,
+ * TT): a_mn = 1 stores A as [K][M] (else [M][K]); b_mn = 1 stores B as [K][N]
+ * (else [N][K]).  The scales do not depend on the storage: sfa [M][K/128]
+ * (1x128 along K), sfb [ceil(N/128)][K/128] (128x128 blocks).  out[m][n] =
+ * C[m][n] + sum_k ..., as or_gemm. */
+void or_gemm_layout(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb,
+                    const uint16_t* c, int a_mn, int b_mn, int64_t M, int64_t N, int64_t K, double* out) {
+    build_tables();
+    operand_t A, B;
+    make_ops(&A, &B, a, sfa, b, sfb, 0, K);
+    if (a_mn) { A.row_stride = 1; A.k_stride = M; }
+    if (b_mn) { B.row_stride = 1; B.k_stride = N; }
+#pragma omp parallel for schedule(dynamic)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double base = c ? bf16_bits_to_double(c[m * N + n]) : 0.0;
+            out[m * N + n] = base + dot(&A, m, &B, n, K);
+        }
+}

@@ -93,6 +93,12 @@ def test_invalid_arguments_rejected_on_host(dg):
     assert tn(p(fake), p(fake), p(fake), p(fake), None, p(fake), p(fake), 2, 128, 100, 256, None) == -1
     assert tn(p(fake), p(fake), p(fake), p(fake), None, p(fake), p(fake), 2, 128, 128, 200, None) == -1
     assert tn(p(fake + 8), p(fake), p(fake), p(fake), None, p(fake), p(fake), 2, 128, 128, 256, None) == -1
+    # dense NN / TN / TT: rows of an MN-major operand need m or n % 16 == 0
+    assert lib.dg_fp8_gemm_nn(p(fake), p(fake), p(fake), p(fake), None, p(fake), 128, 136, 128, None) == -1
+    assert lib.dg_fp8_gemm_tn(p(fake), p(fake), p(fake), p(fake), None, p(fake), 120, 128, 128, None) == -1
+    assert lib.dg_fp8_gemm_tn(p(fake), p(fake), p(fake), p(fake), None, p(fake), 128, 136, 128, None) == -1
+    assert lib.dg_fp8_gemm_tt(p(fake), p(fake), p(fake), p(fake), None, p(fake), 120, 136, 128, None) == -1
+    assert lib.dg_fp8_gemm_tt(p(fake), p(fake), p(fake), p(fake), None, p(fake), 0, 136, 128, None) == 0
     # quantiser: cols % 128, block_rows in {1, 128}
     assert lib.dg_quantize_fp8(p(fake), 4, 100, 1, p(fake), p(fake), None) == -1
     assert lib.dg_quantize_fp8(p(fake), 4, 128, 64, p(fake), p(fake), None) == -1

@@ -724,3 +724,46 @@ def test_k_grouped_tn_full_size_sampled(dg):
     pg, pi, pj = r.integers(0, 8, 2048), r.integers(0, M, 2048), r.integers(0, N, 2048)
     ref = oracle.gemm_k_grouped_tn_points(cs["qa"], cs["ea"], cs["qb"], cs["eb"], cs["ks"], pg, pi, pj, c=cs["c"])
     check_close(d[pg, pi, pj], ref, "k-grouped tn full size")
+
+
+# ------------------------------------- dense NN / TN / TT storage layouts
+
+def _run_dense_layout(dg, p, layout):
+    a = p.qa.T if layout[0] == "t" else p.qa          # A stored [K, M] for "t"
+    b = p.qb.T if layout[1] == "n" else p.qb          # B stored [K, N] for "n"
+    d = torch.empty((p.M, p.N), dtype=torch.int16, device="cuda")
+    c = dev(p.c.view(np.int16)) if p.c is not None else None
+    getattr(dg, f"dg_fp8_gemm_{layout}")(dev(a), dev(p.sfa), dev(b), dev(p.sfb), c, d)
+    torch.cuda.synchronize()
+    return bf16_dev_to_f64(d), a, b
+
+
+@pytest.mark.parametrize("layout", ["nn", "tn", "tt"])
+@pytest.mark.parametrize("bn,schedule,sms", [(0, 0, 0), (128, 1, 0), (256, 1, 0), (128, 2, 7), (256, 3, 7)])
+@pytest.mark.parametrize("M,N,K,with_c", [
+    (1104, 528, 512, True),     # ragged M and N tails
+    (304, 1008, 1536, True),    # shared pieces that start and end inside tiles
+    (128, 512, 128, False),     # one K-block
+])
+def test_dense_layouts_match_oracle(dg, layout, bn, schedule, sms, M, N, K, with_c):
+    dg.dg_set_num_sms(sms)
+    dg.dg_set_tile_config(bn, schedule)
+    try:
+        p = Dense(2800 + M + bn + schedule, M, N, K, with_c=with_c)
+        d, a, b = _run_dense_layout(dg, p, layout)
+        assert dg.dg_get_last_error() == 0
+    finally:
+        dg.dg_set_tile_config(0, 0)
+        dg.dg_set_num_sms(0)
+    ref = oracle.gemm_layout(np.ascontiguousarray(a), p.ea, np.ascontiguousarray(b), p.eb, layout, c=p.c)
+    check_close(d, ref, f"{layout} bn={bn} schedule={schedule} {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("layout", ["nn", "tn", "tt"])
+def test_dense_layouts_full_size_sampled(dg, layout):
+    M, N, K = 4096, 7168, 2048
+    p = Dense(2900, M, N, K, with_c=True)
+    d, _, _ = _run_dense_layout(dg, p, layout)
+    pm, pn = synth.sample_points(2901, np.arange(M), N, 2048)
+    # the oracle's layout calls equal its NT call on the logical operands
+    check_close(d[pm, pn], p.ref_points(pm, pn), f"{layout} {M}x{N}x{K}")

@@ -581,3 +581,39 @@ def test_k_grouped_tn_points_match_the_full_reference():
     pg, pi, pj = r.integers(0, 4, 300), r.integers(0, M, 300), r.integers(0, N, 300)
     pts = oracle.gemm_k_grouped_tn_points(a, sfa, b, sfb, ks, pg, pi, pj, c=c)
     assert np.array_equal(pts, full[pg, pi, pj])
+
+
+# ---- dense NT / NN / TN / TT storage layouts
+
+@pytest.mark.parametrize("layout", ["nt", "nn", "tn", "tt"])
+def test_gemm_layout_vs_numpy_and_nt_identity(layout):
+    M, N, K = 48, 200, 384
+    a, b = _finite_codes(130, (M, K)), _finite_codes(131, (N, K))   # logical [M, K], [N, K]
+    sfa, sfb = _scales(132, (M, 3)), _scales(133, (2, 3))
+    c = synth.normal_bf16_bits(134, (M, N))
+    sa = np.ascontiguousarray(a.T) if layout[0] == "t" else a
+    sb = np.ascontiguousarray(b.T) if layout[1] == "n" else b
+    d = oracle.gemm_layout(sa, sfa, sb, sfb, layout, c=c)
+    # the same products in the same order as the NT call on the logical operands
+    assert np.array_equal(d, oracle.gemm(a, sfa, b, sfb, c=c))
+    want = c.view(ml_dtypes.bfloat16).astype(np.float64) + _deq_a(a, sfa) @ _deq_b(b, sfb, N).T
+    np.testing.assert_allclose(d, want, rtol=1e-12, atol=1e-300)
+
+
+@pytest.mark.parametrize("layout", ["nn", "tn", "tt"])
+def test_gemm_layout_single_nonzero_lands_at_its_index(layout):
+    M, N, K = 20, 260, 512
+    a = np.zeros((M, K), np.uint8)
+    b = np.zeros((N, K), np.uint8)
+    a[7, 300] = 0x40       # 2.0
+    b[257, 300] = 0xC4     # -3.0
+    sfa = np.full((M, 4), 127, np.uint8)
+    sfb = np.full((3, 4), 127, np.uint8)
+    sfa[7, 2] = 130        # 2^3
+    sfb[2, 2] = 125        # 2^-2
+    sa = np.ascontiguousarray(a.T) if layout[0] == "t" else a
+    sb = np.ascontiguousarray(b.T) if layout[1] == "n" else b
+    d = oracle.gemm_layout(sa, sfa, sb, sfb, layout)
+    want = np.zeros((M, N))
+    want[7, 257] = 2.0 * -3.0 * 8.0 * 0.25
+    assert np.array_equal(d, want)
