@@ -77,6 +77,25 @@ def shapes_from(args):
     return [(m, n, k) for (n, k) in DENSE_NK for m in DENSE_M]
 
 
+# ---------------------------------------------------------------- ranks
+
+def max_over_ranks(x: float, use_dist: bool, device) -> float:
+    """The largest of x over all ranks (the slowest rank sets the job's time);
+    x itself when the run is not distributed.  Every rank calls it at the same
+    point, in the same order."""
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if use_dist:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world: int, flops_per_rank: float, ms_max: float) -> float:
+    """Whole-job throughput: every rank does flops_per_rank in a step whose
+    time is the maximum over ranks ("weak" scaling: work per GPU fixed)."""
+    return world * flops_per_rank / (ms_max * 1e-3) / 1e12
+
+
 def flops(m, n, k):
     return 2.0 * m * n * k
 
@@ -460,9 +479,7 @@ def run_grouped(args, dg, torch, rank, world, use_dist, local_rank):
         torch.cuda.synchronize()
         ref_ms = [sum(rev[s_][i][0].elapsed_time(rev[s_][i][1]) for s_ in range(args.steps)) / args.steps
                   if refs[i] is not None else None for i in range(len(cases))]
-    t = torch.tensor([sum(ms)], dtype=torch.float64, device="cuda")
-    if use_dist:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    step_ms_max = max_over_ranks(sum(ms), use_dist, "cuda")
     peaks, peak_kind = load_peaks()
     fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
     hbm = peaks["hbm_gbs"]
@@ -487,9 +504,9 @@ def run_grouped(args, dg, torch, rank, world, use_dist, local_rank):
                 "kernel": f"gemm_kernel on {pc['case']}",
                 "peak_source": f"{peak_kind}: FP8 = bf16 burst {peaks['bf16_tflops']} x {FP8_PER_BF16}; HBM {hbm} GB/s"}
     if rank == 0:
-        value = world * sum(c[2] for c in cases) / (float(t.item()) * 1e-3) / 1e12
+        value = whole_job_tflops(world, sum(c[2] for c in cases), step_ms_max)
         line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": round(float(t.item()), 4), "higher_is_better": True,
+                "warmup": args.warmup, "ms_per_step": round(step_ms_max, 4), "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
                 "config": {"workload": args.workload, "cases": len(cases), "cuda_graph": bool(args.graph),
                            "l2": "flushed before every timed call: 256 MB write then 256 MB read, not timed",
@@ -665,13 +682,10 @@ def main():
     per_shape_ms = [sum(events[s][i][0].elapsed_time(events[s][i][1]) for s in range(args.steps)) / args.steps
                     for i in range(len(shapes))]
     step_ms = sum(per_shape_ms)
-    t = torch.tensor([step_ms], dtype=torch.float64, device="cuda")
-    if use_dist:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    step_ms_max = float(t.item())
+    step_ms_max = max_over_ranks(step_ms, use_dist, "cuda")
 
     sweep_flops = sum(flops(*s) for s in shapes)
-    value = world * sweep_flops / (step_ms_max * 1e-3) / 1e12
+    value = whole_job_tflops(world, sweep_flops, step_ms_max)
 
     peaks, peak_kind = load_peaks()
     fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
@@ -736,12 +750,10 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         ems = e0.elapsed_time(e1) / e2e_steps
-        te = torch.tensor([ems], dtype=torch.float64, device="cuda")
-        if use_dist:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": round(world * sweep_flops / (float(te.item()) * 1e-3) / 1e12, 2), "unit": UNIT,
+        ems_max = max_over_ranks(ems, use_dist, "cuda")
+        e2e = {"value": round(whole_job_tflops(world, sweep_flops, ems_max), 2), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": round(float(te.item()), 3)}
+               "ms_per_step": round(ems_max, 3)}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
