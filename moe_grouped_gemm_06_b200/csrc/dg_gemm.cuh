@@ -1,6 +1,7 @@
 // dg_gemm.cuh -- the persistent, warp-specialised, block-scaled GEMM for sm_100a.
 //
-//   D = C + A * B^T   (A: M x K e4m3, B: N x K e4m3 or e2m1, both K-major;
+//   D = C + A * B^T   (A: M x K e4m3, B: N x K e4m3 or e2m1, K-major, or
+//                      either stored with K as the row index (MN-major);
 //                      C, D: bf16 row-major; FP32 accumulation in TMEM)
 //
 // with DeepSeek-V3 fine-grained scaling: one UE8M0 scale per 1x128 row-group
@@ -9,8 +10,9 @@
 // (fine-grained scaling), "优化技术" (persistent warp specialisation, TMA
 // loads/stores, unified block scheduler with L2 rasterisation, unaligned
 // block sizes); "DeepGEMM：统一高性能张量核心 GEMM 计算库编译与使用指南"
-// (zhouruolin.cn), section 五 (D = C + A @ B, NT layout, packed UE8M0 scales,
-// M-grouped contiguous and masked layouts); "DeepSeek 发布 DeepGEMM 重大更新"
+// (zhouruolin.cn), section 五 (D = C + A @ B, NT layout and on SM100 also TN,
+// NN and TT, packed UE8M0 scales, M-grouped contiguous and masked layouts,
+// the K-grouped weight-gradient layout); "DeepSeek 发布 DeepGEMM 重大更新"
 // (linlog.top), section "FP4 精度支持" (FP8 x FP4).
 //
 // Roles (320 threads, one CTA per SM, persistent over work units):
@@ -312,7 +314,7 @@ struct WorkIter {
 // tm_sfa / tm_sfb view the packed scale words as rows of 512 bytes so that
 // the peer's scale loads can complete on the leader's barrier.
 //
-// MAJ != kMajorK: A and/or B staged MN-major (TN / NN layouts): each 128-wide
+// MAJ != kMajorK: A and/or B staged MN-major (NN, TN, TT layouts): each 128-wide
 // M or N block of a stage is one TMA box of 128 elements x 128 K rows, and
 // the MMA reads it through an MN-major descriptor (plain FP8 tiles of width
 // 128 or 256 only).

@@ -409,13 +409,13 @@ struct Problem {
   const int32_t* ks = nullptr;  // k-grouped: K of each group (device)
 };
 
+// mean K of a k-grouped call's groups (the planner's K), at least one block
+int k_plan_mn(const Problem& p) { return std::max(128, (int)(p.k / p.groups) / 128 * 128); }
+
 // fixed_ws / fixed_ws_bytes: when given, stream-K partials go to this
 // caller-provided device buffer instead of the per-stream workspace, and the
 // planner only considers plans that fit in fixed_ws_bytes (whole tiles
 // always do).
-// mean K of a k-grouped call's groups (the planner's K), at least one block
-int k_plan_mn(const Problem& p) { return std::max(128, (int)(p.k / p.groups) / 128 * 128); }
-
 template <bool FP4, int LAYOUT, int EPI = dg::kEpiPlain, bool BF16 = false, int MAJ = dg::kMajorK>
 dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, size_t fixed_ws_bytes = 0) {
   constexpr bool kAMn = (MAJ & dg::kAMajorMN) != 0;
