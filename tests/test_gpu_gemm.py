@@ -94,6 +94,7 @@ def test_pack_sf_bit_exact(dg, rows, ng, row_div):
     (1100, 520, 512, True),     # several m-blocks, no split-K, ragged tails
     (64, 2112, 7168, True),     # stream-K over all SMs (17 tiles)
     (3, 64, 256, True),         # tiny M
+    (1, 136, 512, True),        # a single row (one partial 32-row store box)
 ])
 def test_dense_matches_oracle(dg, M, N, K, with_c):
     p = Dense(2000 + M + N, M, N, K, with_c=with_c).upload()
