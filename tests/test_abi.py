@@ -255,3 +255,21 @@ def test_fast_division_matches_integer_division(dg):
                 assert dg.lib().dg_debug_fastdiv(d, n) == n // d, (d, n)
     assert dg.lib().dg_debug_fastdiv(0, 5) == 0xFFFFFFFF
     assert dg.lib().dg_debug_fastdiv(3, 2 ** 31) == 0xFFFFFFFF
+
+
+def test_mn_major_layouts_refuse_widths_other_than_128_and_256(dg):
+    # MN-major operands are staged in 128-wide column blocks: a forced width
+    # of 192 has no plan and is refused on the host, before any launch
+    lib = dg.lib()
+    fake = 1 << 20
+    p = lambda v: __import__("ctypes").c_void_p(v)
+    dg.dg_set_num_sms(148)
+    dg.dg_set_tile_config(192, 0)
+    try:
+        for fn in (lib.dg_fp8_gemm_nn, lib.dg_fp8_gemm_tn, lib.dg_fp8_gemm_tt):
+            assert fn(p(fake), p(fake), p(fake), p(fake), None, p(fake), 256, 256, 256, None) == -2
+        assert lib.dg_k_grouped_fp8_gemm_tn_contiguous(p(fake), p(fake), p(fake), p(fake), None, p(fake), p(fake),
+                                                       2, 256, 256, 512, None) == -2
+    finally:
+        dg.dg_set_tile_config(0, 0)
+        dg.dg_set_num_sms(0)
