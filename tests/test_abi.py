@@ -273,3 +273,32 @@ def test_mn_major_layouts_refuse_widths_other_than_128_and_256(dg):
     finally:
         dg.dg_set_tile_config(0, 0)
         dg.dg_set_num_sms(0)
+
+
+def test_automatic_plans_cover_every_tile_once_on_random_shapes(dg):
+    # properties of the heuristic's own choice (no forced width or schedule)
+    # over seeded random dense shapes and SM counts
+    rng = __import__("numpy").random.default_rng(77)
+    try:
+        for _ in range(400):
+            m = int(rng.integers(1, 9000))
+            n = 8 * int(rng.integers(1, 5000))
+            k = 128 * int(rng.integers(1, 150))
+            sms = int(rng.choice([148, 132, 64, 7]))
+            dg.dg_set_num_sms(sms)
+            cfg = dg.dg_query_dense_config(m, n, k)
+            bn = cfg["block_n"]
+            assert bn in (64, 128, 192, 256), cfg
+            tiles = -(-m // 128) * -(-n // bn)
+            assert cfg["dp_tiles"] + cfg["sk_tiles"] == tiles, (m, n, k, sms, cfg)
+            assert 1 <= cfg["grid"] <= sms
+            if cfg["sk_tiles"] == 0:
+                assert cfg["grid"] == min(tiles, sms) and cfg["workspace_bytes"] == 0
+                continue
+            assert cfg["dp_tiles"] % cfg["grid"] == 0            # whole waves before the shared tail
+            if cfg["sk_split"] > 0:
+                assert cfg["sk_tiles"] * cfg["sk_split"] <= cfg["grid"] and 2 <= cfg["sk_split"] <= k // 128
+            else:
+                assert cfg["max_segments"] == _brute_force_segments(cfg["sk_tiles"], k // 128, cfg["grid"])
+    finally:
+        dg.dg_set_num_sms(0)
