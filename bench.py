@@ -24,6 +24,14 @@ runs the full sweep on its own GPU and value aggregates all ranks ("weak").
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                   [--shape M,N,K] [--no-e2e] [--no-cpu]
+                  [--workload dense | contiguous | nn_contiguous | kgrouped_tn | masked
+                              | fp4 | moe_decode_fp4 | bf16] [--graph]
+
+The default workload (dense) is the headline line.  The others time each case
+alone after an L2 flush and report per-case TFLOPS and roofline fractions:
+MoE prefill (contiguous, NT and NN), the MoE weight gradient (K-grouped TN),
+decode (masked, plain or as a CUDA graph with --graph), FP8 x FP4, the FP8 x
+FP4 decode step with SwiGLU, and BF16 against cuBLAS.
 """
 from __future__ import annotations
 
