@@ -56,6 +56,7 @@ FLUSH_BYTES = 256 << 20
 HOLD_CYCLES = 6_000_000  # ~3 ms at 2 GHz: longer than the host needs to enqueue one step
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_PER_BF16 = 2.0  # nominal dense FP8 : BF16 tensor throughput (4.5 : 2.25 PFLOP/s)
+FP8_SPEC_TFLOPS = 4500.0  # nominal dense FP8 peak of one B200
 
 
 def parse_args():
@@ -74,6 +75,8 @@ def parse_args():
                     help="grouped workloads: capture each case's call in a CUDA graph and time its replay")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="time the dense sweep only (skip the grouped, decode and FP8 x FP4 cases)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     return ap.parse_args()
 
@@ -404,8 +407,73 @@ def grouped_cases(dg, torch, workload, gen, seed):
     return cases
 
 
+def make_flush(torch):
+    """L2 flush between timed calls: write 256 MB (> 126 MB L2), then read
+    another 256 MB so that L2 ends up holding clean lines of unrelated data:
+    no input of the timed call is cached and no dirty line of the flush is
+    written back inside it."""
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush_rd = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
+
+    def flush_l2():
+        flush.zero_()
+        flush_rd.max()
+    return flush_l2
+
+
+def time_calls(torch, calls, steps, warmup, flush_l2):
+    """Mean CUDA-event time (ms) of each call over `steps` steps, each call
+    alone after an L2 flush; every step is enqueued behind a short device
+    sleep so no timed call waits for the host.  Returns (ms list, launches of
+    this library inside the timed steps)."""
+    import moe_grouped_gemm_06_b200 as dg
+    stream = torch.cuda.current_stream()
+
+    def step(events):
+        torch.cuda._sleep(HOLD_CYCLES)
+        for i, call in enumerate(calls):
+            flush_l2()
+            if events is not None:
+                events[i][0].record(stream)
+            call()
+            if events is not None:
+                events[i][1].record(stream)
+
+    for _ in range(warmup):
+        step(None)
+    torch.cuda.synchronize()
+    if steps <= 0:
+        return [], 0
+    events = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
+              for _ in range(steps)]
+    launches0 = dg.dg_launch_count()
+    for s_ in range(steps):
+        step(events[s_])
+    torch.cuda.synchronize()
+    launches = dg.dg_launch_count() - launches0
+    ms = [sum(events[s_][i][0].elapsed_time(events[s_][i][1]) for s_ in range(steps)) / steps
+          for i in range(len(calls))]
+    return ms, launches
+
+
+def case_entries(cases, ms, tensor_peak, hbm, ref_ms=None):
+    """Per-case TFLOP/s, GB/s, the binding roofline and the fraction of it."""
+    ridge = tensor_peak * 1e12 / (hbm * 1e9)
+    out = []
+    for i, ((name, _, f, by), m_) in enumerate(zip(cases, ms)):
+        tf, gbs = f / (m_ * 1e-3) / 1e12, by / (m_ * 1e-3) / 1e9
+        bound = "tensor" if f / by >= ridge else "hbm"
+        entry = {"case": name, "us": round(m_ * 1e3, 2), "tflops": round(tf, 1), "gbs": round(gbs, 1),
+                 "bound": bound, "frac": round(tf / tensor_peak if bound == "tensor" else gbs / hbm, 4)}
+        if ref_ms is not None and ref_ms[i] is not None:
+            entry["cublas_us"] = round(ref_ms[i] * 1e3, 2)
+            entry["cublas_tflops"] = round(f / (ref_ms[i] * 1e-3) / 1e12, 1)
+        out.append(entry)
+    return out
+
+
 def run_grouped(args, dg, torch, rank, world, use_dist, local_rank):
-    """--workload contiguous | masked | fp4: each case timed alone (L2
+    """--workload contiguous | masked | fp4 | ...: each case timed alone (L2
     flushed before every call), one JSON line with per-case TFLOPS, GB/s
     and roofline fraction."""
     gen = torch.Generator(device="cuda")
@@ -416,7 +484,8 @@ def run_grouped(args, dg, torch, rank, world, use_dist, local_rank):
         # one CUDA graph per case (the calls read their group metadata on the
         # device, so a captured launch is replayable); first call eager
         cap = torch.cuda.Stream()
-        for i, (name, call, f, by) in enumerate(cases):
+        for i, case in enumerate(cases):
+            name, call = case[0], case[1]
             with torch.cuda.stream(cap):
                 call()
             cap.synchronize()
@@ -426,84 +495,37 @@ def run_grouped(args, dg, torch, rank, world, use_dist, local_rank):
             # the graph holds raw pointers into the case's tensors: keep the
             # original call (whose closure owns them) alive with the graph
             graphs.append((g, call))
-            cases[i] = (name, g.replay, f, by)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    flush_rd = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
-    stream = torch.cuda.current_stream()
+            cases[i] = (name, g.replay) + tuple(case[2:])
+    flush_l2 = make_flush(torch)
 
     refs = [c[4] if len(c) > 4 else None for c in cases]
     cases = [c[:4] for c in cases]
-
-    def step(events):
-        torch.cuda._sleep(HOLD_CYCLES)
-        for i, (_, call, _, _) in enumerate(cases):
-            flush.zero_()
-            flush_rd.max()
-            if events is not None:
-                events[i][0].record(stream)
-            call()
-            if events is not None:
-                events[i][1].record(stream)
-
-    for _ in range(max(args.warmup, 1)):
-        step(None)
+    time_calls(torch, [c[1] for c in cases], 0, max(args.warmup, 1), flush_l2)   # warm-up only
     err = dg.dg_get_last_error()
     assert err == 0, f"device error during warm-up: {dg.status_string(err)} ({err})"
-    events = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in cases]
-              for _ in range(args.steps)]
     sampler = ClockSampler(local_rank)
     if use_dist:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     sampler.start()
     time.sleep(0.3)
-    launches0 = dg.dg_launch_count()
-    for s_ in range(args.steps):
-        step(events[s_])
-    torch.cuda.synchronize()
-    launches = dg.dg_launch_count() - launches0
+    ms, launches = time_calls(torch, [c[1] for c in cases], args.steps, 0, flush_l2)
     clocks = sampler.stop()
     err = dg.dg_get_last_error()
     assert err == 0, f"device error during timing: {dg.status_string(err)} ({err})"
-    ms = [sum(events[s_][i][0].elapsed_time(events[s_][i][1]) for s_ in range(args.steps)) / args.steps
-          for i in range(len(cases))]
     # library references (cuBLAS for bf16), timed the same way, after ours
     ref_ms = [None] * len(cases)
     if any(r is not None for r in refs):
-        rev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in cases]
-               for _ in range(args.steps)]
-        for s_ in range(-max(args.warmup, 1), args.steps):
-            torch.cuda._sleep(HOLD_CYCLES)
-            for i, r in enumerate(refs):
-                if r is None:
-                    continue
-                flush.zero_()
-                flush_rd.max()
-                if s_ >= 0:
-                    rev[s_][i][0].record(stream)
-                r()
-                if s_ >= 0:
-                    rev[s_][i][1].record(stream)
-        torch.cuda.synchronize()
-        ref_ms = [sum(rev[s_][i][0].elapsed_time(rev[s_][i][1]) for s_ in range(args.steps)) / args.steps
-                  if refs[i] is not None else None for i in range(len(cases))]
+        idx = [i for i, r in enumerate(refs) if r is not None]
+        rms, _ = time_calls(torch, [refs[i] for i in idx], args.steps, args.warmup, flush_l2)
+        for i, v in zip(idx, rms):
+            ref_ms[i] = v
     step_ms_max = max_over_ranks(sum(ms), use_dist, "cuda")
     peaks, peak_kind = load_peaks()
     fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
     hbm = peaks["hbm_gbs"]
     tensor_peak = peaks["bf16_tflops"] if args.workload == "bf16" else fp8_peak
-    ridge = tensor_peak * 1e12 / (hbm * 1e9)
-    per_case = []
-    for (name, _, f, by), m_ in zip(cases, ms):
-        tf, gbs = f / (m_ * 1e-3) / 1e12, by / (m_ * 1e-3) / 1e9
-        bound = "tensor" if f / by >= ridge else "hbm"
-        entry = {"case": name, "us": round(m_ * 1e3, 2), "tflops": round(tf, 1), "gbs": round(gbs, 1),
-                 "bound": bound, "frac": round(tf / tensor_peak if bound == "tensor" else gbs / hbm, 4)}
-        r_ms = ref_ms[len(per_case)]
-        if r_ms is not None:
-            entry["cublas_us"] = round(r_ms * 1e3, 2)
-            entry["cublas_tflops"] = round(f / (r_ms * 1e-3) / 1e12, 1)
-        per_case.append(entry)
+    per_case = case_entries(cases, ms, tensor_peak, hbm, ref_ms)
     dom = max(range(len(cases)), key=lambda i: ms[i])
     pc = per_case[dom]
     roofline = {"bound": pc["bound"], "achieved": pc["tflops"] if pc["bound"] == "tensor" else pc["gbs"],
@@ -522,6 +544,56 @@ def run_grouped(args, dg, torch, rank, world, use_dist, local_rank):
                 "roofline": roofline, "cpu_baseline": None, "e2e": None, "gpu_launches": int(launches),
                 "clocks": clocks, "per_case": per_case}
         print(json.dumps(line), flush=True)
+
+
+def measure_configs(dg, torch, rank, steps, warmup, flush_l2, fp8_peak, hbm):
+    """The other configurations, each case timed alone after an L2 flush
+    like the sweep: the small dense case (128 x 512 x 1024, C = 0), the MoE
+    prefill (contiguous, 2 cases), the MoE decode (masked, 6 cases) and
+    FP8 x FP4 (dense and contiguous, 4 cases).  Returns {name: [per-case]}
+    and the library launches inside their timed steps."""
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(4321 + rank)
+    out, launches = {}, 0
+    small = make_inputs(dg, torch, 128, 512, 1024, gen)
+    small_case = [("dense M=128 N=512 K=1024 C=0",
+                   lambda x=small: dg.dg_fp8_gemm_nt(x["a"], x["sfa"], x["b"], x["sfb"], None, x["d"]),
+                   flops(128, 512, 1024), alg_bytes(128, 512, 1024, with_c=False))]
+    groups = [("dense_small", small_case)]
+    for key, wl in (("contiguous_prefill", "contiguous"), ("masked_decode", "masked"), ("fp8xfp4", "fp4")):
+        groups.append((key, [c[:4] for c in grouped_cases(dg, torch, wl, gen, 99 + rank)]))
+    for key, cases in groups:
+        ms, n = time_calls(torch, [c[1] for c in cases], steps, warmup, flush_l2)
+        launches += n
+        out[key] = case_entries(cases, ms, fp8_peak, hbm)
+    del groups, small
+    torch.cuda.empty_cache()
+    return out, launches
+
+
+def probe_tensor_peaks(dg, torch, kblocks=4096, reps=3):
+    """TFLOP/s of the tensor pipe alone: the library's own tcgen05 loop (one
+    CTA per SM, operands resident in shared memory, no global traffic), best
+    of `reps` launches timed with CUDA events, for the block-scaled FP8 MMA
+    the GEMMs issue, the plain FP8 MMA and bf16, at N = 128 and 256."""
+    stream = torch.cuda.current_stream()
+    out = {}
+    for kind in ("fp8_block_scaled", "fp8_plain", "bf16"):
+        for bn in (128, 256):
+            dg.dg_probe_mma_peak(kind, bn, 256)
+            best = None
+            for _ in range(reps):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                f = dg.dg_probe_mma_peak(kind, bn, kblocks)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                t = f / (e0.elapsed_time(e1) * 1e-3) / 1e12
+                best = t if best is None else max(best, t)
+            out[f"{kind}_n{bn}"] = round(best, 1)
+    err = dg.dg_get_last_error()
+    assert err == 0, f"device error in the tensor probe: {dg.status_string(err)} ({err})"
+    return out
 
 
 # ---------------------------------------------------------------- CPU oracle
@@ -634,15 +706,7 @@ def main():
     gen = torch.Generator(device="cuda")
     gen.manual_seed(1234 + rank)
     inputs = [make_inputs(dg, torch, m, n, k, gen) for (m, n, k) in shapes]
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    flush_rd = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
-
-    def flush_l2():
-        # write 256 MB (> 126 MB L2), then read another 256 MB so that L2 ends
-        # up holding clean lines of unrelated data: no input of the timed call
-        # is cached and no dirty line of the flush is written back inside it
-        flush.zero_()
-        flush_rd.max()
+    flush_l2 = make_flush(torch)
     stream = torch.cuda.current_stream()
     torch.cuda.synchronize()
 
@@ -665,6 +729,7 @@ def main():
         sweep(None)
     err = dg.dg_get_last_error()
     assert err == 0, f"device error during warm-up: {dg.status_string(err)} ({err})"
+    probe = probe_tensor_peaks(dg, torch)
 
     events = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in shapes] for _ in range(args.steps)]
@@ -681,6 +746,13 @@ def main():
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
     launches = dg.dg_launch_count() - launches0
+    peaks, peak_kind = load_peaks()
+    fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
+    hbm = peaks["hbm_gbs"]
+    per_config, config_launches = None, 0
+    if not args.shape and not args.no_configs:
+        per_config, config_launches = measure_configs(dg, torch, rank, args.steps, args.warmup, flush_l2,
+                                                      fp8_peak, hbm)
     if use_dist:
         dist.barrier()
     clocks = sampler.stop()
@@ -695,9 +767,6 @@ def main():
     sweep_flops = sum(flops(*s) for s in shapes)
     value = whole_job_tflops(world, sweep_flops, step_ms_max)
 
-    peaks, peak_kind = load_peaks()
-    fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
-    hbm = peaks["hbm_gbs"]
     ridge = fp8_peak * 1e12 / (hbm * 1e9)
     per_shape = []
     for (m, n, k), ms in zip(shapes, per_shape_ms):
@@ -721,10 +790,16 @@ def main():
         achieved = alg_bytes(dm, dn, dk) / (per_shape_ms[dom] * 1e-3) / 1e9
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                     "frac": round(achieved / hbm, 4)}
+    fp8_probe = max(probe["fp8_block_scaled_n128"], probe["fp8_block_scaled_n256"])
+    if dom_bound == "tensor":
+        roofline["frac_vs_probe"] = round(achieved / fp8_probe, 4)
+        roofline["frac_vs_spec"] = round(achieved / FP8_SPEC_TFLOPS, 4)
     roofline["traffic"] = recorded_traffic(dom_workload)
     roofline["kernel"] = f"gemm_kernel on {dom_workload} ({per_shape_ms[dom] / step_ms * 100:.0f}% of step time)"
     roofline["peak_source"] = (f"{peak_kind}: FP8 = bf16 burst {peaks['bf16_tflops']} x {FP8_PER_BF16} "
-                               f"(nominal FP8:BF16 ratio); HBM {hbm} GB/s")
+                               f"(nominal FP8:BF16 ratio); HBM {hbm} GB/s; beside it the block-scaled FP8 "
+                               f"tcgen05 loop measured in this run, {fp8_probe} TFLOP/s (frac_vs_probe), and the "
+                               f"nominal dense FP8 peak {FP8_SPEC_TFLOPS} TFLOP/s (frac_vs_spec)")
 
     # ---- end to end through the C ABI from pinned host buffers
     e2e = None
@@ -782,6 +857,8 @@ def main():
                        "parallelism": f"replicas x{world}", "wall_s_timed_region": round(wall, 3)},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
             "clocks": clocks, "per_shape": per_shape,
+            "per_config": per_config, "per_config_launches": int(config_launches),
+            "tensor_peak_probe": probe,
         }
         print(json.dumps(line), flush=True)
     if use_dist:

@@ -363,6 +363,41 @@ dg_status dg_query_dense_config(int m, int n, int k, int64_t workspace_cap, int*
                                 int* sk_tiles, int* sk_split, int* max_segments, int* grid,
                                 int64_t* workspace_bytes);
 
+/* Layouts named by dg_query_config. */
+enum { DG_LAYOUT_DENSE = 0, DG_LAYOUT_CONTIGUOUS = 1, DG_LAYOUT_MASKED = 2 };
+
+/* Plan of an NT call of the given layout as the library would launch it on
+ * the current device: block width (block_n), grid size in CTAs and the work
+ * units (output tiles) the persistent grid walks (masked: counted at max_m
+ * rows per group; the kernel walks only the tiles of the valid rows).
+ *   layout     DG_LAYOUT_DENSE / _CONTIGUOUS / _MASKED
+ *   fp4        nonzero: e2m1 B (the *_fp8_fp4_* calls)
+ *   swiglu     nonzero: the masked *_swiglu calls (masked layout only)
+ *   rows       dense m, contiguous m_total, masked max_m
+ *   num_groups 1 for dense; expected_m the masked hint (0 = none)
+ * Any output pointer may be NULL.  Nothing is launched.  DG_ERR_INVALID_ARG
+ * for an unknown layout, non-positive sizes, k not a multiple of 128 or
+ * swiglu outside the masked layout. */
+dg_status dg_query_config(int layout, int fp4, int swiglu, int rows, int n, int k, int num_groups, int expected_m,
+                          int* block_n, int* grid, int64_t* units);
+
+/* Tensor-core throughput probe: one CTA per SM issues kblocks x 4
+ * tcgen05 MMAs of M = 128, N = block_n (128 or 256), K = 32 (bf16: 16) from
+ * operand tiles held in shared memory, with no global-memory traffic, into a
+ * TMEM accumulator.  Kinds:
+ *   DG_PROBE_FP8_SCALED  kind::mxf8f6f4.block_scale, e4m3, UE8M0 scales (the
+ *                        instruction of the GEMM kernels)
+ *   DG_PROBE_FP8_PLAIN   kind::f8f6f4, e4m3, no scales (the per-K-block
+ *                        promotion variant's instruction)
+ *   DG_PROBE_BF16        kind::f16, bf16 operands
+ * One launch performs SMs x kblocks x 4 x 2 x 128 x block_n x 32 FLOPs (bf16:
+ * x 16); time it with events on `stream` to get the pipe's peak rate, the
+ * denominator beside the nominal dense FP8 peak of the B200 (4.5 PFLOP/s).
+ * Asynchronous.  DG_ERR_INVALID_ARG for an unknown kind, another width or
+ * kblocks outside [1, 2^22]. */
+enum { DG_PROBE_FP8_SCALED = 0, DG_PROBE_FP8_PLAIN = 1, DG_PROBE_BF16 = 2 };
+dg_status dg_probe_mma_peak(int kind, int block_n, int kblocks, void* stream);
+
 /* Output tiles of an m x n problem cut into block_m x block_n tiles (the
  * count the heuristic balances against the SM count; "DeepSeek 开源第三弹 ...
  * DeepGEMM" (app.myzaker.com), section "非对齐块大小"). */

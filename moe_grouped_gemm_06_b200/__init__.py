@@ -25,7 +25,7 @@ __all__ = [
     "dg_fp8_gemm_tn", "dg_fp8_gemm_tt",
     "dg_quantize_fp8", "dg_quantize_fp4", "dg_pack_sf", "dg_packed_sf_words", "dg_get_num_sms",
     "dg_set_num_sms", "dg_set_pdl", "dg_get_pdl", "dg_set_tile_config", "dg_get_mk_alignment_for_contiguous_layout", "dg_get_last_error",
-    "dg_debug_starved_wait", "dg_launch_count", "dg_query_dense_config", "dg_num_tiles", "dg_debug_fastdiv", "dg_shutdown",
+    "dg_debug_starved_wait", "dg_launch_count", "dg_query_dense_config", "dg_query_config", "dg_probe_mma_peak", "dg_num_tiles", "dg_debug_fastdiv", "dg_shutdown",
     "SYMBOLS",
 ]
 
@@ -73,6 +73,8 @@ SYMBOLS = {
     "dg_status_string": (ctypes.c_char_p, [_INT]),
     "dg_launch_count": (ctypes.c_uint64, []),
     "dg_query_dense_config": (_INT, [_INT, _INT, _INT, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "dg_query_config": (_INT, [_INT, _INT, _INT, _INT, _INT, _INT, _INT, _INT, _VP, _VP, _VP]),
+    "dg_probe_mma_peak": (_INT, [_INT, _INT, _INT, _VP]),
     "dg_num_tiles": (_I64, [_INT, _INT, _INT, _INT]),
     "dg_debug_fastdiv": (ctypes.c_uint32, [ctypes.c_uint32, ctypes.c_uint32]),
     "dg_shutdown": (None, []),
@@ -333,6 +335,35 @@ def dg_query_dense_config(m: int, n: int, k: int, workspace_cap: int = 0) -> dic
            "dg_query_dense_config")
     keys = ("block_n", "dp_tiles", "sk_tiles", "sk_split", "max_segments", "grid", "workspace_bytes")
     return dict(zip(keys, (v.value for v in vals)))
+
+
+LAYOUTS = {"dense": 0, "contiguous": 1, "masked": 2}
+
+
+def dg_query_config(layout: str, rows: int, n: int, k: int, groups: int = 1, fp4: bool = False,
+                    expected_m: int = 0, swiglu: bool = False) -> dict:
+    """Plan of an NT call (block_n, grid, units = output tiles) as the
+    library would launch it; nothing is launched."""
+    bn, grid, units = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int64(0)
+    _check(lib().dg_query_config(LAYOUTS[layout], int(fp4), int(swiglu), rows, n, k, groups, expected_m,
+                                 ctypes.byref(bn), ctypes.byref(grid), ctypes.byref(units)), "dg_query_config")
+    return {"block_n": bn.value, "grid": grid.value, "units": units.value}
+
+
+PROBE_KINDS = {"fp8_block_scaled": 0, "fp8_plain": 1, "bf16": 2}
+
+
+def dg_probe_mma_peak(kind: str, block_n: int, kblocks: int, stream=None) -> float:
+    """Enqueues the tensor-core throughput probe; returns the FLOPs that one
+    launch performs (time it with CUDA events on the same stream)."""
+    _check(lib().dg_probe_mma_peak(PROBE_KINDS[kind], block_n, kblocks, _stream(stream)), "dg_probe_mma_peak")
+    k_per_mma = 16 if kind == "bf16" else 32
+    return float(dg_get_num_sms_device()) * kblocks * 4 * 2 * 128 * block_n * k_per_mma
+
+
+def dg_get_num_sms_device() -> int:
+    """SMs of the current device (the probe's grid), ignoring dg_set_num_sms."""
+    return torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
 
 
 def dg_num_tiles(m: int, n: int, block_m: int, block_n: int) -> int:

@@ -123,7 +123,10 @@ struct GemmArgs {
 // BF16 = true: A and B bf16 (kind::f16, no scales); a stage then holds 64
 // K-elements, the same 128-byte rows as 128 e4m3 elements, so the staging,
 // descriptors and schedules are shared with the FP8 kernels.
-template <int BN, bool FP4, int CTAS = 1, bool BF16 = false>
+// PREFIX = true (masked and k-grouped layouts): shared memory also holds the
+// per-group prefix of tile counts or K-blocks; the other layouts give those
+// bytes to the stage ring.
+template <int BN, bool FP4, int CTAS = 1, bool BF16 = false, bool PREFIX = true>
 struct Cfg {
   static_assert(!(BF16 && FP4), "bf16 A and B");
   static constexpr int kKPerStage = BF16 ? 64 : kBK;  // K-elements per stage
@@ -150,7 +153,7 @@ struct Cfg {
   static constexpr int kSfbBytes = BF16 ? 0 : kSfbChunks * 512;
   static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes + kSfrBytes;
   static constexpr int kEpiBytes = kEpiWarps * 32 * 64;        // one 32 x 64 B staging box per epilogue warp
-  static constexpr int kMaskBytes = ((kMaxMaskedGroups + 1) * 4 + 15) / 16 * 16;
+  static constexpr int kMaskBytes = PREFIX ? ((kMaxMaskedGroups + 1) * 4 + 15) / 16 * 16 : 0;
   static constexpr int kBarBytes = 256;
   static constexpr int kBudget = 232448 - 1024;              // 227 KB minus alignment slack
   static constexpr int kStagesRaw = (kBudget - kEpiBytes - kMaskBytes - kBarBytes) / kStageBytes;
@@ -325,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const __grid_constant__ CUtensorMap tm_sfb, const GemmArgs args) {
   static_assert(CTAS == 1 || (CTAS == 2 && LAYOUT == kDense), "CTA pairs serve the dense layout");
   static_assert(EPI == kEpiPlain || (CTAS == 1 && BN % (2 * kSwiGluBlock) == 0), "SwiGLU tiles hold whole block pairs");
-  using C = Cfg<BN, FP4, CTAS, BF16>;
+  using C = Cfg<BN, FP4, CTAS, BF16, (LAYOUT == kMasked || LAYOUT == kKGrouped)>;
   static_assert(!BF16 || (CTAS == 1 && EPI == kEpiPlain), "bf16: single CTAs, plain epilogue");
   constexpr bool kAMn = (MAJ & kAMajorMN) != 0;
   constexpr bool kBMn = (MAJ & kBMajorMN) != 0;

@@ -13,6 +13,7 @@
 #include "../../include/dg.h"
 #include "dg_gemm.cuh"
 #include "dg_prep.cuh"
+#include "dg_probe.cuh"
 
 namespace {
 
@@ -329,7 +330,7 @@ float* workspace(size_t bytes, cudaStream_t s) {
 template <int BN, bool FP4, int LAYOUT, int CTAS, int EPI = dg::kEpiPlain, bool BF16 = false, int MAJ = dg::kMajorK>
 dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td, const CUtensorMap& tsfa,
                       const CUtensorMap& tsfb, const dg::GemmArgs& args, int grid, cudaStream_t s) {
-  using C = dg::Cfg<BN, FP4, CTAS, BF16>;
+  using C = dg::Cfg<BN, FP4, CTAS, BF16, (LAYOUT == dg::kMasked || LAYOUT == dg::kKGrouped)>;
   auto kern = dg::gemm_kernel<BN, FP4, LAYOUT, CTAS, EPI, BF16, MAJ>;
   static std::atomic<uint64_t> attr_set_mask{0};  // one bit per device
   int dev = 0;
@@ -416,31 +417,52 @@ int k_plan_mn(const Problem& p) { return std::max(128, (int)(p.k / p.groups) / 1
 // caller-provided device buffer instead of the per-stream workspace, and the
 // planner only considers plans that fit in fixed_ws_bytes (whole tiles
 // always do).
-template <bool FP4, int LAYOUT, int EPI = dg::kEpiPlain, bool BF16 = false, int MAJ = dg::kMajorK>
-dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, size_t fixed_ws_bytes = 0) {
-  constexpr bool kAMn = (MAJ & dg::kAMajorMN) != 0;
-  constexpr bool kBMn = (MAJ & dg::kBMajorMN) != 0;
+// The plan a call of this layout and operand kind runs (block width, schedule,
+// grid), as run_gemm launches it; dg_query_config reports it.
+Plan select_plan(const Problem& p, int layout, bool fp4, bool bf16, bool mn, bool swiglu, int sms,
+                 size_t ws_cap) {
   // a bf16 stage covers 64 K-elements in the time an e4m3 stage covers 128:
   // the planner sees bf16 as an e4m3 problem of twice the K
-  const int k_plan = BF16 ? 2 * p.k : p.k;
-  const int sms = num_sms();
-  if (sms <= 0) return DG_ERR_CUDA;
+  const int k_plan = bf16 ? 2 * p.k : p.k;
   const long long m_blocks = ceil_div(p.rows, dg::kBM);
   Plan plan;
-  if (LAYOUT == dg::kMasked) {
+  if (layout == dg::kMasked) {
     const int em = p.expected_m > 0 ? std::min(p.expected_m, p.rows) : p.rows;
     plan = plan_gemm((long long)p.groups * ceil_div(em, dg::kBM), p.n, p.k, sms, false);
-    if (EPI == dg::kEpiSwiGlu && plan.bn != 128 && plan.bn != 256 && !forced_block_n())
+    if (swiglu && plan.bn != 128 && plan.bn != 256 && !forced_block_n())
       plan.bn = plan.bn > 192 ? 256 : 128;  // SwiGLU tiles hold whole gate/up block pairs
     plan.grid = (int)std::min<long long>((long long)p.groups * m_blocks * ceil_div(p.n, plan.bn), sms);
-  } else if (LAYOUT == dg::kKGrouped) {
+  } else if (layout == dg::kKGrouped) {
     // every group has the same tiles; planned at the mean K of a group
     plan = plan_gemm((long long)p.groups * m_blocks, p.n, k_plan_mn(p), sms, false, 0, false, false, true);
   } else {
     // MN-major operands run in 128- and 256-wide tiles only
-    plan = plan_gemm(m_blocks, p.n, k_plan, sms, LAYOUT == dg::kDense, fixed_ws != nullptr ? fixed_ws_bytes : 0, FP4,
-                     BF16, MAJ != dg::kMajorK);
+    plan = plan_gemm(m_blocks, p.n, k_plan, sms, layout == dg::kDense, ws_cap, fp4, bf16, mn);
   }
+  return plan;
+}
+
+// Work units (tiles) of a plan, as the kernel counts them (masked: at the
+// maximum of max_m rows per group).
+long long plan_units(const Problem& p, const Plan& plan, int layout) {
+  const long long nb = ceil_div(p.n, plan.bn), mb = ceil_div(p.rows, dg::kBM);
+  if (layout == dg::kDense) return mb * nb;
+  return (long long)(layout == dg::kContig ? 1 : p.groups) * mb * nb;
+}
+
+// fixed_ws / fixed_ws_bytes: when given, stream-K partials go to this
+// caller-provided device buffer instead of the per-stream workspace, and the
+// planner only considers plans that fit in fixed_ws_bytes (whole tiles
+// always do).
+template <bool FP4, int LAYOUT, int EPI = dg::kEpiPlain, bool BF16 = false, int MAJ = dg::kMajorK>
+dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, size_t fixed_ws_bytes = 0) {
+  constexpr bool kAMn = (MAJ & dg::kAMajorMN) != 0;
+  constexpr bool kBMn = (MAJ & dg::kBMajorMN) != 0;
+  const int sms = num_sms();
+  if (sms <= 0) return DG_ERR_CUDA;
+  const long long m_blocks = ceil_div(p.rows, dg::kBM);
+  const Plan plan = select_plan(p, LAYOUT, FP4, BF16, MAJ != dg::kMajorK, EPI == dg::kEpiSwiGlu, sms,
+                                fixed_ws != nullptr ? fixed_ws_bytes : 0);
   if (plan.grid <= 0) return DG_ERR_UNSUPPORTED;  // (a forced width this layout cannot use)
 
   dg::GemmArgs args{};
@@ -567,6 +589,17 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
   const int threads = 256;
   const int blocks = (int)std::min<long long>(ceil_div(items, threads), (long long)sms * 8);
   if (launch(dg::sk_reduce_kernel, dim3(blocks), dim3(threads), 0, s, 1, r) != cudaSuccess) return DG_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return DG_OK;
+}
+
+template <int KIND, int BN>
+dg_status launch_probe(int kblocks, int grid, cudaStream_t s) {
+  auto kern = dg::mma_peak_kernel<KIND, BN>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dg::kProbeSmem) != cudaSuccess)
+    return DG_ERR_CUDA;
+  kern<<<grid, dg::kProbeThreads, dg::kProbeSmem, s>>>(kblocks, timeout_ns());
+  if (cudaGetLastError() != cudaSuccess) return DG_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return DG_OK;
 }
@@ -917,6 +950,40 @@ dg_status dg_query_dense_config(int m, int n, int k, int64_t workspace_cap, int*
   if (grid) *grid = p.grid;
   if (workspace_bytes) *workspace_bytes = (int64_t)p.ws_bytes();
   return DG_OK;
+}
+
+dg_status dg_query_config(int layout, int fp4, int swiglu, int rows, int n, int k, int num_groups, int expected_m,
+                          int* block_n, int* grid, int64_t* units) {
+  if (layout < DG_LAYOUT_DENSE || layout > DG_LAYOUT_MASKED || rows <= 0 || n <= 0 || k <= 0 || k % 128 != 0 ||
+      num_groups <= 0 || expected_m < 0 || (swiglu && layout != DG_LAYOUT_MASKED))
+    return DG_ERR_INVALID_ARG;
+  const int sms = num_sms();
+  if (sms <= 0) return DG_ERR_CUDA;
+  const int lay = layout == DG_LAYOUT_DENSE ? dg::kDense : (layout == DG_LAYOUT_CONTIGUOUS ? dg::kContig : dg::kMasked);
+  Problem p{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, rows, n, k,
+            lay == dg::kDense ? 1 : num_groups, expected_m};
+  const Plan plan = select_plan(p, lay, fp4 != 0, false, false, swiglu != 0, sms, 0);
+  if (block_n) *block_n = plan.bn;
+  if (grid) *grid = plan.grid;
+  if (units) *units = plan_units(p, plan, lay);
+  return DG_OK;
+}
+
+dg_status dg_probe_mma_peak(int kind, int block_n, int kblocks, void* stream) {
+  if (kind < DG_PROBE_FP8_SCALED || kind > DG_PROBE_BF16 || (block_n != 128 && block_n != 256) || kblocks <= 0 ||
+      kblocks > (1 << 22))
+    return DG_ERR_INVALID_ARG;
+  const int grid = device_sms();
+  if (grid <= 0) return DG_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (kind == DG_PROBE_FP8_SCALED)
+    return block_n == 128 ? launch_probe<dg::kProbeScaled, 128>(kblocks, grid, s)
+                          : launch_probe<dg::kProbeScaled, 256>(kblocks, grid, s);
+  if (kind == DG_PROBE_FP8_PLAIN)
+    return block_n == 128 ? launch_probe<dg::kProbePlain, 128>(kblocks, grid, s)
+                          : launch_probe<dg::kProbePlain, 256>(kblocks, grid, s);
+  return block_n == 128 ? launch_probe<dg::kProbeBf16, 128>(kblocks, grid, s)
+                        : launch_probe<dg::kProbeBf16, 256>(kblocks, grid, s);
 }
 
 uint32_t dg_debug_fastdiv(uint32_t d, uint32_t n) {

@@ -547,6 +547,100 @@ def test_fp8_fp4_full_size_sampled(dg, N, K):
     check_close(d[pm, pn], p.ref_points(pm, pn), f"fp8xfp4 4096x{N}x{K}")
 
 
+@pytest.mark.parametrize("N,K", synth.GROUPED_NK)
+def test_fp8_fp4_contiguous_full_size_sampled(dg, N, K):
+    # the FP8 x FP4 MoE prefill at full size: 8 experts of U[6000, 10000]
+    # tokens each padded to 128 (padding rows of A full of junk and NaN
+    # codes), e2m1 weights with 1x32 scales, in the plan the bench times
+    cs = _contiguous_case(6300 + N, 8, 6000, 10000, N, K, fp4=True)
+    cfg = dg.dg_query_config("contiguous", cs["M"], N, K, groups=8, fp4=True)
+    print(f"fp8xfp4 contiguous {cs['M']}x{N}x{K}: {cfg}", flush=True)
+    assert cfg["grid"] == dg.dg_get_num_sms() and cfg["units"] > 4 * cfg["grid"]
+    d = _run_contiguous(dg, cs, N, fp4=True)
+    valid_rows = np.nonzero(cs["mi"] >= 0)[0]
+    pm, pn = synth.sample_points(6400 + N, valid_rows, N, 4096)
+    ref = np.empty(pm.size)
+    for g in range(8):
+        sel = cs["mi"][pm] == g
+        assert sel.any()
+        ref[sel] = oracle.gemm_points(cs["qa"], cs["ea"], cs["qb"][g], cs["eb"][g], pm[sel], pn[sel], c=cs["c"],
+                                      b_fp4=True)
+    check_close(d[pm, pn], ref, f"fp8xfp4 contiguous {N}x{K}")
+    # the rows after the padding rows of every group are that group's
+    pad_end = np.nonzero(np.diff((cs["mi"] < 0).astype(np.int8)) == -1)[0] + 1
+    edge = pad_end[pad_end < cs["M"]]
+    for m in edge[:4]:
+        g = int(cs["mi"][m])
+        pn_e = np.arange(0, N, 97)
+        check_close(d[m, pn_e], oracle.gemm_points(cs["qa"], cs["ea"], cs["qb"][g], cs["eb"][g], np.full(pn_e.size, m),
+                                                    pn_e, c=cs["c"], b_fp4=True), f"first row of group {g}")
+
+
+_FP4_B_CACHE = {}
+
+
+def _fp4_grouped_b(seed, G, N, K):
+    key = (seed, G, N, K)
+    if key not in _FP4_B_CACHE:
+        _FP4_B_CACHE.clear()
+        _FP4_B_CACHE[key] = quantize_groups_b(seed, G, N, K, fp4=True)
+    return _FP4_B_CACHE[key]
+
+
+@pytest.mark.parametrize("swiglu", [False, True])
+def test_masked_fp4_full_size_sampled(dg, swiglu):
+    # the FP8 x FP4 MoE decode at full size: 32 experts, max_m = 256,
+    # masked_m ~ U[0, 2 x 128], linear1 shape (N, K) = (4096, 7168), plain or
+    # with SwiGLU fused (gate / up rows interleaved in blocks of 64, D has
+    # N / 2 columns); rows >= masked_m must stay untouched bit for bit
+    G, max_m, N, K, em = 32, 256, 4096, 7168, 128
+    mm = synth.masked_counts(5900, G, em, max_m)
+    xa = synth.normal_f32(5901, (G * max_m, K))
+    qa, ea = oracle.quantize_fp8(xa, 1)
+    del xa
+    qa = qa.reshape(G, max_m, K)
+    ea = ea.reshape(G, max_m, K // 128)
+    for g in range(G):
+        v = int(mm[g])
+        qa[g, v:] = synth.junk_bytes(5902 + g, (max_m - v, K))
+    sfa = np.concatenate([oracle.pack_sf(ea[g], max_m).ravel() for g in range(G)])
+    qb, eb, sfb = _fp4_grouped_b(5950, G, N, K)
+    cols = N // 2 if swiglu else N
+    cfg = dg.dg_query_config("masked", max_m, N, K, groups=G, fp4=True, expected_m=em, swiglu=swiglu)
+    print(f"fp8xfp4 masked swiglu={swiglu}: {cfg}", flush=True)
+    assert cfg["grid"] == dg.dg_get_num_sms()
+    d = torch.full((G, max_m, cols), SENTINEL, dtype=torch.int16, device="cuda")
+    fn = dg.dg_m_grouped_fp8_fp4_gemm_nt_masked_swiglu if swiglu else dg.dg_m_grouped_fp8_fp4_gemm_nt_masked
+    fn(dev(qa), dev(sfa), dev(qb), dev(sfb), d, dev(mm), expected_m=em)
+    torch.cuda.synchronize()
+    rows_valid = torch.arange(max_m, device="cuda")[None, :] < dev(mm)[:, None]
+    assert bool((d == SENTINEL).all(dim=2)[~rows_valid].all()), "rows >= masked_m were written"
+    dd = bf16_dev_to_f64(d)
+    r = synth.rng(5960 + swiglu)
+    valid = [(g, m) for g in range(G) for m in range(int(mm[g]))]
+    pick = r.choice(len(valid), size=2048, replace=False)
+    pj = r.integers(0, cols, size=pick.size)
+    pg = np.array([valid[j][0] for j in pick])
+    pm = np.array([valid[j][1] for j in pick])
+    got = dd[pg, pm, pj]
+    ref = np.empty(pick.size)
+    for g in range(G):
+        sel = pg == g
+        if not sel.any():
+            continue
+        if swiglu:
+            # output column j = 64 p + i reads gate column 128 p + i and up
+            # column 128 p + 64 + i; the oracle's SwiGLU with blocks of one
+            # column applied to the (gate, up) pair of each point
+            p_, i_ = pj[sel] // 64, pj[sel] % 64
+            gate = oracle.gemm_points(qa[g], ea[g], qb[g], eb[g], pm[sel], 128 * p_ + i_, b_fp4=True)
+            up = oracle.gemm_points(qa[g], ea[g], qb[g], eb[g], pm[sel], 128 * p_ + 64 + i_, b_fp4=True)
+            ref[sel] = oracle.swiglu_interleaved(np.stack([gate, up], axis=-1), block=1)[:, 0]
+        else:
+            ref[sel] = oracle.gemm_points(qa[g], ea[g], qb[g], eb[g], pm[sel], pj[sel], b_fp4=True)
+    check_close(got, ref, f"fp8xfp4 masked full size swiglu={swiglu}")
+
+
 # ------------------------------------------------------------------ failure paths
 
 def test_starved_wait_times_out_and_context_survives(dg):
@@ -768,3 +862,22 @@ def test_dense_layouts_full_size_sampled(dg, layout):
     pm, pn = synth.sample_points(2901, np.arange(M), N, 2048)
     # the oracle's layout calls equal its NT call on the logical operands
     check_close(d[pm, pn], p.ref_points(pm, pn), f"{layout} {M}x{N}x{K}")
+
+
+# ------------------------------------------------------------------ tensor probe
+
+@pytest.mark.parametrize("kind", ["fp8_block_scaled", "fp8_plain", "bf16"])
+def test_tensor_probe_runs_and_reports_a_rate(dg, kind):
+    # the throughput probe the bench divides by: it must finish, leave no
+    # device error, and land between a tenth of and twice the nominal dense
+    # peak of its kind (FP8 4.5, bf16 2.25 PFLOP/s)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dg.dg_probe_mma_peak(kind, 256, 64)
+    e0.record()
+    f = dg.dg_probe_mma_peak(kind, 256, 2048)
+    e1.record()
+    torch.cuda.synchronize()
+    tflops = f / (e0.elapsed_time(e1) * 1e-3) / 1e12
+    nominal = 2250.0 if kind == "bf16" else 4500.0
+    print(f"{kind}: {tflops:.0f} TFLOP/s", flush=True)
+    assert 0.1 * nominal < tflops < 2.0 * nominal
