@@ -68,7 +68,7 @@ def parse_args():
     ap.add_argument("--shape", default=None, help="run one M,N,K shape instead of the sweep")
     ap.add_argument("--workload", default="dense",
                     choices=["dense", "contiguous", "masked", "fp4", "moe_decode_fp4", "bf16", "nn_contiguous",
-                             "kgrouped_tn"],
+                             "kgrouped_tn", "promotion"],
                     help="dense: the DeepSeek-V3 dense sweep (default); contiguous / masked / fp4: the "
                          "M-grouped prefill, masked decode and FP8 x FP4 cases, one JSON line each")
     ap.add_argument("--graph", action="store_true",
@@ -391,6 +391,28 @@ def grouped_cases(dg, torch, workload, gen, seed):
             cases.append((f"bf16 M={m} N={n} K={k}", (lambda a=a, b=b, d=d: dg.dg_bf16_gemm_nt(a, b, None, d)),
                           2.0 * m * n * k, 2 * (m * k + n * k + m * n),
                           (lambda a=a, b=b, d_ref=d_ref: torch.matmul(a, b.t(), out=d_ref))))
+    elif workload == "promotion":
+        # the two ways of applying the scales on the same operands: inside the
+        # block-scaled MMA (the library's plan, and forced to 128-wide tiles
+        # like the promotion kernel), and per-K-block promotion
+        for (m, n, k) in [(4096, 7168, 16384), (64, 7168, 16384), (4096, 4096, 7168), (4096, 7168, 2048)]:
+            x = make_inputs(dg, torch, m, n, k, gen)
+            f, by = flops(m, n, k), alg_bytes(m, n, k)
+
+            def scaled(x=x, bn=0):
+                if bn:
+                    dg.dg_set_tile_config(bn, 0)
+                try:
+                    dg.dg_fp8_gemm_nt(x["a"], x["sfa"], x["b"], x["sfb"], x["c"], x["d"])
+                finally:
+                    if bn:
+                        dg.dg_set_tile_config(0, 0)
+            cases.append((f"block-scaled MMA M={m} N={n} K={k}", scaled, f, by))
+            cases.append((f"block-scaled MMA, 128-wide tiles M={m} N={n} K={k}",
+                          (lambda x=x: scaled(x, 128)), f, by))
+            cases.append((f"per-K-block promotion M={m} N={n} K={k}",
+                          (lambda x=x: dg.dg_fp8_gemm_nt_promoted(x["a"], x["sfa"], x["b"], x["sfb"], x["c"], x["d"])),
+                          f, by))
     elif workload == "fp4":
         for (n, k) in GROUPED_NK:
             m = 4096

@@ -92,6 +92,20 @@ typedef enum {
 dg_status dg_fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
                          const void* c, void* d, int m, int n, int k, void* stream);
 
+/* Dense NT FP8 GEMM with the scales applied by per-K-block promotion instead
+ * of inside the MMA: the same operands, layouts, result definition,
+ * requirements and errors as dg_fp8_gemm_nt.  Each 128-deep K-block of a
+ * 128 x 128 tile is summed unscaled by kind::f8f6f4 MMAs into a TMEM buffer
+ * of its own (four rotate); epilogue warps read it, multiply by
+ * sa[m, kb] * sb[n/128, kb] and add into FP32 registers, then D = bf16(acc +
+ * C).  This is the two-level accumulation of the pages' Hopper design
+ * ("DeepSeek 开源第三弹 ... DeepGEMM" (app.myzaker.com), sections "DeepGEMM"
+ * and "持久化线程束专用化"), built on sm_100a as the measured alternative to
+ * dg_fp8_gemm_nt's block-scaled MMA.  Tiles are always 128 wide; shared
+ * tiles use the per-stream workspace as dg_fp8_gemm_nt does. */
+dg_status dg_fp8_gemm_nt_promoted(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                                  const void* c, void* d, int m, int n, int k, void* stream);
+
 /* Dense FP8 GEMM in the other three storage layouts (the guide, section 五:
  * SM100 takes all of NT, TN, NN and TT).  The first letter names A's storage,
  * the second B's, relative to D = A * B with A [m][k] and B [k][n]:
@@ -238,9 +252,21 @@ dg_status dg_m_grouped_fp8_fp4_gemm_nt_masked_swiglu(const void* a, const int32_
  * All calls on a device share the array and it keeps the last call's
  * contents, so two calls whose kernels overlap on the GPU (different streams,
  * or different host threads without ordering) race and give wrong results;
- * order them on one stream.  The first call on each device looks up the
- * array's device address (cudaGetSymbolAddress) with that device current;
- * make that first call before any stream capture. */
+ * order them on one stream.
+ *
+ * When the 32 MiB are committed: with CUDA's lazy module loading (the default
+ * since CUDA 12.2) the array is allocated on a device when this library's
+ * module is first loaded there -- at its first kernel launch or symbol lookup
+ * on that device, which may be this call.  That load can fail for lack of
+ * memory (DG_ERR_CUDA) if the caller has already claimed the device's memory,
+ * so make one warm-up call per device before fixing the memory budget, or set
+ * CUDA_MODULE_LOADING=EAGER.
+ *
+ * The first call on each device (and in each new context of it) looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current and
+ * caches it per device and context; make that first call before any stream
+ * capture.  After a device reset the next call looks the address up again;
+ * dg_shutdown() also forgets the cached addresses. */
 dg_status dg_fp8_gemm_nt_noalloc(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
                                  const void* c, void* d, int m, int n, int k, void* stream);
 
@@ -403,7 +429,9 @@ dg_status dg_probe_mma_peak(int kind, int block_n, int kblocks, void* stream);
  * DeepGEMM" (app.myzaker.com), section "非对齐块大小"). */
 int64_t dg_num_tiles(int m, int n, int block_m, int block_n);
 
-/* Releases the stream-K workspaces of all devices (synchronises each). */
+/* Releases the stream-K workspaces of all devices (synchronises each) and
+ * forgets the cached scratch addresses of dg_fp8_gemm_nt_noalloc.  Call it
+ * before resetting a device this library has used. */
 void dg_shutdown(void);
 
 #ifdef __cplusplus

@@ -20,7 +20,7 @@ import torch
 __all__ = [
     "DGError", "lib", "dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
     "dg_m_grouped_fp8_gemm_nt_masked", "dg_m_grouped_fp8_fp4_gemm_nt_masked",
-    "dg_m_grouped_fp8_gemm_nt_masked_swiglu", "dg_m_grouped_fp8_fp4_gemm_nt_masked_swiglu", "dg_fp8_gemm_nt_noalloc", "dg_noalloc_scratch_bytes", "dg_fp8_fp4_gemm_nt", "dg_bf16_gemm_nt", "dg_m_grouped_fp8_fp4_gemm_nt_contiguous",
+    "dg_m_grouped_fp8_gemm_nt_masked_swiglu", "dg_m_grouped_fp8_fp4_gemm_nt_masked_swiglu", "dg_fp8_gemm_nt_noalloc", "dg_noalloc_scratch_bytes", "dg_fp8_gemm_nt_promoted", "dg_fp8_fp4_gemm_nt", "dg_bf16_gemm_nt", "dg_m_grouped_fp8_fp4_gemm_nt_contiguous",
     "dg_m_grouped_fp8_gemm_nn_contiguous", "dg_k_grouped_fp8_gemm_tn_contiguous", "dg_fp8_gemm_nn",
     "dg_fp8_gemm_tn", "dg_fp8_gemm_tt",
     "dg_quantize_fp8", "dg_quantize_fp4", "dg_pack_sf", "dg_packed_sf_words", "dg_get_num_sms",
@@ -45,6 +45,7 @@ SYMBOLS = {
     "dg_m_grouped_fp8_gemm_nt_masked_swiglu": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _I32P, _INT, _INT, _INT, _INT, _INT, _VP]),
     "dg_m_grouped_fp8_fp4_gemm_nt_masked_swiglu": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _I32P, _INT, _INT, _INT, _INT,
                                                           _INT, _VP]),
+    "dg_fp8_gemm_nt_promoted": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _INT, _INT, _INT, _VP]),
     "dg_fp8_gemm_nt_noalloc": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _INT, _INT, _INT, _VP]),
     "dg_fp8_gemm_nn": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _INT, _INT, _INT, _VP]),
     "dg_fp8_gemm_tn": (_INT, [_VP, _I32P, _VP, _I32P, _VP, _VP, _INT, _INT, _INT, _VP]),
@@ -137,6 +138,15 @@ def dg_fp8_gemm_nt(a, sfa, b, sfb, c, d, stream=None) -> None:
     n = b.shape[0]
     _check(lib().dg_fp8_gemm_nt(_p(a), _p(sfa), _p(b), _p(sfb), _p(c), _p(d), m, n, k, _stream(stream)),
            "dg_fp8_gemm_nt")
+
+
+def dg_fp8_gemm_nt_promoted(a, sfa, b, sfb, c, d, stream=None) -> None:
+    """As dg_fp8_gemm_nt, with the scales applied by per-K-block promotion
+    (unscaled MMA per K-block, scaled and summed in FP32 by the epilogue)."""
+    m, k = a.shape
+    n = b.shape[0]
+    _check(lib().dg_fp8_gemm_nt_promoted(_p(a), _p(sfa), _p(b), _p(sfb), _p(c), _p(d), m, n, k, _stream(stream)),
+           "dg_fp8_gemm_nt_promoted")
 
 
 def dg_fp8_gemm_nt_noalloc(a, sfa, b, sfb, c, d, stream=None) -> None:

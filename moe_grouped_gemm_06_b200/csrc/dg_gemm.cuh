@@ -56,8 +56,15 @@ enum : int { kMajorK = 0, kAMajorMN = 1, kBMajorMN = 2 };
 
 // Epilogues: D = bf16(acc + C), or SwiGLU on B rows interleaved in blocks of
 // kSwiGluBlock (gate rows, then the matching up rows): act = bf16(silu(gate)
-// * up), half as many columns as the GEMM.
-enum : int { kEpiPlain = 0, kEpiSwiGlu = 1 };
+// * up), half as many columns as the GEMM.  kEpiPromote: D = bf16(acc + C)
+// where the scales are not applied by the MMA: each 128-deep K-block is
+// summed unscaled by a plain kind::f8f6f4 MMA into a TMEM buffer of its own,
+// and the epilogue warps "promote" it -- multiply by sa * sb and add into
+// FP32 registers -- the two-level accumulation of the pages' Hopper design
+// ("DeepSeek 开源第三弹 ... DeepGEMM" (app.myzaker.com), sections "DeepGEMM"
+// and "持久化线程束专用化"), kept as the measured alternative to the
+// block-scaled MMA.
+enum : int { kEpiPlain = 0, kEpiSwiGlu = 1, kEpiPromote = 2 };
 constexpr int kSwiGluBlock = 64;
 
 // Unsigned division by a run-time divisor d >= 1 fixed per launch, as one
@@ -126,9 +133,12 @@ struct GemmArgs {
 // PREFIX = true (masked and k-grouped layouts): shared memory also holds the
 // per-group prefix of tile counts or K-blocks; the other layouts give those
 // bytes to the stage ring.
-template <int BN, bool FP4, int CTAS = 1, bool BF16 = false, bool PREFIX = true>
+// PROMO = true (kEpiPromote): no scale words are staged (the epilogue reads
+// them from global memory) and TMEM holds only per-K-block partial sums.
+template <int BN, bool FP4, bool BF16 = false, bool PREFIX = true, bool PROMO = false>
 struct Cfg {
   static_assert(!(BF16 && FP4), "bf16 A and B");
+  static_assert(!PROMO || (!FP4 && !BF16 && BN == 128), "promotion: e4m3 A and B, 128-wide tiles");
   static constexpr int kKPerStage = BF16 ? 64 : kBK;  // K-elements per stage
   // The scale-factor operand of the MMA is addressed in TMEM columns of 32
   // rows (a 128-row chunk spans 4 columns), and that address must be even: a
@@ -141,16 +151,16 @@ struct Cfg {
   static constexpr int kSfbChunks = (kMaxOffRows + BN + 127) / 128;  // 128-row scale chunks a tile can touch
   static constexpr bool kRebase = (BN % 64 != 0);
   static constexpr int kSfrChunks = (BN + 127) / 128;                // re-based chunks (tile rows only)
-  static constexpr int kSfrBytes = (kRebase && !BF16) ? kSfrChunks * 512 : 0;
+  static constexpr int kSfrBytes = (kRebase && !BF16 && !PROMO) ? kSfrChunks * 512 : 0;
   // FP32 accumulator buffers in TMEM: three of 128 columns (BN = 128), two at
   // columns 0 and 256 (BN = 192), one (BN = 256); scale factors after them.
-  static constexpr int kAccBufs = (BN <= 128) ? 3 : (BN <= 240 ? 2 : 1);
+  // Promotion: four 128-column buffers of K-block partial sums, no scales.
+  static constexpr int kAccBufs = PROMO ? 4 : ((BN <= 128) ? 3 : (BN <= 240 ? 2 : 1));
   static constexpr int kABytes = kBM * kBK;                  // 16 KB
-  static constexpr int kBRows = BN / CTAS;                   // B rows each CTA of a pair loads
-  static constexpr int kBBytes = kBRows * kBK;               // smem bytes (FP4 lands padded to 1 B/elt)
+  static constexpr int kBBytes = BN * kBK;                   // smem bytes (FP4 lands padded to 1 B/elt)
   static constexpr int kBTxBytes = FP4 ? kBBytes / 2 : kBBytes;  // bytes the TMA copy reports (packed)
-  static constexpr int kSfaBytes = BF16 ? 0 : 512;
-  static constexpr int kSfbBytes = BF16 ? 0 : kSfbChunks * 512;
+  static constexpr int kSfaBytes = (BF16 || PROMO) ? 0 : 512;
+  static constexpr int kSfbBytes = (BF16 || PROMO) ? 0 : kSfbChunks * 512;
   static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes + kSfrBytes;
   static constexpr int kEpiBytes = kEpiWarps * 32 * 64;        // one 32 x 64 B staging box per epilogue warp
   static constexpr int kMaskBytes = PREFIX ? ((kMaxMaskedGroups + 1) * 4 + 15) / 16 * 16 : 0;
@@ -164,17 +174,18 @@ struct Cfg {
   static constexpr uint32_t kAccStride = (BN <= 128) ? 128 : 256;
   static constexpr uint32_t kColSfa = (kAccBufs - 1) * kAccStride + BN;  // even, 4-column aligned
   static constexpr uint32_t kColSfb = kColSfa + 4;
-  static_assert(kColSfb + 4 * kSfbChunks <= kTmemCols, "TMEM columns");
+  static_assert(PROMO ? kAccBufs * kAccStride <= kTmemCols : kColSfb + 4 * kSfbChunks <= kTmemCols, "TMEM columns");
   // Instruction descriptor of kind::mxf8f6f4 with block scaling: A = E4M3,
-  // B = E4M3 (0) or E2M1 (5), both K-major, UE8M0 scales, M = 128 per CTA
-  // (256 for a CTA pair), N = BN.
+  // B = E4M3 (0) or E2M1 (5), both K-major, UE8M0 scales, M = 128, N = BN.
   static constexpr uint32_t kIdescScaled = (0u << 7) | ((FP4 ? 5u : 0u) << 10) | ((uint32_t)(BN >> 3) << 17) |
-                                           (1u << 23) | ((uint32_t)((kBM * CTAS) >> 4) << 24);
+                                           (1u << 23) | ((uint32_t)(kBM >> 4) << 24);
   // kind::f16: FP32 accumulator (bits 4-5 = 1), A and B bf16 (formats 1),
   // both K-major, N >> 3, M >> 4
   static constexpr uint32_t kIdescBf16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                                         ((uint32_t)((kBM * CTAS) >> 4) << 24);
-  static constexpr uint32_t kIdesc = BF16 ? kIdescBf16 : kIdescScaled;
+                                         ((uint32_t)(kBM >> 4) << 24);
+  // kind::f8f6f4 (promotion): FP32 accumulator, A and B E4M3, K-major
+  static constexpr uint32_t kIdescPlain = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+  static constexpr uint32_t kIdesc = BF16 ? kIdescBf16 : (PROMO ? kIdescPlain : kIdescScaled);
 };
 
 struct Unit {
@@ -313,32 +324,27 @@ struct WorkIter {
   }
 };
 
-// CTAS = 2: a cluster of two CTAs computes 256 x BN tiles (dense layout only);
-// tm_sfa / tm_sfb view the packed scale words as rows of 512 bytes so that
-// the peer's scale loads can complete on the leader's barrier.
-//
 // MAJ != kMajorK: A and/or B staged MN-major (NN, TN, TT layouts): each 128-wide
 // M or N block of a stage is one TMA box of 128 elements x 128 K rows, and
 // the MMA reads it through an MN-major descriptor (plain FP8 tiles of width
 // 128 or 256 only).
-template <int BN, bool FP4, int LAYOUT, int CTAS, int EPI = kEpiPlain, bool BF16 = false, int MAJ = kMajorK>
+template <int BN, bool FP4, int LAYOUT, int EPI = kEpiPlain, bool BF16 = false, int MAJ = kMajorK>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                const __grid_constant__ CUtensorMap tm_d, const __grid_constant__ CUtensorMap tm_sfa,
-                const __grid_constant__ CUtensorMap tm_sfb, const GemmArgs args) {
-  static_assert(CTAS == 1 || (CTAS == 2 && LAYOUT == kDense), "CTA pairs serve the dense layout");
-  static_assert(EPI == kEpiPlain || (CTAS == 1 && BN % (2 * kSwiGluBlock) == 0), "SwiGLU tiles hold whole block pairs");
-  using C = Cfg<BN, FP4, CTAS, BF16, (LAYOUT == kMasked || LAYOUT == kKGrouped)>;
-  static_assert(!BF16 || (CTAS == 1 && EPI == kEpiPlain), "bf16: single CTAs, plain epilogue");
+    gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a32,
+                const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_d,
+                const GemmArgs args) {
+  static_assert(EPI == kEpiPlain || BN % (2 * kSwiGluBlock) == 0, "SwiGLU tiles hold whole block pairs");
+  constexpr bool kPromo = (EPI == kEpiPromote);
+  using C = Cfg<BN, FP4, BF16, (LAYOUT == kMasked || LAYOUT == kKGrouped), kPromo>;
+  static_assert(!BF16 || EPI == kEpiPlain, "bf16: plain epilogue");
+  static_assert(!kPromo || (LAYOUT == kDense && MAJ == kMajorK), "promotion: dense NT");
   constexpr bool kAMn = (MAJ & kAMajorMN) != 0;
   constexpr bool kBMn = (MAJ & kBMajorMN) != 0;
-  static_assert(MAJ == kMajorK || (!FP4 && !BF16 && CTAS == 1 && EPI == kEpiPlain && BN % 128 == 0),
-                "MN-major operands: FP8, single CTAs, plain epilogue, 128-wide column blocks");
+  static_assert(MAJ == kMajorK || (!FP4 && !BF16 && EPI == kEpiPlain && BN % 128 == 0),
+                "MN-major operands: FP8, plain epilogue, 128-wide column blocks");
   static_assert(LAYOUT != kKGrouped || MAJ == (kAMajorMN | kBMajorMN), "k-grouped: A and B MN-major");
   // D and C of the masked and k-grouped layouts are [groups][rows][n]
   constexpr bool kGroupRows = (LAYOUT == kMasked || LAYOUT == kKGrouped);
-  constexpr bool kPair = (CTAS == 2);
-  constexpr int kTileM = kBM * CTAS;
   constexpr int S = C::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -352,26 +358,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(s_prefix) + C::kMaskBytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + S;
-  uint64_t* tfull = bars + 2 * S;
-  uint64_t* tempty = bars + 2 * S + 3;
-  uint64_t* drain = bars + 2 * S + 6;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 * S + 7);
+  uint64_t* tfull = bars + 2 * S;       // [4]: accumulator buffer b holds a result
+  uint64_t* tempty = bars + 2 * S + 4;  // [4]: the epilogue has read buffer b
+  uint64_t* drain = bars + 2 * S + 8;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 * S + 9);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
 
   const int warp = threadIdx.x / 32;
   const uint32_t lane = lane_id();
   const GemmArgs& a = args;
-  const uint32_t rank = kPair ? cluster_ctarank() : 0u;   // 0 = leader (issues the MMAs)
-  const int cta_id = blockIdx.x / CTAS, num_ctas = gridDim.x / CTAS;
+  const int cta_id = blockIdx.x, num_ctas = gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 3; ++b) {
+    for (int b = 0; b < 4; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], kEpiWarps * CTAS);  // the pair's epilogues release the leader
+      mbar_init(&tempty[b], kEpiWarps);
     }
     mbar_init(drain, 1);
     *s_abort = 0;
@@ -379,21 +384,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tm_a);
+    if constexpr (!kAMn) prefetch_tmap(&tm_a32);
     prefetch_tmap(&tm_b);
     prefetch_tmap(&tm_d);
-    if constexpr (kPair) {
-      prefetch_tmap(&tm_sfa);
-      prefetch_tmap(&tm_sfb);
-    }
   }
   if (warp == 1) {
-    if constexpr (kPair) {
-      tmem_alloc_pair(s_tmem, kTmemCols);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(s_tmem, kTmemCols);
-      tmem_relinquish();
-    }
+    tmem_alloc(s_tmem, kTmemCols);
+    tmem_relinquish();
   }
   // Prologue above touches no global memory; with programmatic dependent
   // launch it overlaps the previous kernel's tail.  Everything below may
@@ -442,10 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   tc_fence_before();
-  if constexpr (kPair)
-    cluster_sync_all();  // both CTAs' barriers initialised before any cross-CTA arrival
-  else
-    __syncthreads();
+  __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
   if (LAYOUT == kMasked)
@@ -480,13 +474,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int c0 = n0 / 128;
         const int c1 = (min(n0 + BN, a.n) - 1) / 128;
         const int nchunks = c1 - c0 + 1;
-        const int a_row = u.mb * kTileM + (int)rank * kBM;
+        const int a_row = u.mb * kBM;
         const int a_grp = (LAYOUT == kMasked) ? u.g : 0;
         const int b_grp = (LAYOUT == kDense || LAYOUT == kKGrouped) ? 0 : u.g;
         // MN-major B: the 128-wide column blocks of the tile that hold
         // columns below n (a block wholly past n is not loaded; the MMA
         // columns it feeds are never stored)
         const int b_blocks = kBMn ? min(BN / 128, (a.n - n0 + 127) / 128) : 1;
+        // K-major A: a tile with fewer than 128 valid rows (an M tail, the
+        // last block of a masked group) loads only the 32-row boxes that hold
+        // them; the MMA's remaining rows read stale shared memory and feed
+        // accumulator rows that are never stored
+        int a_boxes = 4;
+        if constexpr (!kAMn) {
+          int lim = a.rows;
+          if (LAYOUT == kMasked) lim = min(max(__ldg(a.masked_m + u.g), 0), a.rows);
+          a_boxes = max(1, min(4, (lim - a_row + 31) / 32));
+        }
+        const uint32_t a_bytes = (a_boxes == 4) ? (uint32_t)C::kABytes : (uint32_t)a_boxes * (32 * 128);
         const int32_t* sfa_g = a.sfa + (LAYOUT == kMasked ? (long long)u.g * a.sfa_group_words : 0);
         const int32_t* sfb_g = a.sfb + (long long)b_grp * a.sfb_group_words;
         for (int kb = kb0; kb < kb1; ++kb) {
@@ -494,42 +499,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          const bool new_sfa = !BF16 && (((kb & 3) == 0) || kb == kb0);
-          const bool new_sfb = !BF16 && (FP4 || new_sfa);
-          uint32_t bytes = C::kABytes + (kBMn ? (uint32_t)b_blocks * (kBK * 128) : (uint32_t)C::kBTxBytes);
+          const bool new_sfa = !BF16 && !kPromo && (((kb & 3) == 0) || kb == kb0);
+          const bool new_sfb = !BF16 && !kPromo && (FP4 || new_sfa);
+          uint32_t bytes = a_bytes + (kBMn ? (uint32_t)b_blocks * (kBK * 128) : (uint32_t)C::kBTxBytes);
           if (new_sfa) bytes += C::kSfaBytes;
           if (new_sfb) bytes += 512u * nchunks;
           DG_CHECK(((smem_u32(s_a + stage * C::kABytes) | smem_u32(s_b + stage * C::kBBytes)) & 1023) == 0 &&
                        u.mb < a.num_m_blocks && u.nb < a.num_n_blocks && kb < a.kb_total,
                    6);
-          if constexpr (kPair) {
-            // both CTAs' loads complete on the leader's barrier, which expects
-            // the bytes of both.  A cta_group::2 copy names its barrier by this
-            // CTA's shared address with the peer bit (bit 24) cleared.
-            const uint32_t bar = smem_u32(&full[stage]) & kPeerBitMask;
-            if (rank == 0) mbar_arrive_expect_tx(&full[stage], bytes * CTAS);
-            tma_load_3d_pair(s_a + stage * C::kABytes, &tm_a, bar, kb * kBK, a_row, 0);
-            tma_load_3d_pair(s_b + stage * C::kBBytes, &tm_b, bar, kb * kBK, n0 + (int)rank * C::kBRows, 0);
-            if (new_sfa) tma_load_2d_pair(s_sfa + stage * C::kSfaBytes, &tm_sfa, bar, 0,
-                                          (kb >> 2) * a.sfa_chunks + a_row / 128);
-            if (new_sfb) {
-              const int q = FP4 ? kb : (kb >> 2);
-              for (int ch = 0; ch < nchunks; ++ch)
-                tma_load_2d_pair(s_sfb + stage * C::kSfbBytes + ch * 512, &tm_sfb, bar, 0, q * a.sfb_chunks + c0 + ch);
-            }
-            filled_phase[stage] = phase;
-            filled_mask |= 1u << stage;
-            if (++stage == S) {
-              stage = 0;
-              phase ^= 1;
-            }
-            continue;
-          }
           mbar_arrive_expect_tx(&full[stage], bytes);
-          if constexpr (kAMn)
+          if constexpr (kAMn) {
             tma_load_3d(s_a + stage * C::kABytes, &tm_a, &full[stage], a_row, kb * kBK, a_grp);
-          else
+          } else if (a_boxes == 4) {
             tma_load_3d(s_a + stage * C::kABytes, &tm_a, &full[stage], kb * C::kKPerStage, a_row, a_grp);
+          } else {
+            // 32-row boxes land 4 KB apart, at 1024-byte-aligned addresses,
+            // so the 128-byte swizzle places their rows where one 128-row
+            // box would
+            for (int i = 0; i < a_boxes; ++i)
+              tma_load_3d(s_a + stage * C::kABytes + i * (32 * 128), &tm_a32, &full[stage], kb * C::kKPerStage,
+                          a_row + 32 * i, a_grp);
+          }
           if constexpr (kBMn) {
             for (int cb = 0; cb < b_blocks; ++cb)
               tma_load_3d(s_b + stage * C::kBBytes + cb * (kBK * 128), &tm_b, &full[stage], n0 + 128 * cb, kb * kBK,
@@ -561,10 +551,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (!ok && rank == 0) {
+      if (!ok) {
         // never leave copies in flight into shared memory: wait (bounded) for
-        // the last fill of every stage (a pair's fills all count on the
-        // leader's barriers; the final cluster barrier holds the peer)
+        // the last fill of every stage
         for (int s = 0; s < S; ++s)
           if (filled_mask & (1u << s)) {
             uint64_t t0 = global_timer_ns();
@@ -579,7 +568,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     // warp-wide loop with per-K-block warp synchronisation measured 1.8x
     // slower).  It also re-bases the B scale words when a tile starts an odd
     // number of 32-row groups into its first scale chunk.
-    if (lane == 0 && rank == 0) {
+    if (kPromo && lane == 0) {
+      // promotion: every K-block's four unscaled MMAs go to the next of the
+      // rotating partial-sum buffers, which the epilogue scales and frees
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t kcount = 0;
+      bool ok = true;
+      WorkIter<LAYOUT> it(a, cta_id, num_ctas);
+      Unit u;
+      while (ok && it.next(a, s_prefix, num_units, u)) {
+        for (int kb = u.kb0; kb < u.kb1; ++kb, ++kcount) {
+          const int buf = (int)(kcount % C::kAccBufs);
+          const uint32_t use = kcount / C::kAccBufs;
+          if (!dg_wait(&tempty[buf], (use & 1) ^ 1, s_abort, limit) || !dg_wait(&full[stage], phase, s_abort, limit)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d_t = tmem_base + C::kColAcc + buf * C::kAccStride;
+          const uint64_t adesc = sdesc_k_sw128(s_a + stage * C::kABytes);
+          const uint64_t bdesc = sdesc_k_sw128(s_b + stage * C::kBBytes);
+#pragma unroll
+          for (int ks = 0; ks < kBK / 32; ++ks)
+            tc_mma_f8f6f4(d_t, adesc + (uint64_t)(2 * ks), bdesc + (uint64_t)(2 * ks), C::kIdesc, ks > 0 ? 1u : 0u);
+          tc_commit(&empty[stage]);
+          tc_commit(&tfull[buf]);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      tc_commit(drain);
+      uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < limit) {
+      }
+    } else if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
@@ -656,20 +681,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             fence_proxy_async_smem();
           }
-          if (new_sfa) {
-            if constexpr (kPair)
-              tc_cp_32x128b_x4_pair(sfa_t, sdesc_sf_32x16(s_sfa + stage * C::kSfaBytes));
-            else
-              tc_cp_32x128b_x4(sfa_t, sdesc_sf_32x16(s_sfa + stage * C::kSfaBytes));
-          }
+          if (new_sfa) tc_cp_32x128b_x4(sfa_t, sdesc_sf_32x16(s_sfa + stage * C::kSfaBytes));
           if (new_sfb) {
             const int ncp = rebase ? C::kSfrChunks : nchunks;
             for (int ch = 0; ch < ncp; ++ch) {
-              const uint64_t sd = sdesc_sf_32x16((rebase ? sfb_reb : sfb_src) + ch * 512);
-              if constexpr (kPair)
-                tc_cp_32x128b_x4_pair(tmem_base + C::kColSfb + 4 * ch, sd);
-              else
-                tc_cp_32x128b_x4(tmem_base + C::kColSfb + 4 * ch, sd);
+              tc_cp_32x128b_x4(tmem_base + C::kColSfb + 4 * ch,
+                               sdesc_sf_32x16((rebase ? sfb_reb : sfb_src) + ch * 512));
             }
           }
           // K-major: a K-step of 32 e4m3 is 32 bytes along the swizzled rows
@@ -687,34 +704,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int ks = 0; ks < kBK / 32; ++ks) {
             const uint32_t idb = FP4 ? (uint32_t)ks : ida;
             const uint32_t idesc = C::kIdesc | kMajBits | (ida << 29) | (idb << 4);
-            if constexpr (kPair)
-              tc_mma_mxf8f6f4_pair(d_t, adesc + (uint64_t)(ks * 2), bdesc + (uint64_t)(ks * 2), idesc,
-                                   sfa_t | (ida << 30), sfb_t | (idb << 30), (kb > kb0 || ks > 0) ? 1u : 0u);
-            else
-              tc_mma_mxf8f6f4(d_t, adesc + kAStep * ks, bdesc + kBStep * ks, idesc, sfa_t | (ida << 30),
-                              sfb_t | (idb << 30), (kb > kb0 || ks > 0) ? 1u : 0u);
+            tc_mma_mxf8f6f4(d_t, adesc + kAStep * ks, bdesc + kBStep * ks, idesc, sfa_t | (ida << 30),
+                            sfb_t | (idb << 30), (kb > kb0 || ks > 0) ? 1u : 0u);
           }
-          if constexpr (kPair)
-            tc_commit_pair_mc(&empty[stage], 0x3);  // frees the stage in both CTAs
-          else
-            tc_commit(&empty[stage]);
+          tc_commit(&empty[stage]);
           if (++stage == S) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        if constexpr (kPair)
-          tc_commit_pair_mc(&tfull[buf], 0x3);  // both CTAs' epilogues may read
-        else
-          tc_commit(&tfull[buf]);
+        tc_commit(&tfull[buf]);
         ++local;
       }
       // all tcgen05 work of this thread complete before TMEM is released
-      if constexpr (kPair)
-        tc_commit_pair(drain);
-      else
-        tc_commit(drain);
+      tc_commit(drain);
       uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < limit) {
       }
@@ -732,7 +736,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nch_w = max(0, min(kChunks, kNch - half * kChunks));  // chunks of this warp
     uint8_t* stg = s_epi + (warp - 2) * (32 * 64);
     int local = 0;
-    // where this warp releases an accumulator buffer: the leader's barrier
     // C of one unit for this warp's 32 rows x kCols columns, loaded
     // coalesced: in load i the four lanes 4r..4r+3 read the four 16-byte
     // pieces of row 8i + r of each 32-column chunk, so one warp load covers 8
@@ -745,7 +748,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 4; ++i) dst[j][i] = make_uint4(0u, 0u, 0u, 0u);
       if (!want) return;
-      const int rr0 = uu.mb * kTileM + (int)rank * kBM + q * 32;
+      const int rr0 = uu.mb * kBM + q * 32;
       int lim = a.rows;
       if (LAYOUT == kMasked) lim = min(max(__ldg(a.masked_m + uu.g), 0), a.rows);
       const int cw = uu.nb * BN + half * kCols;
@@ -777,19 +780,170 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     };
+    // bf16 result of one 32-column chunk of the 32 rows r0 .. r0 + 31 (vr of
+    // them valid, below `lim`; group g of a grouped D) -> D
+    auto store_rows = [&](int col0, const uint32_t (&packed)[kEpiCols / 2], int r0, int vr, int g, int lim) {
+      const int row = r0 + (int)lane;
+      const long long grow = kGroupRows ? (long long)g * a.rows + row : row;
+      if (vr == 32) {
+        // full 32-row box: swizzled staging (64-byte rows) + TMA store
+        // 64-byte swizzle: the pattern XORs address bits 7-8 into 4-5, so the
+        // staging box needs 512-byte alignment
+        DG_CHECK((smem_u32(stg) & 511) == 0 && stg >= s_epi && stg + 2048 <= s_epi + C::kEpiBytes &&
+                     (col0 % 8) == 0 && r0 + 32 <= lim,
+                 7);
+        if (lane == 0) bulk_wait_group_read<0>();
+        __syncwarp();
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const int pos = ch ^ ((lane >> 1) & 3);
+          *reinterpret_cast<uint4*>(stg + lane * 64 + pos * 16) =
+              make_uint4(packed[4 * ch], packed[4 * ch + 1], packed[4 * ch + 2], packed[4 * ch + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&tm_d, stg, col0, r0, kGroupRows ? g : 0);
+          bulk_commit_group();
+        }
+      } else if ((int)lane < vr &&
+                 DG_CHECK((reinterpret_cast<uintptr_t>(a.d + grow * a.d_cols + col0) & 15) == 0 && row < lim, 2)) {
+        // partial box (M tail or masked group tail): predicated row stores
+        uint4* dst = reinterpret_cast<uint4*>(a.d + grow * a.d_cols + col0);
+#pragma unroll
+        for (int v = 0; v < kEpiCols / 8; ++v)
+          if (col0 + 8 * v < a.d_cols)
+            dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+      }
+    };
+    // D = bf16(acc + C) of one 32-column chunk: C (when given) comes from the
+    // staging box, where stage_c put it; the result overwrites it in place
+    auto add_c_pack = [&](const float (&acc)[kEpiCols], bool with_c, uint32_t (&packed)[kEpiCols / 2]) {
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint4 c4 = with_c ? *reinterpret_cast<const uint4*>(stg + lane * 64 + ((v ^ ((lane >> 1) & 3)) * 16))
+                                : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t cw[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const int i = 4 * v + h;
+          __nv_bfloat162 bv = __floats2bfloat162_rn(acc[2 * i] + __uint_as_float(cw[h] << 16),
+                                                    acc[2 * i + 1] + __uint_as_float(cw[h] & 0xFFFF0000u));
+          packed[i] = *reinterpret_cast<uint32_t*>(&bv);
+        }
+      }
+    };
     // one unit of look-ahead for C where registers allow
     constexpr bool kPrefetchC = (kChunks <= 3);
     uint4 cnext[kChunks][4];
     bool have_next_c = false;  // cnext holds C of the next unit this warp drains
     (void)cnext;
-    auto release_acc = [&](int b) {
-      if constexpr (kPair)
-        mbar_arrive_cluster(mapa_shared(&tempty[b], 0));
-      else
-        mbar_arrive(&tempty[b]);
-    };
+    auto release_acc = [&](int b) { mbar_arrive(&tempty[b]); };
     // the iterator runs one unit ahead, so each unit is decoded once and the
     // next unit (un) is known for the C prefetch
+    if constexpr (kPromo) {
+      // ---- promotion: for every K-block, read this warp's 32 rows x kCols
+      // columns of unscaled partial sums from TMEM, hand the buffer back to
+      // the MMA issuer, and add the partial times sa * sb into FP32
+      // registers (sa: the row's 1x128 code, sb: the 128x128 block's code);
+      // after the unit's last K-block, D = bf16(acc + C) as in the plain
+      // epilogue (or the FP32 sums to a workspace slot for a shared tile)
+      WorkIter<LAYOUT> it(a, cta_id, num_ctas);
+      Unit u;
+      uint32_t kcount = 0;
+      bool ok = true;
+      while (ok && it.next(a, s_prefix, num_units, u)) {
+        const int r0 = u.mb * kBM + q * 32;
+        const int vr = min(32, a.rows - r0);
+        const int colw = u.nb * BN + half * kCols;
+        const bool load_c = a.c != nullptr && u.slot < 0;
+        uint4 creg[kChunks][4];
+        load_c_rows(creg, u, load_c);
+        float acc[kChunks][kEpiCols];
+#pragma unroll
+        for (int j = 0; j < kChunks; ++j)
+#pragma unroll
+          for (int i = 0; i < kEpiCols; ++i) acc[j][i] = 0.f;
+        // this row's packed A word and the B block's word (the same for all
+        // rows of a 128-row block) of K-block group g4; the next group's
+        // words are loaded one group ahead
+        const int32_t* sfa_row = a.sfa + (long long)u.mb * 128 + lane * 4 + q;
+        const int32_t* sfb_blk = a.sfb + (long long)(colw / 128) * 128;
+        auto load_scales = [&](int g4, uint32_t& sa, uint32_t& sb) {
+          sa = (uint32_t)__ldg(sfa_row + (long long)g4 * a.sfa_chunks * 128);
+          sb = colw < a.n ? (uint32_t)__ldg(sfb_blk + (long long)g4 * a.sfb_chunks * 128) : 0x7F7F7F7Fu;
+        };
+        uint32_t sa_w, sb_w, sa_n = 0, sb_n = 0;
+        load_scales(u.kb0 >> 2, sa_w, sb_w);
+        if (((u.kb0 >> 2) + 1) * 4 < u.kb1) load_scales((u.kb0 >> 2) + 1, sa_n, sb_n);
+        for (int kb = u.kb0; kb < u.kb1; ++kb, ++kcount) {
+          if (kb > u.kb0 && (kb & 3) == 0) {
+            sa_w = sa_n;
+            sb_w = sb_n;
+            if (kb + 4 < u.kb1) load_scales((kb >> 2) + 1, sa_n, sb_n);
+          }
+          const int buf = (int)(kcount % C::kAccBufs);
+          const uint32_t use = kcount / C::kAccBufs;
+          int okw = 1;
+          if (lane == 0) okw = dg_wait(&tfull[buf], use & 1, s_abort, limit) ? 1 : 0;
+          okw = __shfl_sync(0xffffffffu, okw, 0);
+          if (!okw) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + C::kColAcc + buf * C::kAccStride +
+                                 (uint32_t)(half * kCols);
+          const int sh = 8 * (kb & 3);
+          const float scale = ue8m0_to_float((sa_w >> sh) & 0xFFu) * ue8m0_to_float((sb_w >> sh) & 0xFFu);
+#pragma unroll
+          for (int j = 0; j < kChunks; ++j) {
+            uint32_t part[kEpiCols];
+            tc_ld_32x32b_x32(t_row + j * kEpiCols, part);
+            tc_wait_ld_regs(part);
+            if (j == kChunks - 1) {
+              // the last TMEM load of this buffer has completed
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&tempty[buf]);
+            }
+#pragma unroll
+            for (int i = 0; i < kEpiCols; ++i) acc[j][i] = fmaf(scale, __uint_as_float(part[i]), acc[j][i]);
+          }
+        }
+        if (!ok) break;
+        if (u.slot >= 0) {
+          // a piece of a shared tile: FP32 sums to its workspace slot
+          float* tile_ws = a.ws + ((long long)u.sk * a.max_seg + u.slot) * (kBM * BN);
+#pragma unroll
+          for (int j = 0; j < kChunks; ++j) {
+            const int col0 = colw + j * kEpiCols;
+            float* dst_row = tile_ws + (q * 32 + (int)lane) * BN + (col0 - u.nb * BN);
+            if (j < nch_w && (int)lane < vr && col0 < a.n &&
+                DG_CHECK(a.ws != nullptr && u.sk < a.sk_tiles && u.slot < a.max_seg &&
+                             (reinterpret_cast<uintptr_t>(dst_row) & 15) == 0,
+                         3)) {
+#pragma unroll
+              for (int v = 0; v < kEpiCols / 4; ++v)
+                if (col0 + 4 * v < a.n)
+                  reinterpret_cast<float4*>(dst_row)[v] =
+                      make_float4(acc[j][4 * v], acc[j][4 * v + 1], acc[j][4 * v + 2], acc[j][4 * v + 3]);
+            }
+          }
+          continue;
+        }
+#pragma unroll
+        for (int j = 0; j < kChunks; ++j) {
+          const int col0 = colw + j * kEpiCols;
+          if (j < nch_w && vr > 0 && col0 < a.n) {
+            if (load_c) stage_c(creg[j]);
+            uint32_t packed[kEpiCols / 2];
+            add_c_pack(acc[j], load_c, packed);
+            store_rows(col0, packed, r0, vr, 0, a.rows);
+          }
+        }
+      }
+    } else {
     WorkIter<LAYOUT> it(a, cta_id, num_ctas);
     Unit u, un;
     bool has_un = it.next(a, s_prefix, num_units, un);
@@ -799,7 +953,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (LAYOUT == kContig && !u.valid) continue;
       const int buf = local % C::kAccBufs;
       const uint32_t use = (uint32_t)(local / C::kAccBufs);
-      const int r0 = u.mb * kTileM + (int)rank * kBM + q * 32;  // first row of this warp (in the group if masked)
+      const int r0 = u.mb * kBM + q * 32;  // first row of this warp (in the group if masked)
       int limit_rows = a.rows;
       if (LAYOUT == kMasked) limit_rows = min(max(__ldg(a.masked_m + u.g), 0), a.rows);
       const int vr = min(32, limit_rows - r0);
@@ -831,6 +985,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         load_c_rows(creg, u, load_c);
       }
+      if constexpr (LAYOUT == kContig) {
+        // The contiguous layout's precondition, checked once per m-block (on
+        // its first n-block) while the MMAs run: every row of a 128-row
+        // block carries the block's group (from its first row) or -1, and
+        // padding rows (-1) only follow the valid rows.  A block that mixes
+        // groups, or has a valid row after a padding row, is reported.
+        if (u.nb == 0 && half == 0) {
+          const int v = __ldg(a.m_indices + row);
+          const int next = (lane == 31 && q < 3) ? __ldg(a.m_indices + row + 1) : v;
+          const uint32_t pad = __ballot_sync(0xffffffffu, v == -1);
+          const uint32_t valid_rows = ~pad;  // must be lanes 0 .. j-1 only
+          const bool mixed = (v != u.g && v != -1) || (v == -1 && next != -1);
+          if (__any_sync(0xffffffffu, mixed) || (valid_rows & (valid_rows + 1u)) != 0u) {
+            if (lane == 0) record_error(-5 /* DG_ERR_BAD_METADATA */);
+          }
+        }
+      }
 
       int ok = 1;
       if (lane == 0 && !empty_k) ok = dg_wait(&tfull[buf], use & 1, s_abort, limit) ? 1 : 0;
@@ -842,37 +1013,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // bf16 result of one 32-column chunk of this warp's rows -> D
       auto store_chunk = [&](int col0, const uint32_t (&packed)[kEpiCols / 2]) {
-        if (vr == 32) {
-          // full 32-row box: swizzled staging (64-byte rows) + TMA store
-          // 64-byte swizzle: the pattern XORs address bits 7-8 into 4-5, so the
-          // staging box needs 512-byte alignment
-          DG_CHECK((smem_u32(stg) & 511) == 0 && stg >= s_epi && stg + 2048 <= s_epi + C::kEpiBytes &&
-                       (col0 % 8) == 0 && r0 + 32 <= (LAYOUT == kMasked ? limit_rows : a.rows),
-                   7);
-          if (lane == 0) bulk_wait_group_read<0>();
-          __syncwarp();
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            const int pos = ch ^ ((lane >> 1) & 3);
-            *reinterpret_cast<uint4*>(stg + lane * 64 + pos * 16) =
-                make_uint4(packed[4 * ch], packed[4 * ch + 1], packed[4 * ch + 2], packed[4 * ch + 3]);
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_3d(&tm_d, stg, col0, r0, kGroupRows ? u.g : 0);
-            bulk_commit_group();
-          }
-        } else if ((int)lane < vr &&
-                   DG_CHECK((reinterpret_cast<uintptr_t>(a.d + grow * a.d_cols + col0) & 15) == 0 && row < limit_rows,
-                            2)) {
-          // partial box (M tail or masked group tail): predicated row stores
-          uint4* dst = reinterpret_cast<uint4*>(a.d + grow * a.d_cols + col0);
-#pragma unroll
-          for (int v = 0; v < kEpiCols / 8; ++v)
-            if (col0 + 8 * v < a.d_cols)
-              dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
-        }
+        store_rows(col0, packed, r0, vr, u.g, limit_rows);
       };
 
       if (u.slot >= 0) {
@@ -889,7 +1030,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_wait_ld_regs(acc);
             float* dst_row = tile_ws + (q * 32 + (int)lane) * BN + (col0 - u.nb * BN);
             if ((int)lane < vr &&
-                DG_CHECK(!kPair && a.ws != nullptr && u.sk < a.sk_tiles && u.slot < a.max_seg && row < a.rows &&
+                DG_CHECK(a.ws != nullptr && u.sk < a.sk_tiles && u.slot < a.max_seg && row < a.rows &&
                              (reinterpret_cast<uintptr_t>(dst_row) & 15) == 0,
                          3)) {
               float4* dst = reinterpret_cast<float4*>(dst_row);
@@ -982,21 +1123,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) release_acc(buf);
       ++local;
     }
+    }  // (kPromo)
     if (lane == 0) bulk_wait_group_all();
     __syncwarp();
   }
 
   tc_fence_before();
-  if constexpr (kPair)
-    cluster_sync_all();  // the leader's MMAs (which also write the peer's TMEM) have drained
-  else
-    __syncthreads();
+  __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    if constexpr (kPair)
-      tmem_dealloc_pair(tmem_base, kTmemCols);
-    else
-      tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 

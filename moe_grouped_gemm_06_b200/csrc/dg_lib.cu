@@ -119,7 +119,6 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t
 
 struct Plan {
   int bn = 128;
-  int ctas = 1;           // 2: a cluster of two CTAs computes 256-row tiles (not launched)
   long long dp_tiles = 0; // tiles computed whole (all tiles when sk_tiles = 0)
   int sk_tiles = 0;       // stream-K tiles after them (dense only)
   int max_seg = 0;        // workspace slots per stream-K tile
@@ -215,8 +214,9 @@ int sk_max_segments(int sk_tiles, int kb, int G) {
 // (allow_sk) and only within ws_cap bytes of workspace (0: no cap).  Ties
 // keep whole tiles.
 // MN-major B (mn_b) is staged in 128-wide column blocks: widths 128 and 256.
+// only_bn: plan this block width alone (the promotion kernels are 128 wide).
 Plan plan_gemm(long long m_blocks, int n, int k, int sms, bool allow_sk, size_t ws_cap = 0, bool fp4 = false,
-               bool bf16 = false, bool mn_b = false) {
+               bool bf16 = false, bool mn_b = false, int only_bn = 0) {
   Plan best;
   best.cost = 1e300;
   const int kb = k / 128;
@@ -230,7 +230,11 @@ Plan plan_gemm(long long m_blocks, int n, int k, int sms, bool allow_sk, size_t 
     if (fp4) wc.per_kb = wc.per_kb_fp4;
     if (bf16) wc.per_kb = wc.per_kb_bf16;
     const int bn = wc.bn;
-    if (forced_block_n() ? bn != forced_block_n() : !wc.automatic) continue;
+    if (only_bn != 0) {
+      if (bn != only_bn) continue;
+    } else if (forced_block_n() ? bn != forced_block_n() : !wc.automatic) {
+      continue;
+    }
     if (mn_b && bn % 128 != 0) continue;
     // 64-wide tiles double the CTAs of a dense problem of at most two
     // m-blocks; elsewhere (and for the grouped layouts) they only add A reads
@@ -327,11 +331,11 @@ float* workspace(size_t bytes, cudaStream_t s) {
 
 // ------------------------------------------------------------ launches
 
-template <int BN, bool FP4, int LAYOUT, int CTAS, int EPI = dg::kEpiPlain, bool BF16 = false, int MAJ = dg::kMajorK>
-dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td, const CUtensorMap& tsfa,
-                      const CUtensorMap& tsfb, const dg::GemmArgs& args, int grid, cudaStream_t s) {
-  using C = dg::Cfg<BN, FP4, CTAS, BF16, (LAYOUT == dg::kMasked || LAYOUT == dg::kKGrouped)>;
-  auto kern = dg::gemm_kernel<BN, FP4, LAYOUT, CTAS, EPI, BF16, MAJ>;
+template <int BN, bool FP4, int LAYOUT, int EPI = dg::kEpiPlain, bool BF16 = false, int MAJ = dg::kMajorK>
+dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& ta32, const CUtensorMap& tb, const CUtensorMap& td,
+                      const dg::GemmArgs& args, int grid, cudaStream_t s) {
+  using C = dg::Cfg<BN, FP4, BF16, (LAYOUT == dg::kMasked || LAYOUT == dg::kKGrouped)>;
+  auto kern = dg::gemm_kernel<BN, FP4, LAYOUT, EPI, BF16, MAJ>;
   static std::atomic<uint64_t> attr_set_mask{0};  // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
@@ -341,7 +345,7 @@ dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
       return DG_ERR_CUDA;
     attr_set_mask.fetch_or(bit);
   }
-  if (launch(kern, dim3(grid), dim3(dg::kThreads), C::kSmemBytes, s, CTAS, ta, tb, td, tsfa, tsfb, args) !=
+  if (launch(kern, dim3(grid), dim3(dg::kThreads), C::kSmemBytes, s, 1, ta, ta32, tb, td, args) !=
       cudaSuccess)
     return DG_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -349,18 +353,14 @@ dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
 }
 
 template <bool FP4, int LAYOUT, int EPI = dg::kEpiPlain, bool BF16 = false, int MAJ = dg::kMajorK>
-dg_status dispatch(int bn, int ctas, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
-                   const CUtensorMap& tsfa, const CUtensorMap& tsfb, const dg::GemmArgs& args, int grid,
-                   cudaStream_t s) {
-  // CTA-pair (cta_group::2) kernels are not launched: on B200 they stopped
-  // with "illegal instruction" and the cause is not yet known.
-  if (ctas != 1) return DG_ERR_UNSUPPORTED;
+dg_status dispatch(int bn, const CUtensorMap& ta, const CUtensorMap& ta32, const CUtensorMap& tb,
+                   const CUtensorMap& td, const dg::GemmArgs& args, int grid, cudaStream_t s) {
   if constexpr (MAJ != dg::kMajorK) {
     // MN-major operands: FP8, plain epilogue, 128-wide column blocks
     static_assert(!FP4 && !BF16 && EPI == dg::kEpiPlain, "MN-major: FP8, plain epilogue");
     switch (bn) {
-      case 128: return launch_gemm<128, false, LAYOUT, 1, EPI, false, MAJ>(ta, tb, td, tsfa, tsfb, args, grid, s);
-      case 256: return launch_gemm<256, false, LAYOUT, 1, EPI, false, MAJ>(ta, tb, td, tsfa, tsfb, args, grid, s);
+      case 128: return launch_gemm<128, false, LAYOUT, EPI, false, MAJ>(ta, ta32, tb, td, args, grid, s);
+      case 256: return launch_gemm<256, false, LAYOUT, EPI, false, MAJ>(ta, ta32, tb, td, args, grid, s);
       default: return DG_ERR_UNSUPPORTED;
     }
   } else if constexpr (LAYOUT == dg::kKGrouped) {
@@ -368,27 +368,32 @@ dg_status dispatch(int bn, int ctas, const CUtensorMap& ta, const CUtensorMap& t
   } else if constexpr (BF16) {
     // bf16: dense tiles of the widths the heuristic picks
     switch (bn) {
-      case 64: return launch_gemm<64, false, LAYOUT, 1, EPI, true>(ta, tb, td, tsfa, tsfb, args, grid, s);
-      case 128: return launch_gemm<128, false, LAYOUT, 1, EPI, true>(ta, tb, td, tsfa, tsfb, args, grid, s);
-      case 192: return launch_gemm<192, false, LAYOUT, 1, EPI, true>(ta, tb, td, tsfa, tsfb, args, grid, s);
-      case 256: return launch_gemm<256, false, LAYOUT, 1, EPI, true>(ta, tb, td, tsfa, tsfb, args, grid, s);
+      case 64: return launch_gemm<64, false, LAYOUT, EPI, true>(ta, ta32, tb, td, args, grid, s);
+      case 128: return launch_gemm<128, false, LAYOUT, EPI, true>(ta, ta32, tb, td, args, grid, s);
+      case 192: return launch_gemm<192, false, LAYOUT, EPI, true>(ta, ta32, tb, td, args, grid, s);
+      case 256: return launch_gemm<256, false, LAYOUT, EPI, true>(ta, ta32, tb, td, args, grid, s);
       default: return DG_ERR_UNSUPPORTED;
     }
+  } else if constexpr (EPI == dg::kEpiPromote) {
+    // per-K-block promotion: e4m3 A and B, 128-wide tiles
+    static_assert(!FP4 && LAYOUT == dg::kDense, "promotion: dense e4m3");
+    if (bn != 128) return DG_ERR_UNSUPPORTED;
+    return launch_gemm<128, false, LAYOUT, EPI>(ta, ta32, tb, td, args, grid, s);
   } else if constexpr (EPI == dg::kEpiSwiGlu) {
     // SwiGLU tiles hold whole (64 gate, 64 up) row blocks: widths 128, 256
     switch (bn) {
-      case 128: return launch_gemm<128, FP4, LAYOUT, 1, EPI>(ta, tb, td, tsfa, tsfb, args, grid, s);
-      case 256: return launch_gemm<256, FP4, LAYOUT, 1, EPI>(ta, tb, td, tsfa, tsfb, args, grid, s);
+      case 128: return launch_gemm<128, FP4, LAYOUT, EPI>(ta, ta32, tb, td, args, grid, s);
+      case 256: return launch_gemm<256, FP4, LAYOUT, EPI>(ta, ta32, tb, td, args, grid, s);
       default: return DG_ERR_UNSUPPORTED;
     }
   } else {
     switch (bn) {
-      case 64: return launch_gemm<64, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
-      case 128: return launch_gemm<128, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
-      case 160: return launch_gemm<160, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
-      case 192: return launch_gemm<192, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
-      case 224: return launch_gemm<224, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
-      case 256: return launch_gemm<256, FP4, LAYOUT, 1>(ta, tb, td, tsfa, tsfb, args, grid, s);
+      case 64: return launch_gemm<64, FP4, LAYOUT>(ta, ta32, tb, td, args, grid, s);
+      case 128: return launch_gemm<128, FP4, LAYOUT>(ta, ta32, tb, td, args, grid, s);
+      case 160: return launch_gemm<160, FP4, LAYOUT>(ta, ta32, tb, td, args, grid, s);
+      case 192: return launch_gemm<192, FP4, LAYOUT>(ta, ta32, tb, td, args, grid, s);
+      case 224: return launch_gemm<224, FP4, LAYOUT>(ta, ta32, tb, td, args, grid, s);
+      case 256: return launch_gemm<256, FP4, LAYOUT>(ta, ta32, tb, td, args, grid, s);
       default: return DG_ERR_UNSUPPORTED;
     }
   }
@@ -420,7 +425,7 @@ int k_plan_mn(const Problem& p) { return std::max(128, (int)(p.k / p.groups) / 1
 // The plan a call of this layout and operand kind runs (block width, schedule,
 // grid), as run_gemm launches it; dg_query_config reports it.
 Plan select_plan(const Problem& p, int layout, bool fp4, bool bf16, bool mn, bool swiglu, int sms,
-                 size_t ws_cap) {
+                 size_t ws_cap, bool promote = false) {
   // a bf16 stage covers 64 K-elements in the time an e4m3 stage covers 128:
   // the planner sees bf16 as an e4m3 problem of twice the K
   const int k_plan = bf16 ? 2 * p.k : p.k;
@@ -437,7 +442,7 @@ Plan select_plan(const Problem& p, int layout, bool fp4, bool bf16, bool mn, boo
     plan = plan_gemm((long long)p.groups * m_blocks, p.n, k_plan_mn(p), sms, false, 0, false, false, true);
   } else {
     // MN-major operands run in 128- and 256-wide tiles only
-    plan = plan_gemm(m_blocks, p.n, k_plan, sms, layout == dg::kDense, ws_cap, fp4, bf16, mn);
+    plan = plan_gemm(m_blocks, p.n, k_plan, sms, layout == dg::kDense, ws_cap, fp4, bf16, mn, promote ? 128 : 0);
   }
   return plan;
 }
@@ -462,7 +467,7 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
   if (sms <= 0) return DG_ERR_CUDA;
   const long long m_blocks = ceil_div(p.rows, dg::kBM);
   const Plan plan = select_plan(p, LAYOUT, FP4, BF16, MAJ != dg::kMajorK, EPI == dg::kEpiSwiGlu, sms,
-                                fixed_ws != nullptr ? fixed_ws_bytes : 0);
+                                fixed_ws != nullptr ? fixed_ws_bytes : 0, EPI == dg::kEpiPromote);
   if (plan.grid <= 0) return DG_ERR_UNSUPPORTED;  // (a forced width this layout cannot use)
 
   dg::GemmArgs args{};
@@ -479,7 +484,7 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
   args.d_cols = (EPI == dg::kEpiSwiGlu) ? p.n / 2 : p.n;
   args.k = p.k;
   args.num_groups = p.groups;
-  args.num_m_blocks = (int)(plan.ctas == 2 ? ceil_div(p.rows, 2 * dg::kBM) : m_blocks);
+  args.num_m_blocks = (int)m_blocks;
   args.num_n_blocks = (int)ceil_div(p.n, plan.bn);
   args.kb_total = p.k / (BF16 ? 64 : 128);
   args.dp_tiles = (int)plan.dp_tiles;
@@ -515,11 +520,14 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
   const int gb = (LAYOUT == dg::kDense || LAYOUT == dg::kKGrouped) ? 1 : p.groups;
   const int gd = (LAYOUT == dg::kMasked || LAYOUT == dg::kKGrouped) ? p.groups : 1;
   const uint64_t k_ext = (uint64_t)std::max(p.k, 128);  // K rows of MN-major maps
-  CUtensorMap ta, tb, td;
+  // ta32: the same A in boxes of 32 rows, for tiles with fewer valid rows
+  CUtensorMap ta, ta32, tb, td;
   bool ok;
   if (BF16) {
     ok = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.a, p.k, p.rows, ga, (uint64_t)p.k * 2,
                   (uint64_t)p.rows * p.k * 2, 64, dg::kBM, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && make_map(&ta32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.a, p.k, p.rows, ga, (uint64_t)p.k * 2,
+                        (uint64_t)p.rows * p.k * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.b, p.k, p.n, gb, (uint64_t)p.k * 2,
                         (uint64_t)p.n * p.k * 2, 64, plan.bn, CU_TENSOR_MAP_SWIZZLE_128B);
   } else if (kAMn) {
@@ -527,9 +535,12 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
     // (K = 0, all groups empty: a map of one box that no load reads)
     ok = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.a, p.rows, k_ext, ga, (uint64_t)p.rows,
                   (uint64_t)p.rows * k_ext, dg::kBM, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ta32 = ta;  // (not used: MN-major tiles are never trimmed)
   } else {
     ok = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.a, p.k, p.rows, ga, (uint64_t)p.k, (uint64_t)p.rows * p.k,
                   128, dg::kBM, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && make_map(&ta32, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.a, p.k, p.rows, ga, (uint64_t)p.k,
+                        (uint64_t)p.rows * p.k, 128, 32, CU_TENSOR_MAP_SWIZZLE_128B);
   }
   if (BF16) {
   } else if (kBMn)
@@ -538,22 +549,10 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
                         128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   else if (FP4)
     ok = ok && make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, p.b, p.k, p.n, gb, (uint64_t)p.k / 2,
-                        (uint64_t)p.n * p.k / 2, 128, plan.bn / plan.ctas, CU_TENSOR_MAP_SWIZZLE_128B);
+                        (uint64_t)p.n * p.k / 2, 128, plan.bn, CU_TENSOR_MAP_SWIZZLE_128B);
   else
     ok = ok && make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.b, p.k, p.n, gb, (uint64_t)p.k, (uint64_t)p.n * p.k,
-                        128, plan.bn / plan.ctas, CU_TENSOR_MAP_SWIZZLE_128B);
-  // packed scale words as rows of 128 words (one 128-row chunk per row): the
-  // CTA-pair kernel loads them with tiled copies that can complete on the
-  // leader's barrier; single-CTA kernels use plain bulk copies instead
-  CUtensorMap tsfa = ta, tsfb = ta;
-  if (plan.ctas == 2) {
-    const uint64_t rows_a = (uint64_t)args.sfa_q * args.sfa_chunks;
-    const uint64_t rows_b = (uint64_t)args.sfb_q * args.sfb_chunks;
-    ok = ok && make_map(&tsfa, CU_TENSOR_MAP_DATA_TYPE_INT32, p.sfa, 128, rows_a, 1, 512, rows_a * 512, 128, 1,
-                        CU_TENSOR_MAP_SWIZZLE_NONE);
-    ok = ok && make_map(&tsfb, CU_TENSOR_MAP_DATA_TYPE_INT32, p.sfb, 128, rows_b, 1, 512, rows_b * 512, 128, 1,
-                        CU_TENSOR_MAP_SWIZZLE_NONE);
-  }
+                        128, plan.bn, CU_TENSOR_MAP_SWIZZLE_128B);
   ok = ok && make_map(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.d, args.d_cols, p.rows, gd, (uint64_t)args.d_cols * 2,
                       (uint64_t)p.rows * args.d_cols * 2, dg::kEpiCols, 32, CU_TENSOR_MAP_SWIZZLE_64B);
   if (!ok) return DG_ERR_CUDA;
@@ -565,7 +564,7 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
                  LAYOUT, (int)FP4, p.rows, p.n, p.k, p.groups, plan.bn, plan.dp_tiles, plan.sk_tiles, plan.sk_split,
                  plan.max_seg, plan.grid, plan.cost);
 
-  dg_status st = dispatch<FP4, LAYOUT, EPI, BF16, MAJ>(plan.bn, plan.ctas, ta, tb, td, tsfa, tsfb, args, plan.grid, s);
+  dg_status st = dispatch<FP4, LAYOUT, EPI, BF16, MAJ>(plan.bn, ta, ta32, tb, td, args, plan.grid, s);
   if (st != DG_OK || plan.sk_tiles == 0) return st;
 
   dg::SkReduceArgs r{};
@@ -632,31 +631,70 @@ dg_status dg_fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const
 // ---------------------------------------------------------------- no-alloc
 //
 // Scratch of dg_fp8_gemm_nt_noalloc: one fixed array per device, part of
-// this library's device image, so it exists on every GPU that loads the
-// library until the process exits.  All calls on a device share it.
+// this library's device image.  It is committed on a device when the module
+// is loaded there (with CUDA's lazy module loading, at the first kernel
+// launch or symbol lookup of this library on that device) and held until the
+// process exits.  All calls on a device share it.
 namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
 }  // namespace
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
 
 namespace {
+// Device address of g_noalloc_scratch, cached per device together with the
+// context it was looked up in: after a device reset (or any other change of
+// the current context) the module is loaded anew and the array may move, so
+// a context that differs from the cached one triggers a new lookup.
+struct NoAllocAddr {
+  std::atomic<void*> ctx{nullptr};
+  std::atomic<float*> addr{nullptr};
+};
+NoAllocAddr g_noalloc_addr[64];
 std::mutex g_noalloc_mutex;
-float* g_noalloc_addr[64] = {};
 
-// Device address of g_noalloc_scratch on the current device.  Host code
-// only holds a stand-in symbol for the array, so the address is looked up
-// once per device, with that device current, and cached.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+CUcontext current_context() {
+  static CtxGetCurrentFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (CtxGetCurrentFn) nullptr;
+    return reinterpret_cast<CtxGetCurrentFn>(p);
+  }();
+  CUcontext ctx = nullptr;
+  if (fn == nullptr || fn(&ctx) != CUDA_SUCCESS) return nullptr;
+  return ctx;
+}
+
+// Host code holds only a stand-in symbol for the array, so its device address
+// is looked up with the device current (cudaGetSymbolAddress allocates
+// nothing); the lock is taken only for a lookup, not on the cached path.
 dg_status noalloc_scratch(float** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DG_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return DG_ERR_CUDA;
-    g_noalloc_addr[dev] = static_cast<float*>(p);
+  NoAllocAddr& e = g_noalloc_addr[dev];
+  void* ctx = current_context();
+  if (ctx != nullptr && e.ctx.load(std::memory_order_acquire) == ctx) {
+    *out = e.addr.load(std::memory_order_relaxed);
+    return DG_OK;
   }
-  *out = g_noalloc_addr[dev];
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return DG_ERR_CUDA;
+  e.addr.store(static_cast<float*>(p), std::memory_order_relaxed);
+  e.ctx.store(current_context(), std::memory_order_release);  // (the lookup made the primary context current)
+  *out = static_cast<float*>(p);
   return DG_OK;
+}
+
+void forget_noalloc_addresses() {
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  for (NoAllocAddr& e : g_noalloc_addr) {
+    e.ctx.store(nullptr, std::memory_order_release);
+    e.addr.store(nullptr, std::memory_order_relaxed);
+  }
 }
 }  // namespace
 
@@ -676,6 +714,16 @@ dg_status dg_fp8_gemm_nt_noalloc(const void* a, const int32_t* sfa, const void* 
 }
 
 size_t dg_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+dg_status dg_fp8_gemm_nt_promoted(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                                  const void* c, void* d, int m, int n, int k, void* stream) {
+  if (m < 0) return DG_ERR_INVALID_ARG;
+  dg_status st = check_common(a, sfa, b, sfb, c, d, n, k);
+  if (st != DG_OK) return st;
+  if (m == 0) return DG_OK;
+  Problem p{a, sfa, b, sfb, c, d, nullptr, nullptr, m, n, k, 1, 0};
+  return run_gemm<false, dg::kDense, dg::kEpiPromote>(p, static_cast<cudaStream_t>(stream));
+}
 
 dg_status dg_bf16_gemm_nt(const void* a, const void* b, const void* c, void* d, int m, int n, int k, void* stream) {
   if (m < 0 || !a || !b || !d || !aligned16(a) || !aligned16(b) || !aligned16(d) || (c && !aligned16(c)))
@@ -999,6 +1047,7 @@ int64_t dg_num_tiles(int m, int n, int block_m, int block_n) {
 }
 
 void dg_shutdown(void) {
+  forget_noalloc_addresses();
   std::lock_guard<std::mutex> lock(g_ws_mutex);
   int prev = 0;
   cudaGetDevice(&prev);

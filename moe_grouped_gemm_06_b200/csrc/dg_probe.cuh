@@ -21,17 +21,6 @@ namespace dg {
 
 enum : int { kProbeScaled = 0, kProbePlain = 1, kProbeBf16 = 2 };
 
-// D (+)= A * B^T with A, B e4m3 (kind::f8f6f4), no scale factors.
-__device__ __forceinline__ void tc_mma_f8f6f4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                              uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // Instruction descriptor of kind::f8f6f4: FP32 accumulator (bits 4-5 = 1),
 // A and B e4m3 (formats 0), both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
 __host__ __device__ constexpr uint32_t idesc_f8f6f4(int m, int n) {

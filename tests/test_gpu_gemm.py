@@ -661,6 +661,30 @@ def test_contiguous_group_index_out_of_range_is_reported(dg):
     assert dg.dg_get_last_error() == -5
 
 
+@pytest.mark.parametrize("kind", ["two_groups_in_a_block", "valid_row_after_padding", "padding_then_valid_warp"])
+def test_contiguous_block_precondition_is_reported(dg, kind):
+    # every 128-row block holds one group's rows, then padding (-1): a block
+    # that mixes groups or has a valid row after a padding row is reported
+    N, K = 128, 256
+    cs = _contiguous_case(7200, 2, 100, 120, N, K)
+    mi = cs["mi"].copy()
+    r0 = int(cs["rows"][0])                  # first padding row of block 0
+    assert 100 <= r0 < 128 and mi[r0] == -1
+    if kind == "two_groups_in_a_block":
+        mi[40] = 1                           # a row of group 1 inside group 0's block
+    elif kind == "valid_row_after_padding":
+        mi[127] = 0                          # group 0 again after its padding
+    else:
+        mi[32:64] = -1                       # a padding warp-row group, then valid rows
+    cs["mi"] = mi
+    _run_contiguous(dg, cs, N)
+    assert dg.dg_get_last_error() == -5
+    # the untouched layout reports nothing
+    cs["mi"] = _contiguous_case(7200, 2, 100, 120, N, K)["mi"]
+    _run_contiguous(dg, cs, N)
+    assert dg.dg_get_last_error() == 0
+
+
 # ------------------------------------------------- NN contiguous (B [G, K, N])
 
 def _nn_case(seed, G, lo, hi, N, K):

@@ -67,3 +67,34 @@ def test_noalloc_keeps_within_its_scratch(dg):
         dg.dg_set_num_sms(0)
     assert free["workspace_bytes"] > dg.dg_noalloc_scratch_bytes()
     assert capped["workspace_bytes"] <= dg.dg_noalloc_scratch_bytes()
+
+
+def test_noalloc_reserves_no_device_memory(dg):
+    # The property the call exists for.  On a stream the library has not used
+    # yet, the allocating call must create a new stream-K workspace (device
+    # memory reserved), while the no-alloc call on another new stream must
+    # leave the device's free memory unchanged.
+    M, N, K = 64, 7168, 16384
+    cfg = dg.dg_query_dense_config(M, N, K, workspace_cap=dg.dg_noalloc_scratch_bytes())
+    assert cfg["sk_tiles"] > 0 and cfg["workspace_bytes"] > 0
+    p = Dense(8100, M, N, K, with_c=True).upload()
+    d = torch.empty((M, N), dtype=torch.int16, device="cuda")
+    dg.dg_fp8_gemm_nt_noalloc(p.t_a, p.t_sfa, p.t_b, p.t_sfb, p.t_c, d)   # warm-up (module, address)
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+    s1 = torch.cuda.Stream()
+    free0, _ = torch.cuda.mem_get_info()
+    with torch.cuda.stream(s1):
+        dg.dg_fp8_gemm_nt_noalloc(p.t_a, p.t_sfa, p.t_b, p.t_sfb, p.t_c, d, stream=s1)
+    s1.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, f"no-alloc call changed free device memory by {free0 - free1} bytes"
+    check_close(bf16_dev_to_f64(d), p.ref(), "noalloc on a new stream")
+
+    s2 = torch.cuda.Stream()
+    with torch.cuda.stream(s2):
+        dg.dg_fp8_gemm_nt(p.t_a, p.t_sfa, p.t_b, p.t_sfb, p.t_c, d, stream=s2)
+    s2.synchronize()
+    free2, _ = torch.cuda.mem_get_info()
+    assert free2 < free1, "control: the allocating call should have reserved a workspace"
