@@ -49,10 +49,13 @@
  * device-side error word and reported later by dg_get_last_error().
  *
  * Scratch memory.  When the host heuristic shares the K-iterations of some
- * tiles out over several CTAs (stream-K: small M, or the last partial wave of
- * tiles), the dense calls keep their FP32 partial sums in a workspace per
- * (device, stream), allocated stream-ordered on first use and grown on
- * demand; dg_shutdown() releases it.  No other call allocates device memory.
+ * tiles out over several CTAs of a launch (per-tile K-slices or stream-K,
+ * mostly the last partial wave of tiles), the dense calls keep their FP32
+ * partial sums in a workspace per (device, stream), allocated stream-ordered
+ * on first use and grown on demand; dg_shutdown() releases it.  A dense plan
+ * that splits every tile over a thread-block cluster (small M) sums the
+ * partials in the cluster's shared memory and needs none.  No other call
+ * allocates device memory.
  */
 #ifndef DG_H_
 #define DG_H_
@@ -347,7 +350,10 @@ int dg_get_pdl(void);
  * 256; the others are only used when forced) and schedule 0 (heuristic), 1
  * (whole tiles only), 2 (the last tiles cut into per-tile K-slices, one per
  * CTA) or 3 (stream-K: the last tiles' K-iterations shared evenly over the
- * grid); 2 and 3 apply to the dense calls whenever such a split exists.
+ * grid), 4, 5 or 6 (every tile's K-blocks cut into 2, 4 or 8 slices
+ * computed by the CTAs of one thread-block cluster and summed through
+ * distributed shared memory; 128- and 256-wide dense NT tiles); 2 to 6 apply
+ * to the dense calls whenever such a split exists.
  * Anything else returns DG_ERR_INVALID_ARG and changes nothing.  Meant for
  * tuning and tests.  The environment variables DG_BLOCK_N and DG_SCHEDULE set
  * the initial values. */
@@ -388,6 +394,15 @@ uint64_t dg_launch_count(void);
 dg_status dg_query_dense_config(int m, int n, int k, int64_t workspace_cap, int* block_n, int* dp_tiles,
                                 int* sk_tiles, int* sk_split, int* max_segments, int* grid,
                                 int64_t* workspace_bytes);
+
+/* Cluster split of the dense plan for (m, n, k) with at most workspace_cap
+ * bytes of workspace: S > 0 when every output tile's K-blocks are cut into S
+ * slices computed by the S CTAs of one thread-block cluster, whose FP32
+ * partial sums are added through distributed shared memory inside the same
+ * kernel (no workspace, no second kernel; the plan dg_query_dense_config then
+ * reports as dp_tiles = the tiles, sk_tiles = 0, grid = tiles x S); 0 when the
+ * plan is another one; -1 for invalid sizes. */
+int dg_query_dense_cluster_split(int m, int n, int k, int64_t workspace_cap);
 
 /* Layouts named by dg_query_config. */
 enum { DG_LAYOUT_DENSE = 0, DG_LAYOUT_CONTIGUOUS = 1, DG_LAYOUT_MASKED = 2 };

@@ -48,7 +48,11 @@ constexpr int kMaxMaskedGroups = 1024;
 
 // kKGrouped: the weight-gradient layout, grouped along K -- group g owns the
 // K rows [K_0 + ... + K_(g-1), ... + K_g) of A and B and its own D[g].
-enum : int { kDense = 0, kContig = 1, kMasked = 2, kKGrouped = 3 };
+// kDenseSplit: the dense layout with every tile's K-blocks cut into `split`
+// slices computed by the CTAs of one thread-block cluster, whose FP32 partial
+// sums are added through distributed shared memory (no workspace, no second
+// kernel); for problems with too few tiles to fill the SMs.
+enum : int { kDense = 0, kContig = 1, kMasked = 2, kKGrouped = 3, kDenseSplit = 4 };
 
 // Operand majorness (template parameter MAJ): which of A and B are stored
 // MN-major (M or N contiguous, K rows) instead of K-major.
@@ -117,6 +121,7 @@ struct GemmArgs {
   // A tile's pieces land in its max_seg workspace slots.
   int dp_tiles, sk_tiles, max_seg, sk_split;
   long long sk_iters;
+  int split;                           // kDenseSplit: CTAs (K-slices) per tile = cluster size
   int sfa_chunks, sfb_chunks;          // ceil(rows/128), ceil(n/128)
   long long sfa_group_words, sfb_group_words;
   int sfa_q, sfb_q;                    // packed groups along K
@@ -248,6 +253,7 @@ struct WorkIter {
 
   __device__ __forceinline__ WorkIter(const GemmArgs& a, int cta_, int G) : t(cta_), step(G), cta(cta_) {
     x = x_end = 0;
+    if (LAYOUT == kDenseSplit) x_end = 1;  // one unit: this CTA's slice of its tile
     if (LAYOUT == kDense && a.sk_tiles > 0) {
       if (a.sk_split > 0) {
         x_end = (cta_ < a.sk_tiles * a.sk_split) ? 1 : 0;  // one piece
@@ -265,6 +271,15 @@ struct WorkIter {
     u.sk = 0;
     u.kb0 = 0;
     u.kb1 = a.kb_total;
+    if (LAYOUT == kDenseSplit) {
+      if (x >= x_end) return false;
+      const int r = cta % a.split;  // = the CTA's rank in its cluster
+      raster_tile_fast(cta / a.split, a, u.mb, u.nb);
+      u.kb0 = (int)((long long)r * a.kb_total / a.split);
+      u.kb1 = (int)((long long)(r + 1) * a.kb_total / a.split);
+      x = x_end;
+      return true;
+    }
     if (t < num_units) {
       if (LAYOUT == kMasked) {
         // the group whose tile range holds t: s_prefix[g] <= t < s_prefix[g + 1]
@@ -345,6 +360,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   static_assert(LAYOUT != kKGrouped || MAJ == (kAMajorMN | kBMajorMN), "k-grouped: A and B MN-major");
   // D and C of the masked and k-grouped layouts are [groups][rows][n]
   constexpr bool kGroupRows = (LAYOUT == kMasked || LAYOUT == kKGrouped);
+  // split tiles: row pitch (floats) of a slice's partial sums in shared memory
+  // (4 floats of padding put the rows of a warp's float4 stores in distinct banks)
+  constexpr int kSplitPitch = BN + 4;
+  static_assert(LAYOUT != kDenseSplit || kBM * kSplitPitch * 4 <= C::kStages * C::kStageBytes,
+                "a split tile's partial sums fit in the stage ring");
+  static_assert(LAYOUT != kDenseSplit || (EPI == kEpiPlain && MAJ == kMajorK), "split tiles: dense NT, plain");
   constexpr int S = C::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -896,20 +917,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  (uint32_t)(half * kCols);
           const int sh = 8 * (kb & 3);
           const float scale = ue8m0_to_float((sa_w >> sh) & 0xFFu) * ue8m0_to_float((sb_w >> sh) & 0xFFu);
+          // both chunks' loads in flight at once, one wait, then the buffer
+          // goes back to the MMA issuer before the FMAs
+          uint32_t part[kChunks][kEpiCols];
 #pragma unroll
-          for (int j = 0; j < kChunks; ++j) {
-            uint32_t part[kEpiCols];
-            tc_ld_32x32b_x32(t_row + j * kEpiCols, part);
-            tc_wait_ld_regs(part);
-            if (j == kChunks - 1) {
-              // the last TMEM load of this buffer has completed
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&tempty[buf]);
-            }
+          for (int j = 0; j < kChunks; ++j) tc_ld_32x32b_x32(t_row + j * kEpiCols, part[j]);
 #pragma unroll
-            for (int i = 0; i < kEpiCols; ++i) acc[j][i] = fmaf(scale, __uint_as_float(part[i]), acc[j][i]);
-          }
+          for (int j = 0; j < kChunks; ++j) tc_wait_ld_regs(part[j]);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[buf]);
+#pragma unroll
+          for (int j = 0; j < kChunks; ++j)
+#pragma unroll
+            for (int i = 0; i < kEpiCols; ++i) acc[j][i] = fmaf(scale, __uint_as_float(part[j][i]), acc[j][i]);
         }
         if (!ok) break;
         if (u.slot >= 0) {
@@ -964,7 +985,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int colw = u.nb * BN + half * kCols;  // first column of this warp
 
       uint4 creg[kChunks][4];
-      const bool load_c = a.c != nullptr && u.slot < 0;
+      // (a split tile adds C when its slices are summed, after the loop)
+      const bool load_c = a.c != nullptr && u.slot < 0 && LAYOUT != kDenseSplit;
       if constexpr (kPrefetchC) {
         if (have_next_c) {
           // C of this unit was loaded while the previous unit was stored
@@ -1015,6 +1037,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto store_chunk = [&](int col0, const uint32_t (&packed)[kEpiCols / 2]) {
         store_rows(col0, packed, r0, vr, u.g, limit_rows);
       };
+
+      if constexpr (LAYOUT == kDenseSplit) {
+        // ---- this CTA's K-slice of a split tile: its FP32 sums go to this
+        // CTA's shared memory (the stage ring, idle once the last MMA has
+        // completed), [kBM][BN + 4] floats; they are summed after the loop
+        float* part = reinterpret_cast<float*>(smem) + (q * 32 + (int)lane) * kSplitPitch + half * kCols;
+#pragma unroll
+        for (int j = 0; j < kChunks; ++j) {
+          if (j < nch_w) {
+            uint32_t acc[kEpiCols];
+            tc_ld_32x32b_x32(t_row + j * kEpiCols, acc);
+            tc_wait_ld_regs(acc);
+#pragma unroll
+            for (int v = 0; v < kEpiCols / 4; ++v)
+              *reinterpret_cast<float4*>(part + j * kEpiCols + 4 * v) =
+                  make_float4(__uint_as_float(acc[4 * v]), __uint_as_float(acc[4 * v + 1]),
+                              __uint_as_float(acc[4 * v + 2]), __uint_as_float(acc[4 * v + 3]));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) release_acc(buf);
+        ++local;
+        continue;
+      }
 
       if (u.slot >= 0) {
         // ---- stream-K piece: FP32 partial sums of kb0..kb1 into the tile's
@@ -1124,10 +1171,63 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++local;
     }
     }  // (kPromo)
+    if constexpr (LAYOUT == kDenseSplit) {
+      // ---- the slices of this CTA's tile lie in the shared memory of the
+      // cluster's CTAs (slice r in CTA r).  Once every CTA has written its
+      // own, CTA r sums rows [r kBM / S, (r + 1) kBM / S) of the tile over the
+      // slices in slice (= K) order, adds C and writes D; the second cluster
+      // barrier keeps every CTA's slice alive until the others have read it.
+      cluster_sync_all();
+      const int splits = a.split;
+      const uint32_t rank = cluster_ctarank();
+      int mb, nb;
+      raster_tile_fast((int)blockIdx.x / splits, a, mb, nb);
+      const int band = kBM / splits;
+      constexpr int kQ = BN / 4;  // float4 columns of a tile row
+      const float* part = reinterpret_cast<const float*>(smem);
+      for (int it = (int)threadIdx.x - 64; it < band * kQ; it += 32 * kEpiWarps) {
+        const int lr = (int)rank * band + it / kQ;
+        const int c4 = it % kQ;
+        const int row = mb * kBM + lr, col = nb * BN + 4 * c4;
+        if (row >= a.rows || col >= a.n) continue;
+        uint2 cw = make_uint2(0u, 0u);
+        if (a.c != nullptr) cw = __ldg(reinterpret_cast<const uint2*>(a.c + (long long)row * a.n + col));
+        const float* src = part + lr * kSplitPitch + 4 * c4;
+        float4 v[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+          if (r < splits) v[r] = ld_shared_cluster_f4(mapa_shared(src, (uint32_t)r));
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+          if (r < splits) {
+            acc.x += v[r].x;
+            acc.y += v[r].y;
+            acc.z += v[r].z;
+            acc.w += v[r].w;
+          }
+        __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x + __uint_as_float(cw.x << 16),
+                                                  acc.y + __uint_as_float(cw.x & 0xFFFF0000u));
+        __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z + __uint_as_float(cw.y << 16),
+                                                  acc.w + __uint_as_float(cw.y & 0xFFFF0000u));
+        *reinterpret_cast<uint2*>(a.d + (long long)row * a.n + col) =
+            make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+      }
+      cluster_sync_all();
+    }
     if (lane == 0) bulk_wait_group_all();
     __syncwarp();
   }
 
+  if constexpr (LAYOUT == kDenseSplit) {
+    // the producer and MMA warps take part in the epilogue's two cluster
+    // barriers (every thread of the cluster arrives at each)
+    if (warp < 2) {
+      __syncwarp();
+      cluster_sync_all();
+      cluster_sync_all();
+    }
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

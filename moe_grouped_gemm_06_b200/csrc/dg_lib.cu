@@ -8,6 +8,7 @@
 #include <cstring>
 #include <map>
 #include <mutex>
+#include <tuple>
 #include <utility>
 
 #include "../../include/dg.h"
@@ -124,6 +125,7 @@ struct Plan {
   int max_seg = 0;        // workspace slots per stream-K tile
   int sk_split = 0;       // > 0: each stream-K tile cut into this many K-slices
   long long sk_iters = 0;
+  int split = 0;          // > 0: every tile cut into this many K-slices on a cluster of as many CTAs
   int grid = 0;
   double cost = 0;        // estimated microseconds
   size_t ws_bytes() const { return (size_t)sk_tiles * max_seg * dg::kBM * bn * sizeof(float); }
@@ -160,14 +162,15 @@ constexpr WidthCost kWidthCosts[] = {
 
 // Tile-configuration override (dg_set_tile_config; initial values from the
 // environment variables DG_BLOCK_N and DG_SCHEDULE): one block width, and/or
-// one schedule: whole tiles (1), tail cut into per-tile K-slices (2) or
-// stream-K tail (3).
+// one schedule: whole tiles (1), tail cut into per-tile K-slices (2),
+// stream-K tail (3), or every tile split over a cluster of 2, 4 or 8 CTAs
+// (4, 5, 6).
 int env_int(const char* name) {
   const char* e = std::getenv(name);
   return e ? std::atoi(e) : 0;
 }
 std::atomic<int> g_force_bn{env_int("DG_BLOCK_N")};
-std::atomic<int> g_force_schedule{(env_int("DG_SCHEDULE") >= 1 && env_int("DG_SCHEDULE") <= 3) ? env_int("DG_SCHEDULE")
+std::atomic<int> g_force_schedule{(env_int("DG_SCHEDULE") >= 1 && env_int("DG_SCHEDULE") <= 6) ? env_int("DG_SCHEDULE")
                                                                                              : 0};
 
 int forced_block_n() {
@@ -214,9 +217,12 @@ int sk_max_segments(int sk_tiles, int kb, int G) {
 // (allow_sk) and only within ws_cap bytes of workspace (0: no cap).  Ties
 // keep whole tiles.
 // MN-major B (mn_b) is staged in 128-wide column blocks: widths 128 and 256.
+int split_capacity(int bn, bool fp4, int cluster);
+
 // only_bn: plan this block width alone (the promotion kernels are 128 wide).
+// allow_split: the dense NT kernels may cut every tile over a cluster (below).
 Plan plan_gemm(long long m_blocks, int n, int k, int sms, bool allow_sk, size_t ws_cap = 0, bool fp4 = false,
-               bool bf16 = false, bool mn_b = false, int only_bn = 0) {
+               bool bf16 = false, bool mn_b = false, int only_bn = 0, bool allow_split = false) {
   Plan best;
   best.cost = 1e300;
   const int kb = k / 128;
@@ -254,7 +260,28 @@ Plan plan_gemm(long long m_blocks, int n, int k, int sms, bool allow_sk, size_t 
     auto floored = [&](double t) { return std::max(t, hbm_floor) + 0.05 * t; };
     dp.cost = floored(std::max((double)waves * tile_time(wc, kb), waves * stream_b(kb))) * (sched >= 2 ? 1e6 : 1.0);
     consider(dp);
-    if (!allow_sk || sched == 1) continue;
+    // (c) every tile's K-blocks cut into S slices computed by the S CTAs of a
+    // cluster, their sums added through distributed shared memory: no
+    // workspace and no fix-up kernel, for problems with few tiles.  The cost
+    // of the sum is the DSMEM reads of one band (kBM / S rows of S slices).
+    if (allow_split && (bn == 128 || bn == 256) && (sched == 0 || sched >= 4)) {
+      for (int sp : {2, 4, 8}) {
+        if ((sched >= 4 && sp != (1 << (sched - 3))) || kb < sp) continue;
+        const int cap = split_capacity(bn, fp4, sp);  // clusters the GPU holds at once
+        if (cap <= 0) continue;
+        const long long kbs = ceil_div(kb, sp);
+        const double piece = std::max(kbs * wc.per_kb + wc.per_tile, stream_b(kbs));
+        const double reduce = 0.8 + 512.0 * bn / 1.2e5;
+        Plan pc;
+        pc.bn = bn;
+        pc.dp_tiles = tiles;
+        pc.split = sp;
+        pc.grid = (int)(tiles * sp);
+        pc.cost = floored((double)ceil_div(tiles, cap) * (piece + reduce));
+        consider(pc);
+      }
+    }
+    if (!allow_sk || sched == 1 || sched >= 4) continue;
     const long long full_waves = tiles / sms;
     for (long long q = full_waves; q >= std::max(0LL, full_waves - 1); --q) {
       const long long sk = tiles - q * sms;
@@ -333,8 +360,8 @@ float* workspace(size_t bytes, cudaStream_t s) {
 
 template <int BN, bool FP4, int LAYOUT, int EPI = dg::kEpiPlain, bool BF16 = false, int MAJ = dg::kMajorK>
 dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& ta32, const CUtensorMap& tb, const CUtensorMap& td,
-                      const dg::GemmArgs& args, int grid, cudaStream_t s) {
-  using C = dg::Cfg<BN, FP4, BF16, (LAYOUT == dg::kMasked || LAYOUT == dg::kKGrouped)>;
+                      const dg::GemmArgs& args, int grid, cudaStream_t s, int cluster = 1) {
+  using C = dg::Cfg<BN, FP4, BF16, (LAYOUT == dg::kMasked || LAYOUT == dg::kKGrouped), EPI == dg::kEpiPromote>;
   auto kern = dg::gemm_kernel<BN, FP4, LAYOUT, EPI, BF16, MAJ>;
   static std::atomic<uint64_t> attr_set_mask{0};  // one bit per device
   int dev = 0;
@@ -345,11 +372,64 @@ dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& ta32, const CUte
       return DG_ERR_CUDA;
     attr_set_mask.fetch_or(bit);
   }
-  if (launch(kern, dim3(grid), dim3(dg::kThreads), C::kSmemBytes, s, 1, ta, ta32, tb, td, args) !=
+  if (launch(kern, dim3(grid), dim3(dg::kThreads), C::kSmemBytes, s, cluster, ta, ta32, tb, td, args) !=
       cudaSuccess)
     return DG_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return DG_OK;
+}
+
+// Clusters of `cluster` CTAs of the split kernel (block width bn) that the
+// current device can hold at once (cudaOccupancyMaxActiveClusters), cached
+// per device; 0 when the query fails.
+template <int BN, bool FP4>
+int split_capacity_of(int cluster) {
+  using C = dg::Cfg<BN, FP4, false, false>;
+  auto kern = dg::gemm_kernel<BN, FP4, dg::kDenseSplit>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cluster);
+  cfg.blockDim = dim3(dg::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = cluster;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+int split_capacity(int bn, bool fp4, int cluster) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int, int>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  const auto key = std::make_tuple(dev, bn, (int)fp4, cluster);
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  int n = 0;
+  if (bn == 128) n = fp4 ? split_capacity_of<128, true>(cluster) : split_capacity_of<128, false>(cluster);
+  if (bn == 256) n = fp4 ? split_capacity_of<256, true>(cluster) : split_capacity_of<256, false>(cluster);
+  cache[key] = n;
+  return n;
+}
+
+template <bool FP4>
+dg_status dispatch_split(int bn, int split, const CUtensorMap& ta, const CUtensorMap& ta32, const CUtensorMap& tb,
+                         const CUtensorMap& td, const dg::GemmArgs& args, int grid, cudaStream_t s) {
+  switch (bn) {
+    case 128: return launch_gemm<128, FP4, dg::kDenseSplit>(ta, ta32, tb, td, args, grid, s, split);
+    case 256: return launch_gemm<256, FP4, dg::kDenseSplit>(ta, ta32, tb, td, args, grid, s, split);
+    default: return DG_ERR_UNSUPPORTED;
+  }
 }
 
 template <bool FP4, int LAYOUT, int EPI = dg::kEpiPlain, bool BF16 = false, int MAJ = dg::kMajorK>
@@ -442,7 +522,8 @@ Plan select_plan(const Problem& p, int layout, bool fp4, bool bf16, bool mn, boo
     plan = plan_gemm((long long)p.groups * m_blocks, p.n, k_plan_mn(p), sms, false, 0, false, false, true);
   } else {
     // MN-major operands run in 128- and 256-wide tiles only
-    plan = plan_gemm(m_blocks, p.n, k_plan, sms, layout == dg::kDense, ws_cap, fp4, bf16, mn, promote ? 128 : 0);
+    plan = plan_gemm(m_blocks, p.n, k_plan, sms, layout == dg::kDense, ws_cap, fp4, bf16, mn, promote ? 128 : 0,
+                     layout == dg::kDense && !promote && !bf16 && !mn);
   }
   return plan;
 }
@@ -560,11 +641,18 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
   if (log_enabled())
     std::fprintf(stderr,
                  "[dg] layout=%d fp4=%d rows=%d n=%d k=%d groups=%d -> block_n=%d dp_tiles=%lld sk_tiles=%d "
-                 "split=%d max_seg=%d grid=%d est=%.1fus\n",
+                 "split=%d max_seg=%d cluster_split=%d grid=%d est=%.1fus\n",
                  LAYOUT, (int)FP4, p.rows, p.n, p.k, p.groups, plan.bn, plan.dp_tiles, plan.sk_tiles, plan.sk_split,
-                 plan.max_seg, plan.grid, plan.cost);
+                 plan.max_seg, plan.split, plan.grid, plan.cost);
 
-  dg_status st = dispatch<FP4, LAYOUT, EPI, BF16, MAJ>(plan.bn, ta, ta32, tb, td, args, plan.grid, s);
+  dg_status st;
+  if constexpr (LAYOUT == dg::kDense && EPI == dg::kEpiPlain && !BF16 && MAJ == dg::kMajorK) {
+    if (plan.split > 0) {
+      args.split = plan.split;
+      return dispatch_split<FP4>(plan.bn, plan.split, ta, ta32, tb, td, args, plan.grid, s);
+    }
+  }
+  st = dispatch<FP4, LAYOUT, EPI, BF16, MAJ>(plan.bn, ta, ta32, tb, td, args, plan.grid, s);
   if (st != DG_OK || plan.sk_tiles == 0) return st;
 
   dg::SkReduceArgs r{};
@@ -944,7 +1032,7 @@ dg_status dg_set_tile_config(int block_n, int schedule) {
     for (const WidthCost& wc : kWidthCosts) known = known || (wc.bn == block_n);
     if (!known) return DG_ERR_INVALID_ARG;
   }
-  if (schedule < 0 || schedule > 3) return DG_ERR_INVALID_ARG;
+  if (schedule < 0 || schedule > 6) return DG_ERR_INVALID_ARG;
   g_force_bn.store(block_n);
   g_force_schedule.store(schedule);
   return DG_OK;
@@ -989,7 +1077,7 @@ dg_status dg_query_dense_config(int m, int n, int k, int64_t workspace_cap, int*
   if (m <= 0 || n <= 0 || k <= 0 || k % 128 != 0 || workspace_cap < 0) return DG_ERR_INVALID_ARG;
   const int sms = num_sms();
   if (sms <= 0) return DG_ERR_CUDA;
-  Plan p = plan_gemm(ceil_div(m, dg::kBM), n, k, sms, true, (size_t)workspace_cap);
+  Plan p = plan_gemm(ceil_div(m, dg::kBM), n, k, sms, true, (size_t)workspace_cap, false, false, false, 0, true);
   if (block_n) *block_n = p.bn;
   if (dp_tiles) *dp_tiles = (int)p.dp_tiles;
   if (sk_tiles) *sk_tiles = p.sk_tiles;
@@ -998,6 +1086,13 @@ dg_status dg_query_dense_config(int m, int n, int k, int64_t workspace_cap, int*
   if (grid) *grid = p.grid;
   if (workspace_bytes) *workspace_bytes = (int64_t)p.ws_bytes();
   return DG_OK;
+}
+
+int dg_query_dense_cluster_split(int m, int n, int k, int64_t workspace_cap) {
+  if (m <= 0 || n <= 0 || k <= 0 || k % 128 != 0 || workspace_cap < 0) return -1;
+  const int sms = num_sms();
+  if (sms <= 0) return -1;
+  return plan_gemm(ceil_div(m, dg::kBM), n, k, sms, true, (size_t)workspace_cap, false, false, false, 0, true).split;
 }
 
 dg_status dg_query_config(int layout, int fp4, int swiglu, int rows, int n, int k, int num_groups, int expected_m,

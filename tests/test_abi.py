@@ -225,7 +225,8 @@ def test_workspace_cap_limits_the_plan(dg):
 
 def test_tile_config_override(dg):
     assert dg.lib().dg_set_tile_config(96, 0) == -1          # not an instantiated width
-    assert dg.lib().dg_set_tile_config(0, 4) == -1           # no such schedule
+    assert dg.lib().dg_set_tile_config(0, 7) == -1           # no such schedule
+    assert dg.lib().dg_set_tile_config(0, -1) == -1
     dg.dg_set_num_sms(148)
     try:
         dg.dg_set_tile_config(256, 1)
@@ -239,6 +240,12 @@ def test_tile_config_override(dg):
     finally:
         dg.dg_set_tile_config(0, 0)
         dg.dg_set_num_sms(0)
+
+
+def test_cluster_split_query_rejects_bad_sizes(dg):
+    assert dg.dg_query_dense_cluster_split(0, 128, 128) == -1
+    assert dg.dg_query_dense_cluster_split(64, 128, 100) == -1
+    assert dg.dg_query_dense_cluster_split(64, 128, 128, -1) == -1
 
 
 def test_fast_division_matches_integer_division(dg):

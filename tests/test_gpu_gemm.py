@@ -151,6 +151,32 @@ def test_dense_shared_tail_is_deterministic_and_agrees_with_whole_tiles(dg):
         check_close(outs[sched][0], p.ref(), f"schedule {sched} vs oracle")
 
 
+@pytest.mark.parametrize("schedule,S", [(4, 2), (5, 4), (6, 8)])
+@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("M,N,K,with_c,fp4", [
+    (64, 2112, 7168, True, False),     # small M: the shape these plans are for
+    (200, 328, 1024, True, False),     # two m-blocks, ragged M and N tails
+    (1, 136, 2048, False, False),      # a single row, no C
+    (128, 904, 1024, True, True),      # FP8 x FP4
+])
+def test_dense_cluster_split_matches_oracle(dg, schedule, S, bn, M, N, K, with_c, fp4):
+    # every tile's K-blocks cut into S slices on a cluster of S CTAs, summed
+    # through distributed shared memory in slice order
+    dg.dg_set_tile_config(bn, schedule)
+    try:
+        if dg.dg_query_dense_cluster_split(M, N, K) != S:
+            pytest.skip(f"no {S}-way split for this shape")
+        cfg = dg.dg_query_dense_config(M, N, K)
+        assert cfg["block_n"] == bn and cfg["sk_tiles"] == 0 and cfg["workspace_bytes"] == 0
+        p = Dense(2650 + M + bn + S, M, N, K, with_c=with_c, fp4=fp4).upload()
+        d1 = p.run(dg)
+        d2 = p.run(dg)
+    finally:
+        dg.dg_set_tile_config(0, 0)
+    assert np.array_equal(d1, d2)          # fixed summation order
+    check_close(d1, p.ref(), f"split S={S} bn={bn} {M}x{N}x{K} fp4={fp4}")
+
+
 @pytest.mark.parametrize("bn", [64, 160, 224])
 @pytest.mark.parametrize("M,N,K,fp4", [(300, 1000, 1024, False), (1100, 2112, 512, False), (200, 904, 512, True)])
 def test_dense_forced_widths(dg, bn, M, N, K, fp4):
