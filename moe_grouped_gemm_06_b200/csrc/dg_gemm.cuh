@@ -122,6 +122,7 @@ struct GemmArgs {
   int dp_tiles, sk_tiles, max_seg, sk_split;
   long long sk_iters;
   int split;                           // kDenseSplit: CTAs (K-slices) per tile = cluster size
+  int a_trim;                          // some tiles have fewer than kBM valid rows of A (M tail, masked)
   int sfa_chunks, sfb_chunks;          // ceil(rows/128), ceil(n/128)
   long long sfa_group_words, sfb_group_words;
   int sfa_q, sfb_q;                    // packed groups along K
@@ -140,10 +141,16 @@ struct GemmArgs {
 // bytes to the stage ring.
 // PROMO = true (kEpiPromote): no scale words are staged (the epilogue reads
 // them from global memory) and TMEM holds only per-K-block partial sums.
-template <int BN, bool FP4, bool BF16 = false, bool PREFIX = true, bool PROMO = false>
+// OVL = true (256-wide tiles, plain epilogue): two accumulators that share 64
+// columns, at columns 0 and 192, instead of a single one: 512 TMEM columns
+// hold two whole 256-column accumulators only without the scale factors, so
+// the second one overlaps the first and the next tile's MMAs wait only until
+// the epilogue has drained the shared columns (it drains them first).
+template <int BN, bool FP4, bool BF16 = false, bool PREFIX = true, bool PROMO = false, bool OVL = false>
 struct Cfg {
   static_assert(!(BF16 && FP4), "bf16 A and B");
   static_assert(!PROMO || (!FP4 && !BF16 && BN == 128), "promotion: e4m3 A and B, 128-wide tiles");
+  static_assert(!OVL || (BN == 256 && !PROMO), "overlapping accumulators: 256-wide tiles");
   static constexpr int kKPerStage = BF16 ? 64 : kBK;  // K-elements per stage
   // The scale-factor operand of the MMA is addressed in TMEM columns of 32
   // rows (a 128-row chunk spans 4 columns), and that address must be even: a
@@ -160,7 +167,7 @@ struct Cfg {
   // FP32 accumulator buffers in TMEM: three of 128 columns (BN = 128), two at
   // columns 0 and 256 (BN = 192), one (BN = 256); scale factors after them.
   // Promotion: four 128-column buffers of K-block partial sums, no scales.
-  static constexpr int kAccBufs = PROMO ? 4 : ((BN <= 128) ? 3 : (BN <= 240 ? 2 : 1));
+  static constexpr int kAccBufs = PROMO ? 4 : (OVL ? 2 : ((BN <= 128) ? 3 : (BN <= 240 ? 2 : 1)));
   static constexpr int kABytes = kBM * kBK;                  // 16 KB
   static constexpr int kBBytes = BN * kBK;                   // smem bytes (FP4 lands padded to 1 B/elt)
   static constexpr int kBTxBytes = FP4 ? kBBytes / 2 : kBBytes;  // bytes the TMA copy reports (packed)
@@ -176,7 +183,7 @@ struct Cfg {
   static_assert(kStages >= 2, "stages");
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kEpiBytes + kMaskBytes + kBarBytes;
   static constexpr uint32_t kColAcc = 0;
-  static constexpr uint32_t kAccStride = (BN <= 128) ? 128 : 256;
+  static constexpr uint32_t kAccStride = OVL ? 192 : ((BN <= 128) ? 128 : 256);
   static constexpr uint32_t kColSfa = (kAccBufs - 1) * kAccStride + BN;  // even, 4-column aligned
   static constexpr uint32_t kColSfb = kColSfa + 4;
   static_assert(PROMO ? kAccBufs * kAccStride <= kTmemCols : kColSfb + 4 * kSfbChunks <= kTmemCols, "TMEM columns");
@@ -350,7 +357,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const GemmArgs args) {
   static_assert(EPI == kEpiPlain || BN % (2 * kSwiGluBlock) == 0, "SwiGLU tiles hold whole block pairs");
   constexpr bool kPromo = (EPI == kEpiPromote);
-  using C = Cfg<BN, FP4, BF16, (LAYOUT == kMasked || LAYOUT == kKGrouped), kPromo>;
+  constexpr bool kOvl = (BN == 256 && EPI == kEpiPlain);
+  using C = Cfg<BN, FP4, BF16, (LAYOUT == kMasked || LAYOUT == kKGrouped), kPromo, kOvl>;
   static_assert(!BF16 || EPI == kEpiPlain, "bf16: plain epilogue");
   static_assert(!kPromo || (LAYOUT == kDense && MAJ == kMajorK), "promotion: dense NT");
   constexpr bool kAMn = (MAJ & kAMajorMN) != 0;
@@ -381,8 +389,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = bars + S;
   uint64_t* tfull = bars + 2 * S;       // [4]: accumulator buffer b holds a result
   uint64_t* tempty = bars + 2 * S + 4;  // [4]: the epilogue has read buffer b
-  uint64_t* drain = bars + 2 * S + 8;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 * S + 9);
+  uint64_t* tovl = bars + 2 * S + 8;    // [2]: the epilogue has read the columns buffer b shares (kOvl)
+  uint64_t* drain = bars + 2 * S + 10;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 * S + 11);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
 
   const int warp = threadIdx.x / 32;
@@ -399,6 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], kEpiWarps);
     }
+    for (int b = 0; b < 2; ++b) mbar_init(&tovl[b], kEpiWarps / 2);  // the warps of one column half
     mbar_init(drain, 1);
     *s_abort = 0;
     fence_mbar_init();
@@ -507,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // them; the MMA's remaining rows read stale shared memory and feed
         // accumulator rows that are never stored
         int a_boxes = 4;
-        if constexpr (!kAMn) {
+        if (!kAMn && a.a_trim) {
           int lim = a.rows;
           if (LAYOUT == kMasked) lim = min(max(__ldg(a.masked_m + u.g), 0), a.rows);
           a_boxes = max(1, min(4, (lim - a_row + 31) / 32));
@@ -648,6 +658,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int buf = local % C::kAccBufs;
         const uint32_t use = (uint32_t)(local / C::kAccBufs);
         if (!dg_wait(&tempty[buf], (use & 1) ^ 1, s_abort, limit)) {
+          ok = false;
+          break;
+        }
+        // overlapping accumulators: the previous tile's epilogue must also have
+        // read the 64 columns its buffer shares with this one
+        if (kOvl && local > 0 && !dg_wait(&tovl[(local - 1) & 1], (uint32_t)((local - 1) >> 1) & 1u, s_abort, limit)) {
           ok = false;
           break;
         }
@@ -1058,7 +1074,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) release_acc(buf);
+        if (lane == 0) {
+          if (kOvl && half == (buf == 0 ? 1 : 0)) mbar_arrive(&tovl[buf]);
+          release_acc(buf);
+        }
         ++local;
         continue;
       }
@@ -1091,7 +1110,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) release_acc(buf);
+        if (lane == 0) {
+          if (kOvl && half == (buf == 0 ? 1 : 0)) mbar_arrive(&tovl[buf]);
+          release_acc(buf);
+        }
         ++local;
         continue;
       }
@@ -1129,8 +1151,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
-#pragma unroll
-        for (int j = 0; j < kChunks; ++j) {
+        // one 32-column chunk j of this warp's columns: TMEM -> +C -> bf16 -> D
+        auto plain_chunk = [&](int j) {
           const int col0 = colw + j * kEpiCols;
           if (j < nch_w && vr > 0 && col0 < a.n) {
             uint32_t acc[kEpiCols];
@@ -1162,6 +1184,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             store_chunk(col0, packed);
           }
+        };
+        if constexpr (kOvl) {
+          // the 64 columns this buffer shares with the other one are drained
+          // first and reported (tovl), so the next tile's MMAs can start:
+          // buffer 0 shares tile columns 192..255 (chunks 2, 3 of column
+          // half 1), buffer 1 tile columns 0..63 (chunks 0, 1 of half 0)
+          static_assert(kChunks == 4, "256-wide tiles: four chunks per warp");
+          const bool owner = (half == (buf == 0 ? 1 : 0));
+          auto shared_drained = [&]() {
+            if (empty_k) return;  // (a tile of an empty group took no accumulator)
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tovl[buf]);
+          };
+          if (owner && buf == 0) {
+            plain_chunk(2);
+            plain_chunk(3);
+            shared_drained();
+            plain_chunk(0);
+            plain_chunk(1);
+          } else {
+            plain_chunk(0);
+            plain_chunk(1);
+            if (owner) shared_drained();
+            plain_chunk(2);
+            plain_chunk(3);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < kChunks; ++j) plain_chunk(j);
         }
       }  // plain epilogue
       if (empty_k) continue;  // (no accumulator taken)

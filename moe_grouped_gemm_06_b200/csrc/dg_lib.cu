@@ -139,7 +139,8 @@ long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
 //   tile = max(K-blocks x per_kb + per_tile, epilogue)
 // With two or three accumulator buffers the epilogue of one tile overlaps the
 // main loop of the next, so a tile costs the slower of the two; at 256
-// columns there is one buffer and the epilogue is inside per_tile.  Widths 160
+// columns the two buffers share 64 columns, so a tile's MMAs wait for the
+// first quarter of the previous tile's epilogue (inside per_tile).  Widths 160
 // and 224 re-base their scale words on the MMA-issuing thread, which costs
 // more than they gain; they are available through dg_set_tile_config but
 // never chosen automatically.
@@ -157,7 +158,7 @@ struct WidthCost {
 constexpr WidthCost kWidthCosts[] = {
     {64, 0.19, 1.5, 1.6, true, 0.21, 0.13},      {128, 0.2305, 1.9, 2.94, true, 0.264, 0.213},
     {160, 0.32, 2.4, 3.6, false, 0.33, 0.26},    {192, 0.368, 1.6, 3.97, true, 0.345, 0.284},
-    {224, 0.41, 3.0, 4.6, false, 0.36, 0.33},    {256, 0.4236, 4.34, 0.0, true, 0.343, 0.357},
+    {224, 0.41, 3.0, 4.6, false, 0.36, 0.33},    {256, 0.4236, 2.6, 2.5, true, 0.343, 0.357},
 };
 
 // Tile-configuration override (dg_set_tile_config; initial values from the
@@ -579,6 +580,9 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
   args.sfb_q = FP4 ? p.k / 128 : args.sfa_q;
   args.sfa_group_words = (long long)args.sfa_q * args.sfa_chunks * 128;
   args.sfb_group_words = (long long)args.sfb_q * args.sfb_chunks * 128;
+  // tiles with fewer than 128 valid rows of A exist only for an M tail or in
+  // the masked layout; elsewhere the producer skips the trimming arithmetic
+  args.a_trim = (!kAMn && (LAYOUT == dg::kMasked || p.rows % dg::kBM != 0)) ? 1 : 0;
   args.raster = 8;
   args.band_div.init((uint32_t)(args.raster * args.num_n_blocks));
   args.group_div.init((uint32_t)(args.num_m_blocks * args.num_n_blocks));
