@@ -16,7 +16,13 @@ host to launch it.
             host->device copies of A, SFA, B, SFB, C and the device->host copy
             of D inside the timed region
   roofline: the dominant kernel (largest share of step time) against the
-            measured peak (MEASURED_PEAKS.json), FP8 peak = measured bf16 x 2
+            measured peak (MEASURED_PEAKS.json), FP8 peak = measured bf16 x 2;
+            beside it frac_vs_probe (the library's own block-scaled FP8
+            tcgen05 loop, measured in the same run: tensor_peak_probe) and
+            frac_vs_spec (nominal dense FP8, 4.5 PFLOP/s)
+  per_config: the other configurations timed the same way after the sweep:
+            the small dense case, MoE prefill (contiguous), MoE decode
+            (masked) and FP8 x FP4 (dense and contiguous)
   cpu_baseline: the CPU oracle on a bounded sample of the same sweep
 
 Multi-GPU: the sweep does not shard (replicas only); with --gpus N each rank
@@ -24,14 +30,16 @@ runs the full sweep on its own GPU and value aggregates all ranks ("weak").
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                   [--shape M,N,K] [--no-e2e] [--no-cpu]
+                  [--no-configs]
                   [--workload dense | contiguous | nn_contiguous | kgrouped_tn | masked
-                              | fp4 | moe_decode_fp4 | bf16] [--graph]
+                              | fp4 | moe_decode_fp4 | bf16 | promotion] [--graph]
 
 The default workload (dense) is the headline line.  The others time each case
 alone after an L2 flush and report per-case TFLOPS and roofline fractions:
 MoE prefill (contiguous, NT and NN), the MoE weight gradient (K-grouped TN),
 decode (masked, plain or as a CUDA graph with --graph), FP8 x FP4, the FP8 x
-FP4 decode step with SwiGLU, and BF16 against cuBLAS.
+FP4 decode step with SwiGLU, BF16 against cuBLAS, and the two ways of
+applying the scales (block-scaled MMA vs per-K-block promotion).
 """
 from __future__ import annotations
 

@@ -200,6 +200,11 @@ struct Cfg {
   static constexpr uint32_t kIdesc = BF16 ? kIdescBf16 : (PROMO ? kIdescPlain : kIdescScaled);
 };
 
+template <bool B>
+struct BoolC {
+  static constexpr bool value = B;
+};
+
 struct Unit {
   int g, mb, nb;
   int kb0, kb1;   // K-blocks of this unit
@@ -525,62 +530,72 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t a_bytes = (a_boxes == 4) ? (uint32_t)C::kABytes : (uint32_t)a_boxes * (32 * 128);
         const int32_t* sfa_g = a.sfa + (LAYOUT == kMasked ? (long long)u.g * a.sfa_group_words : 0);
         const int32_t* sfb_g = a.sfb + (long long)b_grp * a.sfb_group_words;
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!dg_wait(&empty[stage], phase ^ 1, s_abort, limit)) {
-            ok = false;
-            break;
+        // the K-loop in two versions, so that the untrimmed one (every full
+        // tile) carries no per-K-block branch on the box count
+        auto k_loop = [&](auto trim_c) {
+          constexpr bool kTrim = decltype(trim_c)::value;
+          for (int kb = kb0; kb < kb1; ++kb) {
+            if (!dg_wait(&empty[stage], phase ^ 1, s_abort, limit)) {
+              ok = false;
+              break;
+            }
+            const bool new_sfa = !BF16 && !kPromo && (((kb & 3) == 0) || kb == kb0);
+            const bool new_sfb = !BF16 && !kPromo && (FP4 || new_sfa);
+            uint32_t bytes = (kTrim ? a_bytes : (uint32_t)C::kABytes) +
+                             (kBMn ? (uint32_t)b_blocks * (kBK * 128) : (uint32_t)C::kBTxBytes);
+            if (new_sfa) bytes += C::kSfaBytes;
+            if (new_sfb) bytes += 512u * nchunks;
+            DG_CHECK(((smem_u32(s_a + stage * C::kABytes) | smem_u32(s_b + stage * C::kBBytes)) & 1023) == 0 &&
+                         u.mb < a.num_m_blocks && u.nb < a.num_n_blocks && kb < a.kb_total,
+                     6);
+            mbar_arrive_expect_tx(&full[stage], bytes);
+            if constexpr (kAMn) {
+              tma_load_3d(s_a + stage * C::kABytes, &tm_a, &full[stage], a_row, kb * kBK, a_grp);
+            } else if constexpr (!kTrim) {
+              tma_load_3d(s_a + stage * C::kABytes, &tm_a, &full[stage], kb * C::kKPerStage, a_row, a_grp);
+            } else {
+              // 32-row boxes land 4 KB apart, at 1024-byte-aligned addresses,
+              // so the 128-byte swizzle places their rows where one 128-row
+              // box would
+              for (int i = 0; i < a_boxes; ++i)
+                tma_load_3d(s_a + stage * C::kABytes + i * (32 * 128), &tm_a32, &full[stage], kb * C::kKPerStage,
+                            a_row + 32 * i, a_grp);
+            }
+            if constexpr (kBMn) {
+              for (int cb = 0; cb < b_blocks; ++cb)
+                tma_load_3d(s_b + stage * C::kBBytes + cb * (kBK * 128), &tm_b, &full[stage], n0 + 128 * cb, kb * kBK,
+                            b_grp);
+            } else {
+              tma_load_3d(s_b + stage * C::kBBytes, &tm_b, &full[stage], kb * C::kKPerStage, n0, b_grp);
+            }
+            if (new_sfa) {
+              const int32_t* src = sfa_g + ((long long)(kb >> 2) * a.sfa_chunks + u.mb) * 128;
+              if (DG_CHECK(src >= a.sfa && src + 128 <= a.sfa + a.sfa_words &&
+                               ((reinterpret_cast<uintptr_t>(src) | smem_u32(s_sfa + stage * C::kSfaBytes)) & 15) == 0,
+                           4))
+                bulk_load(s_sfa + stage * C::kSfaBytes, src, C::kSfaBytes, &full[stage]);
+            }
+            if (new_sfb) {
+              const int q = FP4 ? kb : (kb >> 2);
+              const int32_t* src = sfb_g + ((long long)q * a.sfb_chunks + c0) * 128;
+              if (DG_CHECK(src >= a.sfb && src + 128 * nchunks <= a.sfb + a.sfb_words && nchunks >= 1 &&
+                               nchunks <= C::kSfbChunks &&
+                               ((reinterpret_cast<uintptr_t>(src) | smem_u32(s_sfb + stage * C::kSfbBytes)) & 15) == 0,
+                           5))
+                bulk_load(s_sfb + stage * C::kSfbBytes, src, 512u * nchunks, &full[stage]);
+            }
+            filled_phase[stage] = phase;
+            filled_mask |= 1u << stage;
+            if (++stage == S) {
+              stage = 0;
+              phase ^= 1;
+            }
           }
-          const bool new_sfa = !BF16 && !kPromo && (((kb & 3) == 0) || kb == kb0);
-          const bool new_sfb = !BF16 && !kPromo && (FP4 || new_sfa);
-          uint32_t bytes = a_bytes + (kBMn ? (uint32_t)b_blocks * (kBK * 128) : (uint32_t)C::kBTxBytes);
-          if (new_sfa) bytes += C::kSfaBytes;
-          if (new_sfb) bytes += 512u * nchunks;
-          DG_CHECK(((smem_u32(s_a + stage * C::kABytes) | smem_u32(s_b + stage * C::kBBytes)) & 1023) == 0 &&
-                       u.mb < a.num_m_blocks && u.nb < a.num_n_blocks && kb < a.kb_total,
-                   6);
-          mbar_arrive_expect_tx(&full[stage], bytes);
-          if constexpr (kAMn) {
-            tma_load_3d(s_a + stage * C::kABytes, &tm_a, &full[stage], a_row, kb * kBK, a_grp);
-          } else if (a_boxes == 4) {
-            tma_load_3d(s_a + stage * C::kABytes, &tm_a, &full[stage], kb * C::kKPerStage, a_row, a_grp);
-          } else {
-            // 32-row boxes land 4 KB apart, at 1024-byte-aligned addresses,
-            // so the 128-byte swizzle places their rows where one 128-row
-            // box would
-            for (int i = 0; i < a_boxes; ++i)
-              tma_load_3d(s_a + stage * C::kABytes + i * (32 * 128), &tm_a32, &full[stage], kb * C::kKPerStage,
-                          a_row + 32 * i, a_grp);
-          }
-          if constexpr (kBMn) {
-            for (int cb = 0; cb < b_blocks; ++cb)
-              tma_load_3d(s_b + stage * C::kBBytes + cb * (kBK * 128), &tm_b, &full[stage], n0 + 128 * cb, kb * kBK,
-                          b_grp);
-          } else {
-            tma_load_3d(s_b + stage * C::kBBytes, &tm_b, &full[stage], kb * C::kKPerStage, n0, b_grp);
-          }
-          if (new_sfa) {
-            const int32_t* src = sfa_g + ((long long)(kb >> 2) * a.sfa_chunks + u.mb) * 128;
-            if (DG_CHECK(src >= a.sfa && src + 128 <= a.sfa + a.sfa_words &&
-                             ((reinterpret_cast<uintptr_t>(src) | smem_u32(s_sfa + stage * C::kSfaBytes)) & 15) == 0,
-                         4))
-              bulk_load(s_sfa + stage * C::kSfaBytes, src, C::kSfaBytes, &full[stage]);
-          }
-          if (new_sfb) {
-            const int q = FP4 ? kb : (kb >> 2);
-            const int32_t* src = sfb_g + ((long long)q * a.sfb_chunks + c0) * 128;
-            if (DG_CHECK(src >= a.sfb && src + 128 * nchunks <= a.sfb + a.sfb_words && nchunks >= 1 &&
-                             nchunks <= C::kSfbChunks &&
-                             ((reinterpret_cast<uintptr_t>(src) | smem_u32(s_sfb + stage * C::kSfbBytes)) & 15) == 0,
-                         5))
-              bulk_load(s_sfb + stage * C::kSfbBytes, src, 512u * nchunks, &full[stage]);
-          }
-          filled_phase[stage] = phase;
-          filled_mask |= 1u << stage;
-          if (++stage == S) {
-            stage = 0;
-            phase ^= 1;
-          }
-        }
+        };
+        if (a_boxes == 4)
+          k_loop(BoolC<false>{});
+        else
+          k_loop(BoolC<true>{});
       }
       if (!ok) {
         // never leave copies in flight into shared memory: wait (bounded) for
