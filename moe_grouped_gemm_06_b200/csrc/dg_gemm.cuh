@@ -1011,6 +1011,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int vr = min(32, limit_rows - r0);
       const int row = r0 + (int)lane;
       const long long grow = kGroupRows ? (long long)u.g * a.rows + row : row;
+      (void)grow;
       // k-grouped tile of an empty group: no accumulator, D = C (or 0)
       const bool empty_k = (LAYOUT == kKGrouped) && u.kb0 == u.kb1;
       const int colw = u.nb * BN + half * kCols;  // first column of this warp
