@@ -1119,15 +1119,21 @@ dg_status dg_query_config(int layout, int fp4, int swiglu, int rows, int n, int 
 }
 
 dg_status dg_probe_mma_peak(int kind, int block_n, int kblocks, void* stream) {
-  if (kind < DG_PROBE_FP8_SCALED || kind > DG_PROBE_BF16 || (block_n != 128 && block_n != 256) || kblocks <= 0 ||
-      kblocks > (1 << 22))
+  const bool narrow = (block_n == 32 || block_n == 64);
+  if (kind < DG_PROBE_FP8_SCALED || kind > DG_PROBE_BF16 || (block_n != 128 && block_n != 256 && !narrow) ||
+      (narrow && kind != DG_PROBE_FP8_SCALED) || kblocks <= 0 || kblocks > (1 << 22))
     return DG_ERR_INVALID_ARG;
   const int grid = device_sms();
   if (grid <= 0) return DG_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (kind == DG_PROBE_FP8_SCALED)
-    return block_n == 128 ? launch_probe<dg::kProbeScaled, 128>(kblocks, grid, s)
-                          : launch_probe<dg::kProbeScaled, 256>(kblocks, grid, s);
+  if (kind == DG_PROBE_FP8_SCALED) {
+    switch (block_n) {
+      case 32: return launch_probe<dg::kProbeScaled, 32>(kblocks, grid, s);
+      case 64: return launch_probe<dg::kProbeScaled, 64>(kblocks, grid, s);
+      case 128: return launch_probe<dg::kProbeScaled, 128>(kblocks, grid, s);
+      default: return launch_probe<dg::kProbeScaled, 256>(kblocks, grid, s);
+    }
+  }
   if (kind == DG_PROBE_FP8_PLAIN)
     return block_n == 128 ? launch_probe<dg::kProbePlain, 128>(kblocks, grid, s)
                           : launch_probe<dg::kProbePlain, 256>(kblocks, grid, s);
