@@ -350,9 +350,9 @@ int dg_get_pdl(void);
  * 256; the others are only used when forced) and schedule 0 (heuristic), 1
  * (whole tiles only), 2 (the last tiles cut into per-tile K-slices, one per
  * CTA) or 3 (stream-K: the last tiles' K-iterations shared evenly over the
- * grid), 4, 5 or 6 (every tile's K-blocks cut into 2, 4 or 8 slices
- * computed by the CTAs of one thread-block cluster and summed through
- * distributed shared memory; 128- and 256-wide dense NT tiles); 2 to 6 apply
+ * grid), or 4 to 10 (every tile's K-blocks cut into S = schedule - 2 slices,
+ * 2 to 8, computed by the CTAs of one thread-block cluster and summed through
+ * distributed shared memory; 128- and 256-wide dense NT tiles); 2 to 10 apply
  * to the dense calls whenever such a split exists.
  * Anything else returns DG_ERR_INVALID_ARG and changes nothing.  Meant for
  * tuning and tests.  The environment variables DG_BLOCK_N and DG_SCHEDULE set
@@ -403,6 +403,12 @@ dg_status dg_query_dense_config(int m, int n, int k, int64_t workspace_cap, int*
  * reports as dp_tiles = the tiles, sk_tiles = 0, grid = tiles x S); 0 when the
  * plan is another one; -1 for invalid sizes. */
 int dg_query_dense_cluster_split(int m, int n, int k, int64_t workspace_cap);
+
+/* Clusters of `cluster` CTAs (2 .. 8) of the split kernel with block width
+ * block_n (128 or 256; fp4 nonzero: e2m1 B) that the current device holds at
+ * once (cudaOccupancyMaxActiveClusters); the planner's capacity for cluster
+ * splits.  -1 for other arguments, 0 when the query fails. */
+int dg_debug_cluster_capacity(int block_n, int fp4, int cluster);
 
 /* Layouts named by dg_query_config. */
 enum { DG_LAYOUT_DENSE = 0, DG_LAYOUT_CONTIGUOUS = 1, DG_LAYOUT_MASKED = 2 };

@@ -25,7 +25,7 @@ __all__ = [
     "dg_fp8_gemm_tn", "dg_fp8_gemm_tt",
     "dg_quantize_fp8", "dg_quantize_fp4", "dg_pack_sf", "dg_packed_sf_words", "dg_get_num_sms",
     "dg_set_num_sms", "dg_set_pdl", "dg_get_pdl", "dg_set_tile_config", "dg_get_mk_alignment_for_contiguous_layout", "dg_get_last_error",
-    "dg_debug_starved_wait", "dg_launch_count", "dg_query_dense_config", "dg_query_dense_cluster_split", "dg_query_config", "dg_probe_mma_peak", "dg_num_tiles", "dg_debug_fastdiv", "dg_shutdown",
+    "dg_debug_starved_wait", "dg_launch_count", "dg_query_dense_config", "dg_query_dense_cluster_split", "dg_debug_cluster_capacity", "dg_query_config", "dg_probe_mma_peak", "dg_num_tiles", "dg_debug_fastdiv", "dg_shutdown",
     "SYMBOLS",
 ]
 
@@ -75,6 +75,7 @@ SYMBOLS = {
     "dg_launch_count": (ctypes.c_uint64, []),
     "dg_query_dense_config": (_INT, [_INT, _INT, _INT, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "dg_query_dense_cluster_split": (_INT, [_INT, _INT, _INT, _I64]),
+    "dg_debug_cluster_capacity": (_INT, [_INT, _INT, _INT]),
     "dg_query_config": (_INT, [_INT, _INT, _INT, _INT, _INT, _INT, _INT, _INT, _VP, _VP, _VP]),
     "dg_probe_mma_peak": (_INT, [_INT, _INT, _INT, _VP]),
     "dg_num_tiles": (_I64, [_INT, _INT, _INT, _INT]),
@@ -351,6 +352,11 @@ def dg_query_dense_config(m: int, n: int, k: int, workspace_cap: int = 0) -> dic
 def dg_query_dense_cluster_split(m: int, n: int, k: int, workspace_cap: int = 0) -> int:
     """S > 0 when the dense plan splits every tile over a cluster of S CTAs."""
     return int(lib().dg_query_dense_cluster_split(m, n, k, int(workspace_cap)))
+
+
+def dg_debug_cluster_capacity(block_n: int, cluster: int, fp4: bool = False) -> int:
+    """Clusters of `cluster` CTAs of the split kernel the device holds at once."""
+    return int(lib().dg_debug_cluster_capacity(block_n, int(fp4), cluster))
 
 
 LAYOUTS = {"dense": 0, "contiguous": 1, "masked": 2}

@@ -49,9 +49,9 @@ constexpr int kMaxMaskedGroups = 1024;
 // kKGrouped: the weight-gradient layout, grouped along K -- group g owns the
 // K rows [K_0 + ... + K_(g-1), ... + K_g) of A and B and its own D[g].
 // kDenseSplit: the dense layout with every tile's K-blocks cut into `split`
-// slices computed by the CTAs of one thread-block cluster, whose FP32 partial
-// sums are added through distributed shared memory (no workspace, no second
-// kernel); for problems with too few tiles to fill the SMs.
+// (2 to 8) slices computed by the CTAs of one thread-block cluster, whose FP32
+// partial sums are added through distributed shared memory (no workspace, no
+// second kernel); for problems with too few tiles to fill the SMs.
 enum : int { kDense = 0, kContig = 1, kMasked = 2, kKGrouped = 3, kDenseSplit = 4 };
 
 // Operand majorness (template parameter MAJ): which of A and B are stored
@@ -1242,19 +1242,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (LAYOUT == kDenseSplit) {
       // ---- the slices of this CTA's tile lie in the shared memory of the
       // cluster's CTAs (slice r in CTA r).  Once every CTA has written its
-      // own, CTA r sums rows [r kBM / S, (r + 1) kBM / S) of the tile over the
-      // slices in slice (= K) order, adds C and writes D; the second cluster
-      // barrier keeps every CTA's slice alive until the others have read it.
+      // own, CTA r sums rows [r kBM / S, (r + 1) kBM / S) of the tile (integer
+      // division: any S from 2 to 8) over the slices in slice (= K) order,
+      // adds C and writes D; the second cluster barrier keeps every CTA's
+      // slice alive until the others have read it.
       cluster_sync_all();
       const int splits = a.split;
       const uint32_t rank = cluster_ctarank();
       int mb, nb;
       raster_tile_fast((int)blockIdx.x / splits, a, mb, nb);
-      const int band = kBM / splits;
+      const int lr0 = (int)rank * kBM / splits;  // this CTA's rows [lr0, lr1) of the tile
+      const int band = ((int)rank + 1) * kBM / splits - lr0;
       constexpr int kQ = BN / 4;  // float4 columns of a tile row
       const float* part = reinterpret_cast<const float*>(smem);
       for (int it = (int)threadIdx.x - 64; it < band * kQ; it += 32 * kEpiWarps) {
-        const int lr = (int)rank * band + it / kQ;
+        const int lr = lr0 + it / kQ;
         const int c4 = it % kQ;
         const int row = mb * kBM + lr, col = nb * BN + 4 * c4;
         if (row >= a.rows || col >= a.n) continue;

@@ -166,15 +166,15 @@ constexpr WidthCost kWidthCosts[] = {
 // Tile-configuration override (dg_set_tile_config; initial values from the
 // environment variables DG_BLOCK_N and DG_SCHEDULE): one block width, and/or
 // one schedule: whole tiles (1), tail cut into per-tile K-slices (2),
-// stream-K tail (3), or every tile split over a cluster of 2, 4 or 8 CTAs
-// (4, 5, 6).
+// stream-K tail (3), or every tile split over a cluster of S = schedule - 2
+// CTAs (4 .. 10: S = 2 .. 8).
 int env_int(const char* name) {
   const char* e = std::getenv(name);
   return e ? std::atoi(e) : 0;
 }
 std::atomic<int> g_force_bn{env_int("DG_BLOCK_N")};
-std::atomic<int> g_force_schedule{(env_int("DG_SCHEDULE") >= 1 && env_int("DG_SCHEDULE") <= 6) ? env_int("DG_SCHEDULE")
-                                                                                             : 0};
+std::atomic<int> g_force_schedule{(env_int("DG_SCHEDULE") >= 1 && env_int("DG_SCHEDULE") <= 10) ? env_int("DG_SCHEDULE")
+                                                                                              : 0};
 
 int forced_block_n() {
   const int b = g_force_bn.load();
@@ -268,8 +268,8 @@ Plan plan_gemm(long long m_blocks, int n, int k, int sms, bool allow_sk, size_t 
     // workspace and no fix-up kernel, for problems with few tiles.  The cost
     // of the sum is the DSMEM reads of one band (kBM / S rows of S slices).
     if (allow_split && (bn == 128 || bn == 256) && (sched == 0 || sched >= 4)) {
-      for (int sp : {2, 4, 8}) {
-        if ((sched >= 4 && sp != (1 << (sched - 3))) || kb < sp) continue;
+      for (int sp = 2; sp <= 8; ++sp) {
+        if ((sched >= 4 && sp != sched - 2) || kb < sp) continue;
         const int cap = split_capacity(bn, fp4, sp);  // clusters the GPU holds at once
         if (cap <= 0) continue;
         const long long kbs = ceil_div(kb, sp);
@@ -1038,7 +1038,7 @@ dg_status dg_set_tile_config(int block_n, int schedule) {
     for (const WidthCost& wc : kWidthCosts) known = known || (wc.bn == block_n);
     if (!known) return DG_ERR_INVALID_ARG;
   }
-  if (schedule < 0 || schedule > 6) return DG_ERR_INVALID_ARG;
+  if (schedule < 0 || schedule > 10) return DG_ERR_INVALID_ARG;
   g_force_bn.store(block_n);
   g_force_schedule.store(schedule);
   return DG_OK;
@@ -1092,6 +1092,11 @@ dg_status dg_query_dense_config(int m, int n, int k, int64_t workspace_cap, int*
   if (grid) *grid = p.grid;
   if (workspace_bytes) *workspace_bytes = (int64_t)p.ws_bytes();
   return DG_OK;
+}
+
+int dg_debug_cluster_capacity(int block_n, int fp4, int cluster) {
+  if ((block_n != 128 && block_n != 256) || cluster < 2 || cluster > 8) return -1;
+  return split_capacity(block_n, fp4 != 0, cluster);
 }
 
 int dg_query_dense_cluster_split(int m, int n, int k, int64_t workspace_cap) {

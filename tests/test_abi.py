@@ -226,7 +226,7 @@ def test_workspace_cap_limits_the_plan(dg):
 
 def test_tile_config_override(dg):
     assert dg.lib().dg_set_tile_config(96, 0) == -1          # not an instantiated width
-    assert dg.lib().dg_set_tile_config(0, 7) == -1           # no such schedule
+    assert dg.lib().dg_set_tile_config(0, 11) == -1          # no such schedule
     assert dg.lib().dg_set_tile_config(0, -1) == -1
     dg.dg_set_num_sms(148)
     try:
@@ -241,6 +241,12 @@ def test_tile_config_override(dg):
     finally:
         dg.dg_set_tile_config(0, 0)
         dg.dg_set_num_sms(0)
+
+
+def test_cluster_capacity_query_rejects_bad_arguments(dg):
+    assert dg.dg_debug_cluster_capacity(192, 4) == -1
+    assert dg.dg_debug_cluster_capacity(128, 1) == -1
+    assert dg.dg_debug_cluster_capacity(256, 9) == -1
 
 
 def test_cluster_split_query_rejects_bad_sizes(dg):

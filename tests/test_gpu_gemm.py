@@ -151,7 +151,7 @@ def test_dense_shared_tail_is_deterministic_and_agrees_with_whole_tiles(dg):
         check_close(outs[sched][0], p.ref(), f"schedule {sched} vs oracle")
 
 
-@pytest.mark.parametrize("schedule,S", [(4, 2), (5, 4), (6, 8)])
+@pytest.mark.parametrize("schedule,S", [(4, 2), (5, 3), (6, 4), (7, 5), (10, 8)])
 @pytest.mark.parametrize("bn", [128, 256])
 @pytest.mark.parametrize("M,N,K,with_c,fp4", [
     (64, 2112, 7168, True, False),     # small M: the shape these plans are for
