@@ -605,12 +605,12 @@ def probe_tensor_peaks(dg, torch, kblocks=4096, reps=3):
     """TFLOP/s of the tensor pipe alone: the library's own tcgen05 loop (one
     CTA per SM, operands resident in shared memory, no global traffic), best
     of `reps` launches timed with CUDA events, for the block-scaled FP8 MMA
-    the GEMMs issue (also at N = 32 and 64: the cost of narrow tiles), the
+    the GEMMs issue (also at N = 32, 64 and 192: the cost of other widths), the
     plain FP8 MMA and bf16, at N = 128 and 256."""
     stream = torch.cuda.current_stream()
     out = {}
     for kind in ("fp8_block_scaled", "fp8_plain", "bf16"):
-        for bn in ((32, 64, 128, 256) if kind == "fp8_block_scaled" else (128, 256)):
+        for bn in ((32, 64, 128, 192, 256) if kind == "fp8_block_scaled" else (128, 256)):
             dg.dg_probe_mma_peak(kind, bn, 256)
             best = None
             for _ in range(reps):

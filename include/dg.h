@@ -429,7 +429,7 @@ dg_status dg_query_config(int layout, int fp4, int swiglu, int rows, int n, int 
                           int* block_n, int* grid, int64_t* units);
 
 /* Tensor-core throughput probe: one CTA per SM issues kblocks x 4
- * tcgen05 MMAs of M = 128, N = block_n (128 or 256; block-scaled e4m3 also 32 or 64), K = 32 (bf16: 16) from
+ * tcgen05 MMAs of M = 128, N = block_n (128 or 256; block-scaled e4m3 also 32, 64 or 192), K = 32 (bf16: 16) from
  * operand tiles held in shared memory, with no global-memory traffic, into a
  * TMEM accumulator.  Kinds:
  *   DG_PROBE_FP8_SCALED  kind::mxf8f6f4.block_scale, e4m3, UE8M0 scales (the

@@ -1124,7 +1124,7 @@ dg_status dg_query_config(int layout, int fp4, int swiglu, int rows, int n, int 
 }
 
 dg_status dg_probe_mma_peak(int kind, int block_n, int kblocks, void* stream) {
-  const bool narrow = (block_n == 32 || block_n == 64);
+  const bool narrow = (block_n == 32 || block_n == 64 || block_n == 192);
   if (kind < DG_PROBE_FP8_SCALED || kind > DG_PROBE_BF16 || (block_n != 128 && block_n != 256 && !narrow) ||
       (narrow && kind != DG_PROBE_FP8_SCALED) || kblocks <= 0 || kblocks > (1 << 22))
     return DG_ERR_INVALID_ARG;
@@ -1136,6 +1136,7 @@ dg_status dg_probe_mma_peak(int kind, int block_n, int kblocks, void* stream) {
       case 32: return launch_probe<dg::kProbeScaled, 32>(kblocks, grid, s);
       case 64: return launch_probe<dg::kProbeScaled, 64>(kblocks, grid, s);
       case 128: return launch_probe<dg::kProbeScaled, 128>(kblocks, grid, s);
+      case 192: return launch_probe<dg::kProbeScaled, 192>(kblocks, grid, s);
       default: return launch_probe<dg::kProbeScaled, 256>(kblocks, grid, s);
     }
   }
