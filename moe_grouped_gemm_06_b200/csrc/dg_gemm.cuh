@@ -373,9 +373,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   static_assert(LAYOUT != kKGrouped || MAJ == (kAMajorMN | kBMajorMN), "k-grouped: A and B MN-major");
   // D and C of the masked and k-grouped layouts are [groups][rows][n]
   constexpr bool kGroupRows = (LAYOUT == kMasked || LAYOUT == kKGrouped);
-  // full 32 x 32 output boxes leave through a TMA store of the staging box
-  // (true) or through coalesced 16-byte stores of the box read back (false)
-  constexpr bool kTmaStoreD = true;
   // split tiles: row pitch (floats) of a slice's partial sums in shared memory
   // (4 floats of padding put the rows of a warp's float4 stores in distinct banks)
   constexpr int kSplitPitch = BN + 4;
@@ -847,7 +844,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         DG_CHECK((smem_u32(stg) & 511) == 0 && stg >= s_epi && stg + 2048 <= s_epi + C::kEpiBytes &&
                      (col0 % 8) == 0 && r0 + 32 <= lim,
                  7);
-        if (kTmaStoreD && lane == 0) bulk_wait_group_read<0>();
+        if (lane == 0) bulk_wait_group_read<0>();
         __syncwarp();
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
@@ -855,25 +852,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4*>(stg + lane * 64 + pos * 16) =
               make_uint4(packed[4 * ch], packed[4 * ch + 1], packed[4 * ch + 2], packed[4 * ch + 3]);
         }
-        if constexpr (kTmaStoreD) {
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_3d(&tm_d, stg, col0, r0, kGroupRows ? g : 0);
-            bulk_commit_group();
-          }
-        } else {
-          // the box read back transposed: four lanes per 64-byte row, eight
-          // rows per coalesced 16-byte store
-          __syncwarp();
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int rw = 8 * i + (int)(lane >> 2), pc = (int)(lane & 3);
-            const uint4 v = *reinterpret_cast<const uint4*>(stg + rw * 64 + ((pc ^ ((rw >> 1) & 3)) * 16));
-            const long long gr = kGroupRows ? (long long)g * a.rows + r0 + rw : (long long)(r0 + rw);
-            if (col0 + 8 * pc < a.d_cols) *reinterpret_cast<uint4*>(a.d + gr * a.d_cols + col0 + 8 * pc) = v;
-          }
-          __syncwarp();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&tm_d, stg, col0, r0, kGroupRows ? g : 0);
+          bulk_commit_group();
         }
       } else if ((int)lane < vr &&
                  DG_CHECK((reinterpret_cast<uintptr_t>(a.d + grow * a.d_cols + col0) & 15) == 0 && row < lim, 2)) {

@@ -141,8 +141,8 @@ long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
 // main loop of the next, so a tile costs the slower of the two; at 256
 // columns the two buffers share 64 columns, so a tile's MMAs wait for the
 // first quarter of the previous tile's epilogue, and the rest of the
-// epilogue's cost per tile is inside per_tile (measured: 0.4 us less than
-// with one buffer).  Widths 160
+// epilogue's cost per tile is inside per_tile (3.1 us: forced 256-wide runs
+// of 4096 x 7168 x 16384 and 4096 x 32768 x 512).  Widths 160
 // and 224 re-base their scale words on the MMA-issuing thread, which costs
 // more than they gain; they are available through dg_set_tile_config but
 // never chosen automatically.
@@ -160,7 +160,7 @@ struct WidthCost {
 constexpr WidthCost kWidthCosts[] = {
     {64, 0.19, 1.5, 1.6, true, 0.21, 0.13},      {128, 0.2305, 1.9, 2.94, true, 0.264, 0.213},
     {160, 0.32, 2.4, 3.6, false, 0.33, 0.26},    {192, 0.368, 1.6, 3.97, true, 0.345, 0.284},
-    {224, 0.41, 3.0, 4.6, false, 0.36, 0.33},    {256, 0.4236, 3.9, 0.0, true, 0.343, 0.357},
+    {224, 0.41, 3.0, 4.6, false, 0.36, 0.33},    {256, 0.4236, 3.1, 0.0, true, 0.343, 0.357},
 };
 
 // Tile-configuration override (dg_set_tile_config; initial values from the
