@@ -844,12 +844,38 @@ def main():
             h2d += sum(hx[key].numel() * hx[key].element_size() for key in ("a", "sfa", "b", "sfb", "c"))
             d2h += hx["d"].numel() * hx["d"].element_size()
 
+        # Copies in, GEMM and copy out of each shape on three streams, ordered
+        # by events: the inputs of shape i+1 travel to the device while shape
+        # i computes and its D travels back (host-to-device and device-to-host
+        # copies use separate copy engines), as a client pipelining its calls
+        # would; a step's inputs are not overwritten before the previous
+        # step's GEMM of that shape has read them, nor its D before it is out.
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        ev = lambda: torch.cuda.Event()
+        done_prev = [None] * len(inputs)   # GEMM of shape i finished (last step)
+        out_prev = [None] * len(inputs)    # D of shape i copied out (last step)
+
         def e2e_step():
-            for x, hx in zip(inputs, host):
-                for key in ("a", "sfa", "b", "sfb", "c"):
-                    x[key].copy_(hx[key], non_blocking=True)
+            for i, (x, hx) in enumerate(zip(inputs, host)):
+                if done_prev[i] is not None:
+                    s_in.wait_event(done_prev[i])
+                with torch.cuda.stream(s_in):
+                    for key in ("a", "sfa", "b", "sfb", "c"):
+                        x[key].copy_(hx[key], non_blocking=True)
+                    arrived = ev()
+                    arrived.record(s_in)
+                stream.wait_event(arrived)
+                if out_prev[i] is not None:
+                    stream.wait_event(out_prev[i])
                 call(x)
-                hx["d"].copy_(x["d"], non_blocking=True)
+                done = ev()
+                done.record(stream)
+                s_out.wait_event(done)
+                with torch.cuda.stream(s_out):
+                    hx["d"].copy_(x["d"], non_blocking=True)
+                    out = ev()
+                    out.record(s_out)
+                done_prev[i], out_prev[i] = done, out
 
         e2e_step()
         torch.cuda.synchronize()
@@ -858,16 +884,18 @@ def main():
         if use_dist:
             dist.barrier()
         torch.cuda.synchronize()
-        e0.record(stream)
+        e0.record(s_in)
         for _ in range(e2e_steps):
             e2e_step()
-        e1.record(stream)
+        s_in.wait_stream(s_out)
+        e1.record(s_in)
         torch.cuda.synchronize()
         ems = e0.elapsed_time(e1) / e2e_steps
         ems_max = max_over_ranks(ems, use_dist, "cuda")
         e2e = {"value": round(whole_job_tflops(world, sweep_flops, ems_max), 2), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": round(ems_max, 3)}
+               "ms_per_step": round(ems_max, 3),
+               "pipeline": "per shape: H2D of the inputs, GEMM, D2H of D on three streams ordered by events"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
