@@ -42,6 +42,12 @@ constexpr int kBK = 128;           // K per pipeline stage (= one scale block)
 constexpr int kEpiWarps = 8;        // 4 TMEM sub-partitions x kEpiParts column parts
 constexpr int kEpiParts = kEpiWarps / 4;
 constexpr int kThreads = 64 + 32 * kEpiWarps;  // warp 0 TMA, warp 1 MMA, the rest epilogue
+// Blocks of tiles whose width is not a multiple of 64 carry one more warp
+// (index 2 + kEpiWarps), which re-bases their B scale words (Cfg::kRebase).
+template <int BN, bool BF16>
+__host__ __device__ constexpr int block_threads() {
+  return kThreads + ((BN % 64 != 0 && !BF16) ? 32 : 0);
+}
 constexpr int kEpiCols = 32;       // columns per epilogue store box
 constexpr int kTmemCols = 512;
 constexpr int kMaxMaskedGroups = 1024;
@@ -163,7 +169,8 @@ struct Cfg {
   static constexpr int kSfbChunks = (kMaxOffRows + BN + 127) / 128;  // 128-row scale chunks a tile can touch
   static constexpr bool kRebase = (BN % 64 != 0);
   static constexpr int kSfrChunks = (BN + 127) / 128;                // re-based chunks (tile rows only)
-  static constexpr int kSfrBytes = (kRebase && !BF16 && !PROMO) ? kSfrChunks * 512 : 0;
+  static constexpr bool kRebaseWarp = kRebase && !BF16 && !PROMO;   // see block_threads()
+  static constexpr int kSfrBytes = kRebaseWarp ? kSfrChunks * 512 : 0;
   // FP32 accumulator buffers in TMEM: three of 128 columns (BN = 128), two at
   // columns 0 and 256 (BN = 192), one (BN = 256); scale factors after them.
   // Promotion: four 128-column buffers of K-block partial sums, no scales.
@@ -181,6 +188,9 @@ struct Cfg {
   static constexpr int kStagesRaw = (kBudget - kEpiBytes - kMaskBytes - kBarBytes) / kStageBytes;
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
   static_assert(kStages >= 2, "stages");
+  // barriers: full, empty (and re-based, kRebaseWarp) per stage; 4 + 4 + 2 + 1
+  // accumulator ones; the TMEM address and the abort flag
+  static_assert(((kRebaseWarp ? 3 : 2) * kStages + 12) * 8 <= kBarBytes, "barrier bytes");
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kEpiBytes + kMaskBytes + kBarBytes;
   static constexpr uint32_t kColAcc = 0;
   static constexpr uint32_t kAccStride = OVL ? 192 : ((BN <= 128) ? 128 : 256);
@@ -356,7 +366,7 @@ struct WorkIter {
 // the MMA reads it through an MN-major descriptor (plain FP8 tiles of width
 // 128 or 256 only).
 template <int BN, bool FP4, int LAYOUT, int EPI = kEpiPlain, bool BF16 = false, int MAJ = kMajorK>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(block_threads<BN, BF16>(), 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a32,
                 const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_d,
                 const GemmArgs args) {
@@ -398,6 +408,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = bars + 2 * S + 10;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 * S + 11);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  uint64_t* rb = bars + 2 * S + 12;     // [S]: the re-base warp is done with the stage (kRebaseWarp)
+  constexpr int kBlockThreads = block_threads<BN, BF16>();
+  static_assert(kBlockThreads == kThreads + (C::kRebaseWarp ? 32 : 0), "re-base warp");
 
   const int warp = threadIdx.x / 32;
   const uint32_t lane = lane_id();
@@ -414,6 +427,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tempty[b], kEpiWarps);
     }
     for (int b = 0; b < 2; ++b) mbar_init(&tovl[b], kEpiWarps / 2);  // the warps of one column half
+    if constexpr (C::kRebaseWarp)
+      for (int s = 0; s < S; ++s) mbar_init(&rb[s], 1);
     mbar_init(drain, 1);
     *s_abort = 0;
     fence_mbar_init();
@@ -437,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (LAYOUT == kMasked) {
     // tiles per group, read from device memory (so the call stays
     // graph-capturable), then an exclusive prefix over the groups
-    for (int g = threadIdx.x; g < a.num_groups; g += kThreads) {
+    for (int g = threadIdx.x; g < a.num_groups; g += kBlockThreads) {
       int mm = __ldg(a.masked_m + g);
       if (mm < 0 || mm > a.rows) record_error(-5 /* DG_ERR_BAD_METADATA */);
       mm = min(max(mm, 0), a.rows);
@@ -453,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // K-blocks per group, read from device memory, then an exclusive prefix
     // (the first K-block of each group); K of a group must be a non-negative
     // multiple of 128 and the groups must fit in the K rows of A and B
-    for (int g = threadIdx.x; g < a.num_groups; g += kThreads) {
+    for (int g = threadIdx.x; g < a.num_groups; g += kBlockThreads) {
       int kk = __ldg(a.ks + g);
       if (kk < 0 || kk % kBK != 0) {
         record_error(-5 /* DG_ERR_BAD_METADATA */);
@@ -612,8 +627,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     // One lane waits on the barriers and issues every tcgen05 operation (a
     // warp-wide loop with per-K-block warp synchronisation measured 1.8x
-    // slower).  It also re-bases the B scale words when a tile starts an odd
-    // number of 32-row groups into its first scale chunk.
+    // slower).  Where the re-base warp exists it also waits for that warp's
+    // hand-over of each stage.
     if (kPromo && lane == 0) {
       // promotion: every K-block's four unscaled MMAs go to the next of the
       // rotating partial-sum buffers, which the epilogue scales and frees
@@ -708,30 +723,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool new_sfa = ((kb & 3) == 0) || kb == kb0;
           const bool new_sfb = FP4 || new_sfa;
           const uint8_t* sfb_src = s_sfb + stage * C::kSfbBytes;
-          uint8_t* sfb_reb = s_sfr + stage * C::kSfrBytes;
-          if (C::kRebase && rebase && new_sfb) {
-            // word w of line l of re-based chunk v = word (off + w) % 4 of line
-            // l of loaded chunk v + (off + w) / 4 (chunks past the loaded range
-            // only feed rows outside the tile)
-            for (int l = 0; l < 32; ++l) {
-              uint4 ld[C::kSfbChunks];
-#pragma unroll
-              for (int c = 0; c < C::kSfbChunks; ++c)
-                ld[c] = *reinterpret_cast<const uint4*>(sfb_src + c * 512 + l * 16);
-#pragma unroll
-              for (int v = 0; v < C::kSfrChunks; ++v) {
-                uint32_t w4[4];
-#pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                  const int j = off + w;
-                  const uint4 q4 = ld[min(v + (j >> 2), C::kSfbChunks - 1)];
-                  const int e = j & 3;
-                  w4[w] = e == 0 ? q4.x : (e == 1 ? q4.y : (e == 2 ? q4.z : q4.w));
-                }
-                *reinterpret_cast<uint4*>(sfb_reb + v * 512 + l * 16) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-              }
+          const uint8_t* sfb_reb = s_sfr + stage * C::kSfrBytes;
+          if constexpr (C::kRebaseWarp) {
+            if (!dg_wait(&rb[stage], phase, s_abort, limit)) {
+              ok = false;
+              break;
             }
-            fence_proxy_async_smem();
+            tc_fence_after();
           }
           if (new_sfa) tc_cp_32x128b_x4(sfa_t, sdesc_sf_32x16(s_sfa + stage * C::kSfaBytes));
           if (new_sfb) {
@@ -773,6 +771,67 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(drain);
       uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < limit) {
+      }
+    }
+  } else if (C::kRebaseWarp && warp == 2 + kEpiWarps) {
+    // ------------------------------------------------------------ scale re-base
+    // A tile that starts an odd number of 32-row groups into its first 128-row
+    // scale chunk reads its B scale words from a re-based copy (the MMA's
+    // scale-factor address must be an even TMEM column): word w of line l of
+    // re-based chunk v is word (off + w) % 4 of line l of loaded chunk
+    // v + (off + w) / 4 (chunks past the loaded range only feed rows outside
+    // the tile).  Lane l builds line l.  The warp walks every K-block of the
+    // MMA lane's sequence, waiting on each stage's fill in order (so no
+    // barrier phase is skipped) and handing the stage on through rb[], which
+    // the MMA lane waits on before it copies the scales: the re-base runs
+    // while the MMA lane is still working on earlier stages.
+    if constexpr (C::kRebaseWarp) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      WorkIter<LAYOUT> it(a, cta_id, num_ctas);
+      Unit u;
+      while (ok && it.next(a, s_prefix, num_units, u)) {
+        if (LAYOUT == kContig && !u.valid) continue;
+        if (LAYOUT == kKGrouped && u.kb0 == u.kb1) continue;
+        const int off = ((u.nb * BN) % 128) / 32;
+        const bool rebase = (off & 1) != 0;
+        for (int kb = u.kb0; kb < u.kb1; ++kb) {
+          // every lane waits (a lane's own acquire of the fill), and the warp
+          // leaves together if any lane gave up
+          const bool got = dg_wait(&full[stage], phase, s_abort, limit);
+          if (!__all_sync(0xffffffffu, got)) {
+            ok = false;
+            break;
+          }
+          const bool new_sfb = FP4 || ((kb & 3) == 0) || kb == u.kb0;
+          if (rebase && new_sfb) {
+            const uint8_t* src = s_sfb + stage * C::kSfbBytes + lane * 16;
+            uint8_t* dst = s_sfr + stage * C::kSfrBytes + lane * 16;
+            uint4 ld[C::kSfbChunks];
+#pragma unroll
+            for (int c = 0; c < C::kSfbChunks; ++c) ld[c] = *reinterpret_cast<const uint4*>(src + c * 512);
+#pragma unroll
+            for (int v = 0; v < C::kSfrChunks; ++v) {
+              uint32_t w4[4];
+#pragma unroll
+              for (int w = 0; w < 4; ++w) {
+                const int j = off + w;
+                const uint4 q4 = ld[min(v + (j >> 2), C::kSfbChunks - 1)];
+                const int e = j & 3;
+                w4[w] = e == 0 ? q4.x : (e == 1 ? q4.y : (e == 2 ? q4.z : q4.w));
+              }
+              *reinterpret_cast<uint4*>(dst + v * 512) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+            fence_proxy_async_smem();  // the copy is read by tcgen05.cp (async proxy)
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&rb[stage]);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
       }
     }
   } else {

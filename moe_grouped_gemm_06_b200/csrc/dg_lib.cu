@@ -160,7 +160,7 @@ struct WidthCost {
 constexpr WidthCost kWidthCosts[] = {
     {64, 0.19, 1.5, 1.6, true, 0.21, 0.13},      {128, 0.2305, 1.9, 2.94, true, 0.264, 0.213},
     {160, 0.32, 2.4, 3.6, false, 0.33, 0.26},    {192, 0.368, 1.6, 3.97, true, 0.345, 0.284},
-    {224, 0.41, 3.0, 4.6, false, 0.36, 0.33},    {256, 0.4236, 3.1, 0.0, true, 0.343, 0.357},
+    {224, 0.45, 3.0, 4.6, false, 0.36, 0.33},    {256, 0.4236, 3.1, 0.0, true, 0.343, 0.357},
 };
 
 // Tile-configuration override (dg_set_tile_config; initial values from the
@@ -375,7 +375,7 @@ dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& ta32, const CUte
       return DG_ERR_CUDA;
     attr_set_mask.fetch_or(bit);
   }
-  if (launch(kern, dim3(grid), dim3(dg::kThreads), C::kSmemBytes, s, cluster, ta, ta32, tb, td, args) !=
+  if (launch(kern, dim3(grid), dim3(dg::block_threads<BN, BF16>()), C::kSmemBytes, s, cluster, ta, ta32, tb, td, args) !=
       cudaSuccess)
     return DG_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -392,7 +392,7 @@ int split_capacity_of(int cluster) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess) return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cluster);
-  cfg.blockDim = dim3(dg::kThreads);
+  cfg.blockDim = dim3(dg::block_threads<BN, false>());
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cudaLaunchAttribute attr;
   attr.id = cudaLaunchAttributeClusterDimension;

@@ -105,7 +105,7 @@ def test_dense_matches_oracle(dg, M, N, K, with_c):
 
 @pytest.mark.parametrize("schedule", [2, 3])
 @pytest.mark.parametrize("sms", [0, 7])
-@pytest.mark.parametrize("bn", [64, 128, 192, 256])
+@pytest.mark.parametrize("bn", [64, 128, 160, 192, 224, 256])
 @pytest.mark.parametrize("M,N,K,with_c,fp4", [
     (1100, 520, 512, True, False),     # ragged M and N tails, 4 K-blocks
     (300, 1000, 1536, True, False),    # pieces that start and end inside tiles
