@@ -215,6 +215,35 @@ def test_grouped_forced_widths(dg, bn):
         dg.dg_set_tile_config(0, 0)
 
 
+@pytest.mark.parametrize("bn", [64, 160, 224])
+def test_grouped_fp4_forced_widths(dg, bn):
+    # FP8 x FP4 grouped calls at widths that start tiles 32 or 96 rows into a
+    # 128-row scale chunk: the B scale words change every K-block, so the
+    # re-base hands every stage over (160 / 224), in both grouped layouts
+    dg.dg_set_tile_config(bn, 1)
+    try:
+        N, K = 1000, 512
+        cs = _contiguous_case(2900 + bn, 3, 60, 200, N, K, fp4=True)
+        d = _run_contiguous(dg, cs, N, fp4=True)
+        ref = oracle.gemm_contiguous(cs["qa"], cs["ea"], cs["qb"], cs["eb"], cs["mi"], c=cs["c"], b_fp4=True)
+        valid = cs["mi"] >= 0
+        check_close(d[valid], ref[valid], f"contiguous fp4 bn={bn}")
+        G, max_m = 3, 256
+        mm = np.array([5, 256, 130], np.int32)
+        qa, ea, sfa, qb, eb, sfb = _masked_fp4_case(3000 + bn, G, max_m, N, K, mm)
+        dm = torch.full((G, max_m, N), SENTINEL, dtype=torch.int16, device="cuda")
+        dg.dg_m_grouped_fp8_fp4_gemm_nt_masked(dev(qa), dev(sfa), dev(qb), dev(sfb), dm, dev(mm), expected_m=128)
+        torch.cuda.synchronize()
+        refm = oracle.gemm_masked(qa, ea, qb, eb, mm, b_fp4=True)
+        ddm = bf16_dev_to_f64(dm)
+        for g in range(G):
+            check_close(ddm[g, :mm[g]], refm[g, :mm[g]], f"masked fp4 bn={bn} g={g}")
+            assert np.all(host(dm).view(np.uint16)[g, mm[g]:] == SENTINEL)
+        assert dg.dg_get_last_error() == 0
+    finally:
+        dg.dg_set_tile_config(0, 0)
+
+
 def test_dense_long_k_accumulation(dg):
     # K = 16384: 128 scaled K-blocks accumulated in FP32 inside TMEM
     p = Dense(2100, 128, 256, 16384, with_c=False).upload()
