@@ -67,8 +67,10 @@ def test_invalid_arguments_rejected_on_host(dg):
     assert lib.dg_fp8_gemm_nt(p(fake + 4), p(fake), p(fake), p(fake), None, p(fake), 128, 128, 128, None) == -1
     # negative M
     assert lib.dg_fp8_gemm_nt(p(fake), p(fake), p(fake), p(fake), None, p(fake), -1, 128, 128, None) == -1
-    # m == 0 is a no-op
+    # m == 0 is a no-op; n == 0 and k == 0 are invalid
     assert lib.dg_fp8_gemm_nt(p(fake), p(fake), p(fake), p(fake), None, p(fake), 0, 128, 128, None) == 0
+    assert lib.dg_fp8_gemm_nt(p(fake), p(fake), p(fake), p(fake), None, p(fake), 128, 0, 128, None) == -1
+    assert lib.dg_fp8_gemm_nt(p(fake), p(fake), p(fake), p(fake), None, p(fake), 128, 128, 0, None) == -1
     # contiguous: m_total must be a multiple of 128, groups > 0
     assert lib.dg_m_grouped_fp8_gemm_nt_contiguous(p(fake), p(fake), p(fake), p(fake), None, p(fake), p(fake),
                                                    100, 128, 128, 2, None) == -1

@@ -448,6 +448,24 @@ def _masked_fp4_case(seed, G, max_m, N, K, masked_m):
     return qa, ea, sfa, qb, eb, sfb
 
 
+def test_masked_at_the_group_limit(dg):
+    # 1024 groups (the most the device-side prefix holds), counts from 0 to
+    # max_m: valid rows against the oracle, every other row bit-exact
+    G, max_m, N, K = 1024, 16, 256, 256
+    mm = synth.rng(6100).integers(0, max_m + 1, size=G).astype(np.int32)
+    mm[:4] = [0, max_m, 1, 0]
+    qa, ea, sfa, qb, eb, sfb = _masked_case(6100, G, max_m, N, K, mm)
+    d = _run_masked(dg, G, max_m, N, qa, sfa, qb, sfb, mm, expected_m=8)
+    ref = oracle.gemm_masked(qa, ea, qb, eb, mm)
+    got = bf16_dev_to_f64(d)
+    sent = host(d).view(np.uint16)
+    for g in range(G):
+        if mm[g] > 0:
+            check_close(got[g, :mm[g]], ref[g, :mm[g]], f"masked G=1024 g={g}")
+        assert np.all(sent[g, mm[g]:] == SENTINEL)
+    assert dg.dg_get_last_error() == 0
+
+
 def test_masked_fp4_matches_oracle(dg):
     G, max_m, N, K = 3, 256, 384, 512
     mm = np.array([5, 256, 130], np.int32)
