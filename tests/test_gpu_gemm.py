@@ -95,6 +95,8 @@ def test_pack_sf_bit_exact(dg, rows, ng, row_div):
     (64, 2112, 7168, True),     # stream-K over all SMs (17 tiles)
     (3, 64, 256, True),         # tiny M
     (1, 136, 512, True),        # a single row (one partial 32-row store box)
+    (5, 8, 128, True),          # the smallest N and K: one tile, one K-block, 8 of its columns
+    (130, 8, 128, False),       # two m-blocks of an 8-column D, full 32-row boxes clipped to 8 columns
 ])
 def test_dense_matches_oracle(dg, M, N, K, with_c):
     p = Dense(2000 + M + N, M, N, K, with_c=with_c).upload()
@@ -446,6 +448,22 @@ def _masked_fp4_case(seed, G, max_m, N, K, masked_m):
     qa, ea, sfa, _, _, _ = _masked_case(seed, G, max_m, N, K, masked_m)
     qb, eb, sfb = quantize_groups_b(seed + 2000, G, N, K, fp4=True)
     return qa, ea, sfa, qb, eb, sfb
+
+
+def test_contiguous_all_padding_rows(dg):
+    # every row is padding (m_indices = -1): nothing to compute, no error,
+    # and D untouched
+    M, N, K, G = 256, 256, 256, 2
+    cs = _contiguous_case(6200, G, 60, 200, N, K)
+    mi = np.full(M, -1, np.int32)
+    d = torch.full((M, N), SENTINEL, dtype=torch.int16, device="cuda")
+    assert cs["M"] >= M
+    qa = np.ascontiguousarray(cs["qa"][:M])
+    sfa = oracle.pack_sf(np.full((M, K // 128), 127, np.uint8), M)
+    dg.dg_m_grouped_fp8_gemm_nt_contiguous(dev(qa), dev(sfa), dev(cs["qb"]), dev(cs["sfb"]), None, d, dev(mi))
+    torch.cuda.synchronize()
+    assert dg.dg_get_last_error() == 0
+    assert np.all(host(d).view(np.uint16) == SENTINEL)
 
 
 def test_masked_at_the_group_limit(dg):
