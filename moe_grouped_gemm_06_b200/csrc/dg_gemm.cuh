@@ -132,6 +132,7 @@ struct GemmArgs {
   int sfa_chunks, sfb_chunks;          // ceil(rows/128), ceil(n/128)
   long long sfa_group_words, sfb_group_words;
   int sfa_q, sfb_q;                    // packed groups along K
+  int c_prefetch;                      // L2 prefetch of the next unit's C (short K, wide tiles)
   int raster;                          // m-blocks per raster band
   FastDiv band_div;                    // division by raster * num_n_blocks (tiles per band)
   FastDiv group_div;                   // k-grouped: division by num_m_blocks * num_n_blocks
@@ -369,7 +370,7 @@ template <int BN, bool FP4, int LAYOUT, int EPI = kEpiPlain, bool BF16 = false, 
 __global__ void __launch_bounds__(block_threads<BN, BF16>(), 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a32,
                 const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_d,
-                const GemmArgs args) {
+                const __grid_constant__ CUtensorMap tm_c, const GemmArgs args) {
   static_assert(EPI == kEpiPlain || BN % (2 * kSwiGluBlock) == 0, "SwiGLU tiles hold whole block pairs");
   constexpr bool kPromo = (EPI == kEpiPromote);
   constexpr bool kOvl = (BN == 256 && EPI == kEpiPlain);
@@ -1061,6 +1062,18 @@ __global__ void __launch_bounds__(block_threads<BN, BF16>(), 1)
     while (has_un) {
       u = un;
       has_un = it.next(a, s_prefix, num_units, un);
+      if constexpr (!kPrefetchC && EPI == kEpiPlain && LAYOUT != kDenseSplit) {
+        // no register room for the next unit's C here (four chunks a warp):
+        // where a unit's K loop is too short to hide C's HBM latency, bring
+        // this warp's part of the next unit's C into L2 a whole unit ahead
+        if (lane == 0 && a.c_prefetch && a.c != nullptr && has_un && un.valid && un.slot < 0) {
+          const int rn = un.mb * kBM + q * 32;
+          const int cn = un.nb * BN + half * kCols;
+#pragma unroll
+          for (int j = 0; j < kChunks; ++j)
+            if (j < nch_w && cn + j * kEpiCols < a.n) tma_prefetch_3d(&tm_c, cn + j * kEpiCols, rn, kGroupRows ? un.g : 0);
+        }
+      }
       if (LAYOUT == kContig && !u.valid) continue;
       const int buf = local % C::kAccBufs;
       const uint32_t use = (uint32_t)(local / C::kAccBufs);

@@ -361,8 +361,15 @@ float* workspace(size_t bytes, cudaStream_t s) {
 
 // ------------------------------------------------------------ launches
 
+// The tensor maps of one call: A (128-row and 32-row boxes), B, D, and C in
+// D's boxes (for L2 prefetches of the next tile's C; a copy of D's map when
+// there is no C).
+struct Maps {
+  CUtensorMap a, a32, b, d, c;
+};
+
 template <int BN, bool FP4, int LAYOUT, int EPI = dg::kEpiPlain, bool BF16 = false, int MAJ = dg::kMajorK>
-dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& ta32, const CUtensorMap& tb, const CUtensorMap& td,
+dg_status launch_gemm(const Maps& mp,
                       const dg::GemmArgs& args, int grid, cudaStream_t s, int cluster = 1) {
   using C = dg::Cfg<BN, FP4, BF16, (LAYOUT == dg::kMasked || LAYOUT == dg::kKGrouped), EPI == dg::kEpiPromote>;
   auto kern = dg::gemm_kernel<BN, FP4, LAYOUT, EPI, BF16, MAJ>;
@@ -375,7 +382,8 @@ dg_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& ta32, const CUte
       return DG_ERR_CUDA;
     attr_set_mask.fetch_or(bit);
   }
-  if (launch(kern, dim3(grid), dim3(dg::block_threads<BN, BF16>()), C::kSmemBytes, s, cluster, ta, ta32, tb, td, args) !=
+  if (launch(kern, dim3(grid), dim3(dg::block_threads<BN, BF16>()), C::kSmemBytes, s, cluster, mp.a, mp.a32, mp.b, mp.d,
+             mp.c, args) !=
       cudaSuccess)
     return DG_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -426,24 +434,22 @@ int split_capacity(int bn, bool fp4, int cluster) {
 }
 
 template <bool FP4>
-dg_status dispatch_split(int bn, int split, const CUtensorMap& ta, const CUtensorMap& ta32, const CUtensorMap& tb,
-                         const CUtensorMap& td, const dg::GemmArgs& args, int grid, cudaStream_t s) {
+dg_status dispatch_split(int bn, int split, const Maps& mp, const dg::GemmArgs& args, int grid, cudaStream_t s) {
   switch (bn) {
-    case 128: return launch_gemm<128, FP4, dg::kDenseSplit>(ta, ta32, tb, td, args, grid, s, split);
-    case 256: return launch_gemm<256, FP4, dg::kDenseSplit>(ta, ta32, tb, td, args, grid, s, split);
+    case 128: return launch_gemm<128, FP4, dg::kDenseSplit>(mp, args, grid, s, split);
+    case 256: return launch_gemm<256, FP4, dg::kDenseSplit>(mp, args, grid, s, split);
     default: return DG_ERR_UNSUPPORTED;
   }
 }
 
 template <bool FP4, int LAYOUT, int EPI = dg::kEpiPlain, bool BF16 = false, int MAJ = dg::kMajorK>
-dg_status dispatch(int bn, const CUtensorMap& ta, const CUtensorMap& ta32, const CUtensorMap& tb,
-                   const CUtensorMap& td, const dg::GemmArgs& args, int grid, cudaStream_t s) {
+dg_status dispatch(int bn, const Maps& mp, const dg::GemmArgs& args, int grid, cudaStream_t s) {
   if constexpr (MAJ != dg::kMajorK) {
     // MN-major operands: FP8, plain epilogue, 128-wide column blocks
     static_assert(!FP4 && !BF16 && EPI == dg::kEpiPlain, "MN-major: FP8, plain epilogue");
     switch (bn) {
-      case 128: return launch_gemm<128, false, LAYOUT, EPI, false, MAJ>(ta, ta32, tb, td, args, grid, s);
-      case 256: return launch_gemm<256, false, LAYOUT, EPI, false, MAJ>(ta, ta32, tb, td, args, grid, s);
+      case 128: return launch_gemm<128, false, LAYOUT, EPI, false, MAJ>(mp, args, grid, s);
+      case 256: return launch_gemm<256, false, LAYOUT, EPI, false, MAJ>(mp, args, grid, s);
       default: return DG_ERR_UNSUPPORTED;
     }
   } else if constexpr (LAYOUT == dg::kKGrouped) {
@@ -451,32 +457,32 @@ dg_status dispatch(int bn, const CUtensorMap& ta, const CUtensorMap& ta32, const
   } else if constexpr (BF16) {
     // bf16: dense tiles of the widths the heuristic picks
     switch (bn) {
-      case 64: return launch_gemm<64, false, LAYOUT, EPI, true>(ta, ta32, tb, td, args, grid, s);
-      case 128: return launch_gemm<128, false, LAYOUT, EPI, true>(ta, ta32, tb, td, args, grid, s);
-      case 192: return launch_gemm<192, false, LAYOUT, EPI, true>(ta, ta32, tb, td, args, grid, s);
-      case 256: return launch_gemm<256, false, LAYOUT, EPI, true>(ta, ta32, tb, td, args, grid, s);
+      case 64: return launch_gemm<64, false, LAYOUT, EPI, true>(mp, args, grid, s);
+      case 128: return launch_gemm<128, false, LAYOUT, EPI, true>(mp, args, grid, s);
+      case 192: return launch_gemm<192, false, LAYOUT, EPI, true>(mp, args, grid, s);
+      case 256: return launch_gemm<256, false, LAYOUT, EPI, true>(mp, args, grid, s);
       default: return DG_ERR_UNSUPPORTED;
     }
   } else if constexpr (EPI == dg::kEpiPromote) {
     // per-K-block promotion: e4m3 A and B, 128-wide tiles
     static_assert(!FP4 && LAYOUT == dg::kDense, "promotion: dense e4m3");
     if (bn != 128) return DG_ERR_UNSUPPORTED;
-    return launch_gemm<128, false, LAYOUT, EPI>(ta, ta32, tb, td, args, grid, s);
+    return launch_gemm<128, false, LAYOUT, EPI>(mp, args, grid, s);
   } else if constexpr (EPI == dg::kEpiSwiGlu) {
     // SwiGLU tiles hold whole (64 gate, 64 up) row blocks: widths 128, 256
     switch (bn) {
-      case 128: return launch_gemm<128, FP4, LAYOUT, EPI>(ta, ta32, tb, td, args, grid, s);
-      case 256: return launch_gemm<256, FP4, LAYOUT, EPI>(ta, ta32, tb, td, args, grid, s);
+      case 128: return launch_gemm<128, FP4, LAYOUT, EPI>(mp, args, grid, s);
+      case 256: return launch_gemm<256, FP4, LAYOUT, EPI>(mp, args, grid, s);
       default: return DG_ERR_UNSUPPORTED;
     }
   } else {
     switch (bn) {
-      case 64: return launch_gemm<64, FP4, LAYOUT>(ta, ta32, tb, td, args, grid, s);
-      case 128: return launch_gemm<128, FP4, LAYOUT>(ta, ta32, tb, td, args, grid, s);
-      case 160: return launch_gemm<160, FP4, LAYOUT>(ta, ta32, tb, td, args, grid, s);
-      case 192: return launch_gemm<192, FP4, LAYOUT>(ta, ta32, tb, td, args, grid, s);
-      case 224: return launch_gemm<224, FP4, LAYOUT>(ta, ta32, tb, td, args, grid, s);
-      case 256: return launch_gemm<256, FP4, LAYOUT>(ta, ta32, tb, td, args, grid, s);
+      case 64: return launch_gemm<64, FP4, LAYOUT>(mp, args, grid, s);
+      case 128: return launch_gemm<128, FP4, LAYOUT>(mp, args, grid, s);
+      case 160: return launch_gemm<160, FP4, LAYOUT>(mp, args, grid, s);
+      case 192: return launch_gemm<192, FP4, LAYOUT>(mp, args, grid, s);
+      case 224: return launch_gemm<224, FP4, LAYOUT>(mp, args, grid, s);
+      case 256: return launch_gemm<256, FP4, LAYOUT>(mp, args, grid, s);
       default: return DG_ERR_UNSUPPORTED;
     }
   }
@@ -581,6 +587,11 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
   args.sfa_q = (int)ceil_div(p.k / 128, 4);
   args.sfb_q = FP4 ? p.k / 128 : args.sfa_q;
   args.sfa_group_words = (long long)args.sfa_q * args.sfa_chunks * 128;
+  // L2 prefetch of C a unit ahead, where the register prefetch is off (four
+  // 32-column chunks per epilogue warp) and a K loop of at most 16 K-blocks
+  // cannot hide C's HBM latency (measured: 4096 x 32768 x 512 140 -> 125 us;
+  // at K >= 7168 the prefetched lines only compete with A and B in L2, ~1%)
+  args.c_prefetch = (p.c != nullptr && p.k <= 2048) ? 1 : 0;
   args.sfb_group_words = (long long)args.sfb_q * args.sfb_chunks * 128;
   // tiles with fewer than 128 valid rows of A exist only for an M tail or in
   // the masked layout; elsewhere the producer skips the trimming arithmetic
@@ -608,7 +619,8 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
   const int gd = (LAYOUT == dg::kMasked || LAYOUT == dg::kKGrouped) ? p.groups : 1;
   const uint64_t k_ext = (uint64_t)std::max(p.k, 128);  // K rows of MN-major maps
   // ta32: the same A in boxes of 32 rows, for tiles with fewer valid rows
-  CUtensorMap ta, ta32, tb, td;
+  Maps mp;
+  CUtensorMap &ta = mp.a, &ta32 = mp.a32, &tb = mp.b, &td = mp.d;
   bool ok;
   if (BF16) {
     ok = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.a, p.k, p.rows, ga, (uint64_t)p.k * 2,
@@ -642,6 +654,12 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
                         128, plan.bn, CU_TENSOR_MAP_SWIZZLE_128B);
   ok = ok && make_map(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.d, args.d_cols, p.rows, gd, (uint64_t)args.d_cols * 2,
                       (uint64_t)p.rows * args.d_cols * 2, dg::kEpiCols, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+  // C [gd][rows][n] in the same boxes (read only by L2 prefetches)
+  if (p.c != nullptr)
+    ok = ok && make_map(&mp.c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.c, p.n, p.rows, gd, (uint64_t)p.n * 2,
+                        (uint64_t)p.rows * p.n * 2, dg::kEpiCols, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+  else
+    mp.c = td;
   if (!ok) return DG_ERR_CUDA;
 
   if (log_enabled())
@@ -655,10 +673,10 @@ dg_status run_gemm(const Problem& p, cudaStream_t s, float* fixed_ws = nullptr, 
   if constexpr (LAYOUT == dg::kDense && EPI == dg::kEpiPlain && !BF16 && MAJ == dg::kMajorK) {
     if (plan.split > 0) {
       args.split = plan.split;
-      return dispatch_split<FP4>(plan.bn, plan.split, ta, ta32, tb, td, args, plan.grid, s);
+      return dispatch_split<FP4>(plan.bn, plan.split, mp, args, plan.grid, s);
     }
   }
-  st = dispatch<FP4, LAYOUT, EPI, BF16, MAJ>(plan.bn, ta, ta32, tb, td, args, plan.grid, s);
+  st = dispatch<FP4, LAYOUT, EPI, BF16, MAJ>(plan.bn, mp, args, plan.grid, s);
   if (st != DG_OK || plan.sk_tiles == 0) return st;
 
   dg::SkReduceArgs r{};
